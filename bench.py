@@ -1,0 +1,389 @@
+"""Benchmark of the shared-experts-fused GLM4-MoE expert layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload prefill_bf16]
+
+One step = one pass of the whole layer (router -> permute -> grouped SwiGLU
+GEMMs -> combine) over one batch of the workload, inputs resident in HBM.
+Prints one JSON line (rank 0). For N > 1 (torchrun) every rank runs its own
+batch with its own copy of the weights (tokens are independent: weak scaling,
+no collective on the data path); the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from shared_routed_expert_b200 import MoELayer, _lib, build, synth  # noqa: E402
+
+METRIC = "fused MoE layer tokens/s and TFLOP/s or HBM GB/s vs B200 roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": FALLBACK_PEAKS["hbm_gbs"], "bf16_tflops": FALLBACK_PEAKS["bf16_tflops"],
+            "bf16_tflops_sustained": FALLBACK_PEAKS["bf16_tflops"], "source": "fallback"}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+class Dist:
+    def __init__(self, gpus: int):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            torch.cuda.set_device(self.local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", self.local))
+            self.pg = dist
+        self.device = torch.device("cuda", self.local)
+
+    def barrier(self):
+        if self.pg is not None:
+            self.pg.barrier()
+
+    def max(self, v: float) -> float:
+        if self.pg is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=self.device)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg is not None:
+            self.pg.barrier()
+            self.pg.destroy_process_group()
+
+
+# ------------------------------------------------------------------ clocks
+
+class Clocks:
+    """nvidia-smi sampling every 200 ms while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: str):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [c.strip() for c in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() in ("active", "1"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ timing
+
+def time_steps(fn, steps: int, warmup: int, dist: Dist, stream) -> float:
+    """Device time of `steps` back-to-back calls (ms), max over ranks."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    return dist.max(e0.elapsed_time(e1))
+
+
+KERNELS = ["route_logits", "route_topk", "permute_hist", "permute_scan", "permute_scatter",
+           "quant_rows", "gather", "gemm1_tc", "gemm2_tc", "gemm1_simt", "gemm2_simt", "combine"]
+
+
+def kernel_table(steps: int) -> dict:
+    tab = {}
+    total = 0.0
+    for k in KERNELS:
+        n, ms = _lib.moe_profile_read(k)
+        if n:
+            tab[k] = {"launches": n, "total_ms": ms, "ms_per_launch": ms / n}
+            total += ms
+    for k in tab:
+        tab[k]["share"] = tab[k]["total_ms"] / total if total > 0 else None
+    return tab
+
+
+def algorithmic(cfg, kernel: str, counts: np.ndarray | None):
+    """(bound, work per launch, unit) of one kernel launch for this workload."""
+    R, T, H, I, Er = cfg.rows, cfg.T, cfg.H, cfg.I, cfg.n_routed
+    wb = 1 if cfg.w_dtype == "e4m3" else (4 if cfg.w_dtype == "f32" else 2)
+    ab = 4 if cfg.act_dtype == "f32" else 2
+    touched = int((counts > 0).sum()) if counts is not None else cfg.n_experts
+    if kernel.startswith("gemm1"):
+        return "tensor", 2.0 * R * 2 * I * H, touched * 2 * I * H * wb + R * H * (1 if wb == 1 else ab) + R * I * ab
+    if kernel.startswith("gemm2"):
+        return "tensor", 2.0 * R * I * H, touched * H * I * wb + R * I * (1 if wb == 1 else ab) + R * H * ab
+    if kernel == "route_logits":
+        return "alu", 2.0 * T * Er * H, T * H * ab + Er * H * 4
+    if kernel == "combine":
+        return "hbm", None, R * H * ab + T * H * ab + R * 4 * 2
+    if kernel == "gather":
+        return "hbm", None, 2 * R * H * (1 if wb == 1 else ab)
+    return "hbm", None, None
+
+
+# ------------------------------------------------------------------ CPU oracle baseline
+
+def cpu_baseline(cfg, host_inputs: dict, seconds: float = 12.0):
+    import oracle
+    Ly = oracle.Layer(cfg, host_inputs)
+    cores = len(os.sched_getaffinity(0))
+    rng = np.random.default_rng(0)
+    n = max(1, cores)
+    tok = rng.choice(cfg.T, size=min(n, cfg.T), replace=False).astype(np.int32)
+    t0 = time.perf_counter()
+    r = Ly.forward(tokens=tok, n_threads=cores)
+    dt = time.perf_counter() - t0
+    done, used = len(tok), r["threads"]
+    # scale the sample up to roughly `seconds` of CPU work
+    more = int(min(cfg.T - len(tok), max(0, len(tok) * (seconds / max(dt, 1e-3) - 1.0))))
+    if more > 0:
+        tok2 = rng.choice(np.setdiff1d(np.arange(cfg.T), tok), size=more, replace=False).astype(np.int32)
+        t1 = time.perf_counter()
+        r = Ly.forward(tokens=tok2, n_threads=cores)
+        dt += time.perf_counter() - t1
+        done += more
+        used = max(used, r["threads"])
+    return {"value": done / dt, "unit": "tokens/s", "cores": used, "kind": "oracle",
+            "sample": f"{done} tokens of {cfg.name} (router + all {cfg.slots} slots each, fp64 C oracle), {dt:.1f} s"}
+
+
+def run_reference(args, dist: Dist):
+    """The reference arm: the CPU oracle as it stands, bounded sample per step."""
+    if dist.rank != 0:
+        return
+    import oracle
+    cfg = synth.CONFIGS[args.workload]
+    host = synth.to_host(synth.make_inputs(cfg, dist.device))
+    Ly = oracle.Layer(cfg, host)
+    cores = len(os.sched_getaffinity(0))
+    rng = np.random.default_rng(1)
+    per_step = max(1, cores)
+
+    def step():
+        tok = rng.choice(cfg.T, size=per_step, replace=False).astype(np.int32)
+        return Ly.forward(tokens=tok, n_threads=cores)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    used = 1
+    for _ in range(args.steps):
+        used = max(used, step()["threads"])
+    dt = time.perf_counter() - t0
+    value = per_step * args.steps / dt
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000.0 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": describe(cfg), "sample_tokens_per_step": per_step},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": used, "kind": "oracle",
+                             "sample": f"{per_step} random tokens of {cfg.name} per step"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def describe(cfg) -> str:
+    return (f"{cfg.name}: T={cfg.T} H={cfg.H} I={cfg.I} {cfg.n_routed} routed + shared as expert "
+            f"{cfg.shared_id}, top-{cfg.top_k} + shared slot, {cfg.w_dtype} weights, {cfg.act_dtype} "
+            f"activations, seed {cfg.seed}")
+
+
+# ------------------------------------------------------------------ main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="prefill_bf16", choices=list(synth.CONFIGS))
+    ap.add_argument("--ffn", default="auto", choices=["auto", "simt", "tcgen05"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    dist = Dist(args.gpus)
+    torch.cuda.set_device(dist.device)
+    if args.impl == "reference":
+        run_reference(args, dist)
+        dist.close()
+        return
+
+    build.build()
+    cfg = synth.CONFIGS[args.workload]
+    impl = {"auto": _lib.MOE_FFN_AUTO, "simt": _lib.MOE_FFN_SIMT, "tcgen05": _lib.MOE_FFN_TCGEN05}[args.ffn]
+    d = synth.make_inputs(cfg, dist.device)
+    stream = torch.cuda.current_stream(dist.device)
+    fused = MoELayer(cfg, d, fuse_shared=True, impl=impl)
+    out = torch.empty_like(d["x"])
+
+    # expert counts of this batch (for touched-expert bytes)
+    s = _lib.make_shape(cfg)
+    ids = torch.empty(cfg.T, cfg.slots, dtype=torch.int32, device=dist.device)
+    wts = torch.empty(cfg.T, cfg.slots, dtype=torch.float32, device=dist.device)
+    _lib.moe_route_topk(s, d["x"], d["router_w"], d["router_bias"], ids, wts, None, fused.ws)
+    counts = np.bincount(ids.cpu().numpy().ravel(), minlength=cfg.n_experts)
+
+    def step():
+        fused.forward(d["x"], out)
+
+    # timed region: device-resident inputs, per-kernel events on the launching stream
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    clocks = Clocks(vis.split(",")[dist.local] if vis else str(dist.local))
+    clocks.start()
+    _lib.moe_profile_reset()
+    n0 = _lib.moe_launch_count()
+    _lib.moe_profile_enable(True)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    _lib.moe_profile_reset()
+    n0 = _lib.moe_launch_count()
+    ms = time_steps(step, args.steps, 0, dist, stream)
+    launches = _lib.moe_launch_count() - n0
+    _lib.moe_profile_enable(False)
+    clk = clocks.stop()
+    tab = kernel_table(args.steps)
+    st = fused.status()
+    if st != _lib.MOE_OK:
+        raise SystemExit(f"layer reported {_lib.status_string(st)}")
+
+    # unfused GPU baseline (shared expert as its own dense pass), same process
+    unfused = MoELayer(cfg, d, fuse_shared=False, impl=impl)
+    ms_unf = time_steps(lambda: unfused.forward(d["x"], out), args.steps, args.warmup, dist, stream)
+    del unfused
+
+    # end to end through the public API with pinned host buffers
+    x_host = d["x"].cpu().pin_memory()
+    out_host = torch.empty_like(x_host).pin_memory()
+    x_dev = torch.empty_like(d["x"])
+    ms_e2e = time_steps(lambda: fused.forward_host(x_host, out_host, x_dev, out), args.steps,
+                        args.warmup, dist, stream)
+
+    N = dist.world
+    ms_step = ms / args.steps
+    value = N * cfg.T * args.steps / (ms / 1000.0)
+    pk = peaks()
+    flops = cfg.gemm_flops() + cfg.router_flops()
+    wb = 1 if cfg.w_dtype == "e4m3" else 2
+    alg_bytes = int((counts > 0).sum()) * 3 * cfg.H * cfg.I * wb + 2 * cfg.T * cfg.H * 2 + \
+        cfg.n_routed * cfg.H * 4
+    tensor_peak = pk["bf16_tflops"] * (2.0 if cfg.w_dtype == "e4m3" else 1.0)
+
+    roof = None
+    if tab:
+        top = max(tab, key=lambda k: tab[k]["total_ms"])
+        bound, fl, by = algorithmic(cfg, top, counts)
+        t_launch = tab[top]["ms_per_launch"] / 1000.0
+        if bound == "tensor":
+            ach = fl / t_launch / 1e12
+            roof = {"kernel": top, "bound": "tensor", "achieved": ach, "peak": tensor_peak,
+                    "unit": "TFLOP/s", "frac": ach / tensor_peak, "traffic": None,
+                    "peak_source": f"{pk['source']} bf16 burst" + (" x2 (E4M3 nominal ratio)" if wb == 1 else "")}
+        elif bound == "alu":
+            alu_peak = 148 * 128 * 2 * 1.965e9 / 1e12
+            ach = fl / t_launch / 1e12
+            roof = {"kernel": top, "bound": "alu", "achieved": ach, "peak": alu_peak, "unit": "TFLOP/s",
+                    "frac": ach / alu_peak, "traffic": None, "peak_source": "148 SM x 128 FP32 lanes x 2 x 1965 MHz"}
+        else:
+            ach = (by or 0) / t_launch / 1e9
+            roof = {"kernel": top, "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                    "frac": ach / pk["hbm_gbs"], "traffic": None, "peak_source": pk["source"]}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": N, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if cfg.w_dtype == "bf16" else cfg.w_dtype,
+        "data": "synthetic",
+        "config": {"workload": describe(cfg), "global_batch_tokens": N * cfg.T,
+                   "parallelism": f"replicas x{N} (tokens sharded, weights replicated)",
+                   "l2": "inputs larger than L2: every step streams the touched experts' weights "
+                         f"({alg_bytes / 1e9:.2f} GB) through the 126 MB L2",
+                   "ffn_impl": args.ffn},
+        "tflops": flops / (ms_step / 1000.0) / 1e12,
+        "tensor_frac": flops / (ms_step / 1000.0) / 1e12 / tensor_peak,
+        "hbm_gbs": alg_bytes / (ms_step / 1000.0) / 1e9,
+        "hbm_frac": alg_bytes / (ms_step / 1000.0) / 1e9 / pk["hbm_gbs"],
+        "unfused": {"value": N * cfg.T * args.steps / (ms_unf / 1000.0), "ms_per_step": ms_unf / args.steps,
+                    "fused_speedup": ms_unf / ms},
+        "e2e": {"value": N * cfg.T * args.steps / (ms_e2e / 1000.0), "unit": "tokens/s",
+                "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
+                "d2h_bytes_per_step": out_host.numel() * out_host.element_size()},
+        "gpu_launches": int(launches),
+        "roofline": roof,
+        "kernels": tab,
+        "clocks": clk,
+        "peaks": pk,
+    }
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, synth.to_host(d), args.cpu_seconds)
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.close()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,183 @@
+/*
+ * moe.h - C ABI of the shared-experts-fused MoE expert layer for B200 (sm_100a).
+ *
+ * The layer (GLM4-MoE expert layer, "Optimizing GLM4-MoE for production",
+ * Novita AI, section 1 "Shared Experts Fusion"): every token goes through one
+ * shared expert and through the top-k routed experts its router picks, and the
+ * expert outputs are aggregated with weights. The fusion appends the shared
+ * expert to the routed ones as expert number n_routed (160 for GLM-4.7) and
+ * gives every token top_k + 1 slots, the shared expert fixed in the last slot,
+ * so that one routed-MoE pass computes all of them.
+ *
+ * Conventions for every entry point
+ *  - Pointers named x, w13, ids, ... are DEVICE pointers; the caller owns every
+ *    buffer, including the workspace `ws`. The library never allocates device
+ *    memory and never synchronises except in moe_get_status.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Work is enqueued asynchronously on it; calls on one workspace must not
+ *    overlap on the GPU.
+ *  - Tensors are dense, row-major, with the shapes written in brackets.
+ *    bf16 tensors are passed as raw 16-bit patterns, E4M3 tensors as bytes
+ *    (OCP E4M3FN codes), fp32 as float.
+ *  - Errors found on the host (null or misaligned pointers, unsupported sizes or
+ *    dtypes, a workspace that is too small) return immediately with nothing
+ *    enqueued. Errors found on the device (an expert id out of range, a bounded
+ *    wait that ran out) are recorded in the workspace's status word and read
+ *    back by moe_get_status; kernels never trap.
+ *  - Device pointers must be 16-byte aligned; the workspace 256-byte aligned.
+ *  - Calls are thread-safe; no state is kept between calls except the optional
+ *    profiling and launch counters below.
+ */
+#ifndef SRE_MOE_H
+#define SRE_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum moe_status {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,   /* null/misaligned pointer or inconsistent shape */
+    MOE_ERR_UNSUPPORTED = 2,   /* sizes or dtype combination this build does not run */
+    MOE_ERR_WORKSPACE = 3,     /* ws_bytes smaller than moe_workspace_size() */
+    MOE_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed */
+    MOE_ERR_TIMEOUT = 5,       /* a kernel's bounded wait ran out (device-side) */
+    MOE_ERR_DEVICE = 6         /* bad data seen on the device (e.g. expert id out of range) */
+} moe_status;
+
+typedef enum moe_dtype { MOE_F32 = 0, MOE_BF16 = 1, MOE_E4M3 = 2 } moe_dtype;
+
+/* Shape and options of one layer call.
+ *   T            tokens
+ *   H            hidden size; multiple of 256 (router reduction order, tiles)
+ *   I            per-expert intermediate size; multiple of 64
+ *   n_routed     routed experts E_r (1..256)
+ *   top_k        routed experts per token K (1..min(n_routed, 32))
+ *   shared_id    n_routed: a shared expert is stored as expert n_routed (the
+ *                fused layout); -1: no shared expert
+ *   shared_weight  weight of the shared slot (1.0 reproduces the unfused sum)
+ *   renormalize  1: softmax over the K selected logits; 0: full softmax over
+ *                all n_routed logits evaluated at the selected ids
+ *   act_dtype    dtype of x, out and of the expert rows y: MOE_F32 or MOE_BF16
+ *   w_dtype      expert weight dtype: MOE_F32 (with act F32), MOE_BF16 or
+ *                MOE_E4M3 (both with act BF16)
+ * Derived: S = top_k + (shared_id >= 0) slots per token in the fused layout,
+ * E = n_routed + (shared_id >= 0) experts, R = T*S expert rows. */
+typedef struct moe_shape {
+    int32_t T, H, I, n_routed, top_k, shared_id;
+    float shared_weight;
+    int32_t renormalize;
+    int32_t act_dtype, w_dtype;
+} moe_shape;
+
+/* Kernel choice for the expert GEMMs. AUTO picks the tcgen05 tensor-core
+ * kernels for bf16/E4M3 weights and the CUDA-core kernels for fp32. */
+typedef enum moe_ffn_impl { MOE_FFN_AUTO = 0, MOE_FFN_SIMT = 1, MOE_FFN_TCGEN05 = 2 } moe_ffn_impl;
+
+/* Bytes of workspace moe_forward needs for this shape (fused or not). The
+ * other entry points need at most this much. Returns 0 for an invalid shape. */
+size_t moe_workspace_size(const moe_shape* shape, int fuse_shared);
+
+/* Router: logits, top-K selection and slot weights.
+ * Follows the write-up's section 1: each token's router picks its top-8 routed
+ * experts; with the fusion the shared expert takes the 9th slot.
+ *   x        [T, H] act_dtype       router_w [n_routed, H] fp32
+ *   router_bias [n_routed] fp32 or NULL (added to the logits before ranking)
+ *   ids      [T, S] int32 out: slots 0..K-1 = routed ids ranked by
+ *            (logit desc, id asc); slot K = shared_id when shared_id >= 0
+ *   weights  [T, S] fp32 out: softmax weights of the routed slots;
+ *            shared_weight in slot K
+ *   logits   [T, n_routed] fp32 out, or NULL. Logits are fp32 in a fixed order:
+ *            per 256-wide segment of H an fma chain from +0 over ascending h,
+ *            segment sums added in ascending order to a total starting at +0,
+ *            then the bias; so they are reproducible bit for bit.
+ * Needs moe_workspace_size(shape, 1) bytes of ws. */
+moe_status moe_route_topk(const moe_shape* shape, const void* x, const float* router_w,
+                          const float* router_bias, int32_t* ids, float* weights,
+                          float* logits, void* ws, size_t ws_bytes, void* stream);
+
+/* Sort the R = T*S slots by expert: the token permutation of "one routed-MoE
+ * pass" (section 1). Experts in id order; inside an expert, stable by flat slot
+ * index t*S + k, so the shared expert's block is tokens 0..T-1 in order.
+ *   ids      [T, S] int32 with values in [0, E); S = top_k + (shared_id >= 0)
+ *   counts   [E] int32 out     offsets [E + 1] int32 out (exclusive scan)
+ *   perm     [R] int32 out: perm[row] = flat slot index
+ *   inv      [R] int32 out: inv[flat] = row
+ * An id outside [0, E) sets MOE_ERR_DEVICE in the status word (that slot is
+ * dropped). */
+moe_status moe_permute(const moe_shape* shape, const int32_t* ids, int32_t* counts,
+                       int32_t* offsets, int32_t* perm, int32_t* inv, void* ws,
+                       size_t ws_bytes, void* stream);
+
+/* Expert FFNs for all R rows, grouped by expert (section 1: the shared and
+ * routed experts have identical tensor shapes and computation flow, so one
+ * grouped pass serves both). Row r belongs to expert e with
+ * offsets[e] <= r < offsets[e+1] and reads token perm[r] / S of x.
+ * Per row: h = silu(gate . v) * (up . v) (rounded to bf16 for bf16 layers),
+ * y = w2[e] . h. E4M3 layers quantise v per token and h per row to E4M3 with
+ * scale amax/448, and apply the weight scales per output channel.
+ *   x    [T, H] act_dtype
+ *   w13  [E, 2I, H] w_dtype: rows [0, I) gate, [I, 2I) up;  s13 [E, 2I] fp32 (E4M3 only, else NULL)
+ *   w2   [E, H, I]  w_dtype;                                  s2  [E, H]  fp32 (E4M3 only, else NULL)
+ *   y    [R, H] act_dtype out, rows in permuted order
+ * Needs moe_workspace_size(shape, 1) bytes of ws. */
+moe_status moe_grouped_ffn(const moe_shape* shape, const void* x, const int32_t* perm,
+                           const int32_t* offsets, const void* w13, const float* s13,
+                           const void* w2, const float* s2, void* y, void* ws,
+                           size_t ws_bytes, int ffn_impl, void* stream);
+
+/* Weighted aggregation of the expert outputs (section 1: "all expert outputs
+ * are aggregated with weights"):
+ *   out[t] = sum_{k<S} weights[t, k] * y[inv[t*S + k]], fp32, slot order,
+ *   rounded once to act_dtype.
+ *   y [R, H], inv [R], weights [T, S], out [T, H]. */
+moe_status moe_combine(const moe_shape* shape, const void* y, const int32_t* inv,
+                       const float* weights, void* out, void* stream);
+
+/* The whole layer. fuse_shared = 1: the fused top-(K+1) pass (route -> permute
+ * -> grouped FFN over all E experts -> combine). fuse_shared = 0: the unfused
+ * layer of the write-up's zh page, section 2.1 pseudocode: routed top-K pass
+ * plus a separate dense pass of the shared expert, added at the end (the GPU
+ * baseline the fusion is measured against; needs shared_id >= 0).
+ *   x [T, H], router_w [n_routed, H], router_bias [n_routed] or NULL,
+ *   w13 [E, 2I, H], s13, w2 [E, H, I], s2 as in moe_grouped_ffn, out [T, H].
+ * Needs moe_workspace_size(shape, fuse_shared) bytes of ws. */
+moe_status moe_forward(const moe_shape* shape, const void* x, const float* router_w,
+                       const float* router_bias, const void* w13, const float* s13,
+                       const void* w2, const float* s2, int fuse_shared, void* out,
+                       void* ws, size_t ws_bytes, int ffn_impl, void* stream);
+
+/* Per-row E4M3 quantisation used before each E4M3 GEMM: scale = amax/448 in
+ * fp32 (amax = 0 -> 1), codes = E4M3_rn_satfinite(v / scale) (fp32 divide).
+ *   in [rows, cols] bf16, codes [rows, cols] u8 out, scales [rows] fp32 out.
+ * cols must be a multiple of 8. */
+moe_status moe_quant_rows_e4m3(int32_t rows, int32_t cols, const void* in, uint8_t* codes,
+                               float* scales, void* stream);
+
+/* Synchronises `stream`, reads the workspace status word and clears it.
+ * Returns MOE_OK, MOE_ERR_DEVICE or MOE_ERR_TIMEOUT (or MOE_ERR_CUDA). */
+moe_status moe_get_status(void* ws, void* stream);
+
+/* Zero the workspace status word (asynchronously on stream). */
+moe_status moe_clear_status(void* ws, void* stream);
+
+const char* moe_status_string(moe_status s);
+
+/* Number of kernels this library has launched in this process. */
+uint64_t moe_launch_count(void);
+
+/* Optional per-kernel timing: while enabled, every launch is bracketed by CUDA
+ * events on its stream. moe_profile_read synchronises those events and returns,
+ * for kernel name `name`, the number of launches and their summed device time
+ * in milliseconds since the last moe_profile_reset. */
+void moe_profile_enable(int on);
+void moe_profile_reset(void);
+moe_status moe_profile_read(const char* name, int64_t* launches, double* total_ms);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SRE_MOE_H */

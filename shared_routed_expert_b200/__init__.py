@@ -1,0 +1,75 @@
+"""Shared-experts-fused GLM4-MoE expert layer for B200 (sm_100a).
+
+The layer: every token goes through one shared expert and through the top-k
+routed experts its router picks; the outputs are aggregated with weights. The
+fusion appends the shared expert to the routed ones (index n_routed) and gives
+every token top_k + 1 slots, the shared expert fixed in the last one, so one
+routed-MoE pass computes everything ("Optimizing GLM4-MoE for production",
+Novita AI, section 1 "Shared Experts Fusion").
+
+All compute runs in the CUDA library libsre_moe.so (C ABI in include/moe.h);
+this package only marshals arguments. PyTorch supplies device memory and streams.
+"""
+from __future__ import annotations
+
+import torch
+
+from ._lib import (MOE_BF16, MOE_E4M3, MOE_F32, MOE_FFN_AUTO, MOE_FFN_SIMT, MOE_FFN_TCGEN05,
+                   MoeError, alloc_workspace, make_shape, moe_clear_status, moe_combine,
+                   moe_forward, moe_get_status, moe_grouped_ffn, moe_launch_count, moe_permute,
+                   moe_profile_enable, moe_profile_read, moe_profile_reset, moe_quant_rows_e4m3,
+                   moe_route_topk, moe_shape, moe_workspace_size)
+
+__all__ = ["MoELayer", "moe_shape", "make_shape", "alloc_workspace", "moe_workspace_size",
+           "moe_route_topk", "moe_permute", "moe_grouped_ffn", "moe_combine", "moe_forward",
+           "moe_quant_rows_e4m3", "moe_get_status", "moe_clear_status", "moe_launch_count",
+           "moe_profile_enable", "moe_profile_reset", "moe_profile_read", "MoeError",
+           "MOE_F32", "MOE_BF16", "MOE_E4M3", "MOE_FFN_AUTO", "MOE_FFN_SIMT", "MOE_FFN_TCGEN05"]
+
+
+class MoELayer:
+    """One expert layer with its weights resident on a CUDA device.
+
+    weights: dict with router_w [E_r, H] fp32, router_bias [E_r] or None,
+    w13 [E, 2I, H], s13 [E, 2I] or None, w2 [E, H, I], s2 [E, H] or None, all
+    on the device. cfg: a LayerConfig-like object (T is the largest batch).
+    """
+
+    def __init__(self, cfg, weights: dict, fuse_shared: bool = True, impl: int = MOE_FFN_AUTO):
+        self.cfg = cfg
+        self.w = weights
+        self.fuse_shared = fuse_shared
+        self.impl = impl
+        self.device = weights["w13"].device
+        self.max_T = cfg.T
+        self.ws = alloc_workspace(make_shape(cfg), fuse_shared, device=self.device)
+        act = torch.bfloat16 if cfg.act_dtype == "bf16" else torch.float32
+        self.act_dtype = act
+
+    def forward(self, x: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        """x [T, H] on the device -> out [T, H] on the device (asynchronous)."""
+        T = x.shape[0]
+        if T > self.max_T:
+            raise ValueError(f"batch {T} exceeds the layer's maximum {self.max_T}")
+        if out is None:
+            out = torch.empty_like(x)
+        w = self.w
+        moe_forward(make_shape(self.cfg, T), x, w["router_w"], w.get("router_bias"), w["w13"],
+                    w.get("s13"), w["w2"], w.get("s2"), self.fuse_shared, out, self.ws,
+                    impl=self.impl, stream=stream)
+        return out
+
+    def forward_host(self, x_host: torch.Tensor, out_host: torch.Tensor, x_dev: torch.Tensor,
+                     out_dev: torch.Tensor, stream=None) -> torch.Tensor:
+        """Host buffers in and out: copy x to the device, run the layer, copy
+        the result back, all enqueued on `stream` (pinned host memory makes the
+        copies asynchronous)."""
+        s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        with torch.cuda.stream(s):
+            x_dev.copy_(x_host, non_blocking=True)
+            self.forward(x_dev, out_dev, stream=s)
+            out_host.copy_(out_dev, non_blocking=True)
+        return out_host
+
+    def status(self) -> int:
+        return moe_get_status(self.ws)

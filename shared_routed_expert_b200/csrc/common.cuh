@@ -1,0 +1,58 @@
+// Device helpers shared by the layer's kernels (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace sre {
+
+// Device status word layout at the start of the workspace.
+struct DevStatus {
+    unsigned int code;      // 0 ok, else a moe_status value
+    unsigned int info;      // first offending index / wait site
+    unsigned int timeouts;  // number of waits that ran out
+    unsigned int pad[61];
+};
+static_assert(sizeof(DevStatus) == 256, "status block is 256 bytes");
+
+__device__ __forceinline__ void report(DevStatus* st, unsigned code, unsigned info) {
+    if (st == nullptr) return;
+    if (atomicCAS(&st->code, 0u, code) == 0u) st->info = info;
+    if (code == MOE_ERR_TIMEOUT) atomicAdd(&st->timeouts, 1u);
+}
+
+__device__ __forceinline__ float bf16_to_f32(uint16_t b) {
+    return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+__device__ __forceinline__ uint16_t f32_to_bf16(float f) {
+    __nv_bfloat16 h = __float2bfloat16_rn(f);
+    return *reinterpret_cast<uint16_t*>(&h);
+}
+
+// two floats -> packed bf16x2 (low half = a)
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ float e4m3_to_f32(uint8_t c) {
+    __nv_fp8_e4m3 v;
+    v.__x = c;
+    return static_cast<float>(v);
+}
+
+// round to nearest even, saturate to +-448 (cvt.rn.satfinite)
+__device__ __forceinline__ uint8_t f32_to_e4m3(float f) {
+    return static_cast<uint8_t>(__nv_cvt_float_to_fp8(f, __NV_SATFINITE, __NV_E4M3));
+}
+
+__device__ __forceinline__ float silu_f32(float g) { return g / (1.0f + __expf(-g)); }
+
+__host__ __device__ constexpr int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+}  // namespace sre

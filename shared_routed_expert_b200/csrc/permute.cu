@@ -1,0 +1,221 @@
+// Token permutation for the single routed-MoE pass of the fused layer.
+//
+// "Optimizing GLM4-MoE for production" (Novita AI), section 1: the shared
+// expert joins the routed experts so that one routed-MoE pass computes all
+// top-(K+1) slots. That pass needs the R = T*S slots grouped by expert:
+// counts, exclusive offsets and a permutation, experts in id order and, inside
+// an expert, stable by flat slot index (so the result is deterministic and the
+// shared expert's block is tokens 0..T-1 in order).
+//
+// Three kernels, no atomics on the order-defining path:
+//   hist:    per 512-slot chunk, per-expert counts (shared-memory histogram)
+//   scan:    one block; per expert an ordered walk over chunks gives each
+//            chunk's base row; counts, offsets and the GEMM tile prefix
+//   scatter: one warp per chunk walks its slots in order, 32 at a time;
+//            __match_any_sync ranks equal experts inside a group.
+#include "kernels.cuh"
+
+namespace sre {
+
+namespace {
+
+__global__ void __launch_bounds__(256) perm_hist_kernel(const int32_t* __restrict__ ids, int R, int E,
+                                                        int32_t* __restrict__ chunk_hist,
+                                                        DevStatus* status) {
+    extern __shared__ int32_t hist[];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+    __syncthreads();
+    const int base = blockIdx.x * kPermChunk;
+    for (int i = threadIdx.x; i < kPermChunk; i += blockDim.x) {
+        const int f = base + i;
+        if (f >= R) break;
+        const int e = ids[f];
+        if (e < 0 || e >= E) {
+            report(status, MOE_ERR_DEVICE, static_cast<unsigned>(f));
+            continue;
+        }
+        atomicAdd(&hist[e], 1);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x)
+        chunk_hist[static_cast<size_t>(blockIdx.x) * E + e] = hist[e];
+}
+
+// single block, >= E threads (E <= 1024)
+__global__ void perm_scan_kernel(int n_chunks, int E, int32_t* __restrict__ chunk_hist,
+                                 int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                                 int32_t* __restrict__ tile_off) {
+    __shared__ int32_t s_cnt[1024];
+    __shared__ int32_t s_off[1025];
+    const int e = threadIdx.x;
+    int run = 0;
+    if (e < E) {
+        for (int c = 0; c < n_chunks; ++c) {
+            const size_t i = static_cast<size_t>(c) * E + e;
+            const int v = chunk_hist[i];
+            chunk_hist[i] = run;
+            run += v;
+        }
+        counts[e] = run;
+        s_cnt[e] = run;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int acc = 0, tacc = 0;
+        for (int j = 0; j < E; ++j) {
+            s_off[j] = acc;
+            offsets[j] = acc;
+            tile_off[j] = tacc;
+            acc += s_cnt[j];
+            tacc += ceil_div(s_cnt[j], kTileM);
+        }
+        s_off[E] = acc;
+        offsets[E] = acc;
+        tile_off[E] = tacc;
+    }
+    __syncthreads();
+    if (e < E) {
+        const int o = s_off[e];
+        for (int c = 0; c < n_chunks; ++c) chunk_hist[static_cast<size_t>(c) * E + e] += o;
+    }
+}
+
+// one warp per chunk
+__global__ void __launch_bounds__(32) perm_scatter_kernel(const int32_t* __restrict__ ids, int R, int E,
+                                                          const int32_t* __restrict__ chunk_base,
+                                                          int32_t* __restrict__ perm,
+                                                          int32_t* __restrict__ inv) {
+    extern __shared__ int32_t next[];
+    const int lane = threadIdx.x;
+    for (int e = lane; e < E; e += 32) next[e] = chunk_base[static_cast<size_t>(blockIdx.x) * E + e];
+    __syncwarp();
+    const int base = blockIdx.x * kPermChunk;
+    const unsigned lt = (1u << lane) - 1u;
+    for (int g = 0; g < kPermChunk; g += 32) {
+        const int f = base + g + lane;
+        int e = (f < R) ? ids[f] : -1;
+        if (e < 0 || e >= E) e = -1;
+        const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
+        int row = 0;
+        if (e >= 0) {
+            row = next[e] + __popc(peers & lt);
+            perm[row] = f;
+            inv[f] = row;
+        }
+        __syncwarp();
+        if (e >= 0 && (peers & lt) == 0) next[e] += __popc(peers);   // lowest lane of the group
+        __syncwarp();
+    }
+}
+
+// Xp[r] = x[perm[r] / S]: one warp per row, 16-byte vectors.
+__global__ void __launch_bounds__(256) gather_rows_kernel(int R, int S, int row_vecs,
+                                                          const uint4* __restrict__ x,
+                                                          const float* __restrict__ xscale,
+                                                          const int32_t* __restrict__ perm,
+                                                          uint4* __restrict__ xp,
+                                                          float* __restrict__ xpscale) {
+    const int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (r >= R) return;
+    const int f = perm[r];
+    if (f < 0 || f >= R) return;          // a slot dropped for a bad id leaves no row
+    const int t = f / S;
+    const uint4* src = x + static_cast<size_t>(t) * row_vecs;
+    uint4* dst = xp + static_cast<size_t>(r) * row_vecs;
+    for (int i = lane; i < row_vecs; i += 32) dst[i] = src[i];
+    if (xscale != nullptr && lane == 0) xpscale[r] = xscale[t];
+}
+
+// One warp per row: amax (fp32), scale = amax / 448 (IEEE divide, amax = 0 -> 1),
+// codes = E4M3_rn_satfinite(v / scale) (IEEE divide).
+__global__ void __launch_bounds__(256) quant_rows_kernel(int rows, int cols,
+                                                         const uint16_t* __restrict__ in,
+                                                         uint8_t* __restrict__ codes,
+                                                         float* __restrict__ scales) {
+    const int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (r >= rows) return;
+    const uint4* src = reinterpret_cast<const uint4*>(in + static_cast<size_t>(r) * cols);
+    const int nv = cols / 8;
+    float amax = 0.0f;
+    for (int i = lane; i < nv; i += 32) {
+        const uint4 q = src[i];
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            amax = fmaxf(amax, fabsf(__uint_as_float(w[j] << 16)));
+            amax = fmaxf(amax, fabsf(__uint_as_float(w[j] & 0xFFFF0000u)));
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+    const float scale = (amax > 0.0f) ? __fdiv_rn(amax, 448.0f) : 1.0f;
+    uint2* dst = reinterpret_cast<uint2*>(codes + static_cast<size_t>(r) * cols);
+    for (int i = lane; i < nv; i += 32) {
+        const uint4 q = src[i];
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+        uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t lo = f32_to_e4m3(__fdiv_rn(__uint_as_float(w[j] << 16), scale));
+            const uint32_t hi = f32_to_e4m3(__fdiv_rn(__uint_as_float(w[j] & 0xFFFF0000u), scale));
+            packed[j >> 1] |= (lo | (hi << 8)) << ((j & 1) * 16);
+        }
+        dst[i] = make_uint2(packed[0], packed[1]);
+    }
+    if (lane == 0) scales[r] = scale;
+}
+
+}  // namespace
+
+size_t permute_scratch_ints(int R, int E) {
+    return static_cast<size_t>(ceil_div(R, kPermChunk)) * E;
+}
+
+cudaError_t launch_permute(int R, int E, const int32_t* ids, int32_t* counts, int32_t* offsets,
+                           int32_t* perm, int32_t* inv, int32_t* tile_off, int32_t* scratch,
+                           DevStatus* st, cudaStream_t stream) {
+    const int n_chunks = ceil_div(R, kPermChunk);
+    const size_t hsm = static_cast<size_t>(E) * sizeof(int32_t);
+    if (n_chunks > 0) {
+        ProfileScope ps("permute_hist", stream);
+        perm_hist_kernel<<<n_chunks, 256, hsm, stream>>>(ids, R, E, scratch, st);
+        note_launch();
+    }
+    {
+        ProfileScope ps("permute_scan", stream);
+        perm_scan_kernel<<<1, ceil_div(E, 32) * 32, 0, stream>>>(n_chunks, E, scratch, counts,
+                                                                 offsets, tile_off);
+        note_launch();
+    }
+    if (n_chunks > 0) {
+        ProfileScope ps("permute_scatter", stream);
+        perm_scatter_kernel<<<n_chunks, 32, hsm, stream>>>(ids, R, E, scratch, perm, inv);
+        note_launch();
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather_rows(int R, int S, int H, int elem_bytes, const void* x,
+                               const float* xscale, const int32_t* perm, void* xp, float* xpscale,
+                               cudaStream_t stream) {
+    if (R == 0) return cudaSuccess;
+    const int row_vecs = H * elem_bytes / 16;
+    ProfileScope ps("gather", stream);
+    gather_rows_kernel<<<ceil_div(R * 32, 256), 256, 0, stream>>>(
+        R, S, row_vecs, static_cast<const uint4*>(x), xscale, perm, static_cast<uint4*>(xp), xpscale);
+    note_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quant_rows(int rows, int cols, const uint16_t* in, uint8_t* codes,
+                              float* scales, cudaStream_t stream) {
+    if (rows == 0) return cudaSuccess;
+    ProfileScope ps("quant_rows", stream);
+    quant_rows_kernel<<<ceil_div(rows * 32, 256), 256, 0, stream>>>(rows, cols, in, codes, scales);
+    note_launch();
+    return cudaGetLastError();
+}
+
+}  // namespace sre

@@ -1,0 +1,184 @@
+"""Per-kernel parity of the CUDA path against the CPU oracle, through the C ABI.
+
+Integer work (expert ids, counts, offsets, permutation, E4M3 codes) and the
+fixed-order fp32 router logits must match bit for bit; floating-point outputs
+within the stated tolerances."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from shared_routed_expert_b200 import _lib, build, synth
+from shared_routed_expert_b200._lib import MOE_FFN_SIMT, MOE_FFN_TCGEN05
+from tests.parity_util import oracle_logits, rel_err, to_f64, tol_of
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+ROUTE_CASES = {
+    "tiny_fp32": synth.CONFIGS["tiny_fp32"],
+    "bf16_ragged": synth.variant(synth.CONFIGS["prefill_bf16"], T=333, H=512, I=128, n_routed=40,
+                                 top_k=6),
+    "glm_router_T700": synth.variant(synth.CONFIGS["prefill_bf16"], T=700, I=64),
+    "decode_T1": synth.variant(synth.CONFIGS["decode_bf16"], T=1, I=64),
+    "zipf_bias": synth.variant(synth.CONFIGS["skewed_fp8"], T=257, I=64),
+    "no_renorm": synth.variant(synth.CONFIGS["prefill_bf16"], T=100, H=768, I=64, n_routed=33,
+                               top_k=5, renormalize=False),
+    "no_shared": synth.variant(synth.CONFIGS["prefill_bf16"], T=64, H=256, I=64, n_routed=256,
+                               top_k=32, shared=False),
+}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    build.build()
+
+
+def _route(cfg, inp):
+    s = _lib.make_shape(cfg)
+    ws = _lib.alloc_workspace(s, True)
+    ids = torch.empty(cfg.T, cfg.slots, dtype=torch.int32, device=DEV)
+    w = torch.empty(cfg.T, cfg.slots, dtype=torch.float32, device=DEV)
+    L = torch.empty(cfg.T, cfg.n_routed, dtype=torch.float32, device=DEV)
+    _lib.moe_route_topk(s, inp["x"], inp["router_w"], inp["router_bias"], ids, w, L, ws)
+    torch.cuda.synchronize()
+    return ids.cpu().numpy(), w.cpu().numpy(), L.cpu().numpy()
+
+
+@pytest.mark.parametrize("name", list(ROUTE_CASES))
+def test_route_topk_bit_exact(name):
+    cfg = ROUTE_CASES[name]
+    inp = synth.to_device(synth.make_inputs(cfg), DEV)
+    ids, w, L = _route(cfg, inp)
+    Lr = oracle_logits(inp["x"], inp["router_w"], inp["router_bias"])
+    assert np.array_equal(L.view(np.uint32), Lr.view(np.uint32)), "logits differ in some bit"
+    rid, rw = oracle.topk(Lr, cfg.top_k, cfg.renormalize, cfg.shared_id, cfg.shared_weight)
+    assert np.array_equal(ids, rid)
+    assert np.allclose(w, rw, rtol=2e-6, atol=1e-7)
+
+
+def test_route_zero_router_ties_to_lowest_ids():
+    cfg = synth.variant(synth.CONFIGS["prefill_bf16"], T=50, H=256, I=64, n_routed=160, top_k=8)
+    inp = synth.to_device(synth.make_inputs(cfg), DEV)
+    inp["router_w"].zero_()
+    ids, w, _ = _route(cfg, inp)
+    assert np.array_equal(ids, np.tile(np.r_[np.arange(8), 160], (50, 1)))
+    assert np.allclose(w[:, :8], 0.125) and np.all(w[:, 8] == 1.0)
+
+
+def _permute(cfg, ids_np):
+    s = _lib.make_shape(cfg)
+    ws = _lib.alloc_workspace(s, True)
+    E, R = cfg.n_experts, ids_np.size
+    ids = torch.from_numpy(np.ascontiguousarray(ids_np, np.int32)).to(DEV)
+    counts = torch.empty(E, dtype=torch.int32, device=DEV)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    perm = torch.full((R,), -7, dtype=torch.int32, device=DEV)
+    inv = torch.full((R,), -7, dtype=torch.int32, device=DEV)
+    _lib.moe_permute(s, ids, counts, offsets, perm, inv, ws)
+    st = _lib.moe_get_status(ws)
+    return [t.cpu().numpy() for t in (counts, offsets, perm, inv)], st
+
+
+@pytest.mark.parametrize("T,E_r,K", [(1, 8, 2), (333, 40, 6), (4096, 160, 8), (16384, 160, 8),
+                                     (70, 4, 4)])
+def test_permute_bit_exact(T, E_r, K):
+    cfg = synth.variant(synth.CONFIGS["prefill_bf16"], T=T, H=256, I=64, n_routed=E_r, top_k=K)
+    rng = np.random.default_rng(T)
+    routed = np.stack([rng.permutation(E_r)[:K] for _ in range(T)]).astype(np.int32)
+    ids = np.concatenate([routed, np.full((T, 1), E_r, np.int32)], 1)
+    (counts, offsets, perm, inv), st = _permute(cfg, ids)
+    assert st == _lib.MOE_OK
+    rc, ro, rp, ri = oracle.permute(ids, cfg.n_experts)
+    assert np.array_equal(counts, rc) and np.array_equal(offsets, ro)
+    assert np.array_equal(perm, rp) and np.array_equal(inv, ri)
+
+
+def test_permute_one_expert_holds_every_row_and_others_empty():
+    cfg = synth.variant(synth.CONFIGS["prefill_bf16"], T=1000, H=256, I=64, n_routed=8, top_k=1)
+    ids = np.concatenate([np.full((1000, 1), 3), np.full((1000, 1), 8)], 1).astype(np.int32)
+    (counts, offsets, perm, inv), st = _permute(cfg, ids)
+    rc, ro, rp, ri = oracle.permute(ids, 9)
+    assert st == _lib.MOE_OK
+    assert np.array_equal(counts, rc) and counts[3] == 1000 and counts[0] == 0
+    assert np.array_equal(perm, rp) and np.array_equal(inv, ri)
+
+
+def test_permute_flags_out_of_range_ids():
+    cfg = synth.variant(synth.CONFIGS["prefill_bf16"], T=40, H=256, I=64, n_routed=8, top_k=2)
+    ids = np.tile(np.array([[0, 1, 8]], np.int32), (40, 1))
+    ids[17, 1] = 9          # E = 9 experts: 9 is out of range
+    (counts, _, _, _), st = _permute(cfg, ids)
+    assert st == _lib.MOE_ERR_DEVICE
+    assert counts.sum() == ids.size - 1
+
+
+def test_quant_rows_e4m3_bit_exact():
+    g = torch.Generator().manual_seed(7)
+    rows = torch.randn(97, 1536, generator=g) * torch.logspace(-6, 6, 97).unsqueeze(1)
+    rows[5] = 0.0
+    rows[9, ::7] = 1e30          # saturates the amax scaling path cleanly
+    rows = rows.to(torch.bfloat16)
+    d = rows.to(DEV)
+    codes = torch.empty(97, 1536, dtype=torch.uint8, device=DEV)
+    scales = torch.empty(97, dtype=torch.float32, device=DEV)
+    _lib.moe_quant_rows_e4m3(97, 1536, d, codes, scales)
+    torch.cuda.synchronize()
+    rc, rs = oracle.quant_rows_e4m3(rows.float().numpy())
+    assert np.array_equal(scales.cpu().numpy().view(np.uint32), rs.view(np.uint32))
+    assert np.array_equal(codes.cpu().numpy(), rc)
+
+
+@pytest.mark.parametrize("act", ["bf16", "f32"])
+def test_combine_matches_oracle(act):
+    T, S, H = 77, 9, 512
+    g = torch.Generator().manual_seed(3)
+    Y = torch.randn(T * S, H, generator=g)
+    Y = Y.to(torch.bfloat16) if act == "bf16" else Y
+    inv = torch.randperm(T * S, generator=g).to(torch.int32)
+    w = torch.rand(T, S, generator=g)
+    cfg = synth.variant(synth.CONFIGS["prefill_bf16" if act == "bf16" else "tiny_fp32"], T=T, H=H,
+                        I=64, n_routed=8, top_k=S - 1)
+    s = _lib.make_shape(cfg)
+    out = torch.empty(T, H, dtype=Y.dtype, device=DEV)
+    _lib.moe_combine(s, Y.to(DEV), inv.to(DEV), w.to(DEV), out)
+    torch.cuda.synchronize()
+    ref = oracle.combine(Y.float().numpy(), inv.numpy(), w.double().numpy(), act)
+    # one rounding of the output on each side: at most one output ulp apart
+    assert rel_err(to_f64(out), ref) <= (2.0 ** -7 if act == "bf16" else 1e-6)
+
+
+FFN_CASES = {
+    "f32": synth.variant(synth.CONFIGS["tiny_fp32"], T=40, H=256, I=64, n_routed=8, top_k=2),
+    "bf16": synth.variant(synth.CONFIGS["prefill_bf16"], T=150, H=512, I=256, n_routed=12, top_k=3),
+    "e4m3": synth.variant(synth.CONFIGS["prefill_fp8"], T=150, H=512, I=256, n_routed=12, top_k=3),
+    "e4m3_i192": synth.variant(synth.CONFIGS["skewed_fp8"], T=150, H=512, I=192, n_routed=12, top_k=3),
+}
+
+
+@pytest.mark.parametrize("name", list(FFN_CASES))
+@pytest.mark.parametrize("impl", [MOE_FFN_SIMT, MOE_FFN_TCGEN05], ids=["simt", "tcgen05"])
+def test_grouped_ffn_rows_match_oracle(name, impl):
+    cfg = FFN_CASES[name]
+    if impl == MOE_FFN_TCGEN05 and cfg.w_dtype == "f32":
+        pytest.skip("tensor-core path is for bf16/E4M3 weights")
+    inp = synth.make_inputs(cfg)
+    d = synth.to_device(inp, DEV)
+    rng = np.random.default_rng(5)
+    # ragged groups: sizes 0, 1, 127, 128, 129 and the rest random
+    T, S, E = cfg.T, cfg.slots, cfg.n_experts
+    ids = np.stack([np.r_[rng.permutation(cfg.n_routed)[:cfg.top_k], cfg.shared_id] for _ in range(T)])
+    counts, offsets, perm, inv = oracle.permute(ids.astype(np.int32), E)
+    s = _lib.make_shape(cfg)
+    ws = _lib.alloc_workspace(s, True)
+    y = torch.empty(T * S, cfg.H, dtype=d["x"].dtype, device=DEV)
+    _lib.moe_grouped_ffn(s, d["x"], torch.from_numpy(perm).to(DEV), torch.from_numpy(offsets).to(DEV),
+                         d["w13"], d["s13"], d["w2"], d["s2"], y, ws, impl=impl)
+    torch.cuda.synchronize()
+    yg = to_f64(y)
+    Ly = oracle.Layer(cfg, inp)
+    xs = inp["x"].float().numpy()
+    rows = list(range(0, T * S, 7)) + [T * S - 1]
+    ref = np.stack([Ly.expert_ffn(int(ids.ravel()[perm[r]]), xs[perm[r] // S]) for r in rows])
+    assert rel_err(yg[rows], ref) <= tol_of(cfg)

@@ -1,0 +1,132 @@
+"""End-to-end parity of moe_forward (fused and unfused) against the CPU oracle.
+
+Small layers (several tiles plus ragged tails) are compared on every output;
+the full-size workloads - in the launch configuration the benchmark times -
+are compared on sampled tokens, with routing checked on every token."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from shared_routed_expert_b200 import MOE_FFN_AUTO, MOE_FFN_SIMT, MoELayer, _lib, build, synth
+from tests.parity_util import oracle_logits, rel_err, sample_tokens, to_f64, tol_of
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+SMALL = {
+    "tiny_fp32": synth.CONFIGS["tiny_fp32"],
+    "bf16_small": synth.variant(synth.CONFIGS["prefill_bf16"], T=200, H=512, I=256, n_routed=16, top_k=4),
+    "fp8_small": synth.variant(synth.CONFIGS["prefill_fp8"], T=200, H=512, I=256, n_routed=16, top_k=4),
+    "fp8_i192_zipf": synth.variant(synth.CONFIGS["skewed_fp8"], T=300, H=512, I=192, n_routed=24, top_k=4),
+    "decode_small": synth.variant(synth.CONFIGS["decode_bf16"], T=5, H=512, I=128, n_routed=16, top_k=4),
+    "single_token": synth.variant(synth.CONFIGS["prefill_bf16"], T=1, H=256, I=64, n_routed=8, top_k=2),
+    "all_experts": synth.variant(synth.CONFIGS["prefill_bf16"], T=64, H=256, I=64, n_routed=6, top_k=6),
+    "one_routed": synth.variant(synth.CONFIGS["prefill_bf16"], T=130, H=256, I=128, n_routed=1, top_k=1),
+    "shared_w_half": synth.variant(synth.CONFIGS["prefill_bf16"], T=50, H=256, I=64, n_routed=8,
+                                   top_k=2, shared_weight=0.5),
+    "no_renorm": synth.variant(synth.CONFIGS["prefill_bf16"], T=50, H=256, I=64, n_routed=8,
+                               top_k=2, renormalize=False),
+}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    build.build()
+
+
+def _run(cfg, d, fuse=True, impl=MOE_FFN_AUTO):
+    layer = MoELayer(cfg, d, fuse_shared=fuse, impl=impl)
+    out = layer.forward(d["x"])
+    st = layer.status()
+    assert st == _lib.MOE_OK, _lib.status_string(st)
+    return to_f64(out)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_forward_small_matches_oracle(name):
+    cfg = SMALL[name]
+    inp = synth.make_inputs(cfg)
+    d = synth.to_device(inp, DEV)
+    ref = oracle.Layer(cfg, inp).forward()
+    fused = _run(cfg, d, True)
+    assert rel_err(fused, ref["out_rnd"]) <= tol_of(cfg)
+    unfused = _run(cfg, d, False)
+    assert rel_err(unfused, ref["out_rnd"]) <= tol_of(cfg)
+    # fused and unfused GPU paths agree with each other as well
+    assert rel_err(fused, unfused) <= tol_of(cfg)
+
+
+@pytest.mark.parametrize("name", ["bf16_small", "fp8_small"])
+def test_forward_simt_and_tensor_core_paths_agree(name):
+    cfg = SMALL[name]
+    d = synth.to_device(synth.make_inputs(cfg), DEV)
+    assert rel_err(_run(cfg, d, True, MOE_FFN_SIMT), _run(cfg, d, True, MOE_FFN_AUTO)) <= tol_of(cfg)
+
+
+def test_zero_router_routes_everything_to_the_lowest_ids():
+    """All logits tie: every token takes experts 0..K-1 (one expert group holds
+    all T rows, the others are empty)."""
+    cfg = synth.variant(synth.CONFIGS["prefill_bf16"], T=300, H=256, I=128, n_routed=16, top_k=2)
+    inp = synth.make_inputs(cfg)
+    inp["router_w"].zero_()
+    ref = oracle.Layer(cfg, inp).forward()
+    assert np.all(ref["ids"][:, :2] == [0, 1])
+    got = _run(cfg, synth.to_device(inp, DEV))
+    assert rel_err(got, ref["out_rnd"]) <= tol_of(cfg)
+
+
+WORKLOADS = ["prefill_bf16", "decode_bf16", "prefill_fp8", "skewed_fp8"]
+
+
+@pytest.mark.parametrize("name", WORKLOADS)
+def test_full_size_workload(name):
+    """The benchmark's workloads at full size: routing of every token bit-exact,
+    outputs of sampled tokens within tolerance, properties on all tokens."""
+    cfg = synth.CONFIGS[name]
+    d = synth.make_inputs(cfg, DEV)
+    s = _lib.make_shape(cfg)
+    layer = MoELayer(cfg, d)
+    out = layer.forward(d["x"])
+    assert layer.status() == _lib.MOE_OK
+    # routing, every token: same kernels the layer runs, exposed through the ABI
+    ids = torch.empty(cfg.T, cfg.slots, dtype=torch.int32, device=DEV)
+    w = torch.empty(cfg.T, cfg.slots, dtype=torch.float32, device=DEV)
+    _lib.moe_route_topk(s, d["x"], d["router_w"], d["router_bias"], ids, w, None, layer.ws)
+    torch.cuda.synchronize()
+    Lr = oracle_logits(d["x"], d["router_w"], d["router_bias"])
+    rid, rw = oracle.topk(Lr, cfg.top_k, cfg.renormalize, cfg.shared_id, cfg.shared_weight)
+    assert np.array_equal(ids.cpu().numpy(), rid)
+    assert np.allclose(w.cpu().numpy(), rw, rtol=2e-6, atol=1e-7)
+    # outputs on sampled tokens
+    host = synth.to_host(d)
+    tok = sample_tokens(cfg.T, 6 if cfg.T > 1024 else 10)
+    ref = oracle.Layer(cfg, host).forward(tokens=tok)
+    got = to_f64(out)[tok]
+    assert np.all(np.isfinite(to_f64(out)))
+    assert rel_err(got, ref["out_rnd"]) <= tol_of(cfg)
+    del layer, d, host
+    torch.cuda.empty_cache()
+
+
+def test_fused_matches_unfused_full_size_decode():
+    cfg = synth.CONFIGS["decode_bf16"]
+    d = synth.make_inputs(cfg, DEV)
+    a = _run(cfg, d, True)
+    b = _run(cfg, d, False)
+    assert rel_err(a, b) <= tol_of(cfg)
+
+
+def test_launch_counter_and_profile():
+    cfg = SMALL["bf16_small"]
+    d = synth.to_device(synth.make_inputs(cfg), DEV)
+    layer = MoELayer(cfg, d)
+    n0 = _lib.moe_launch_count()
+    _lib.moe_profile_reset()
+    _lib.moe_profile_enable(True)
+    layer.forward(d["x"])
+    _lib.moe_profile_enable(False)
+    torch.cuda.synchronize()
+    assert _lib.moe_launch_count() - n0 >= 6
+    n, ms = _lib.moe_profile_read("combine")
+    assert n == 1 and ms > 0
