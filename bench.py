@@ -262,6 +262,10 @@ def main():
     ap.add_argument("--ffn", default="auto", choices=["auto", "simt", "tcgen05"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--quick", action="store_true",
+                    help="only the fused device-timed region (for ncu launch lists and captures)")
+    ap.add_argument("--tokens", type=int, default=None, help="override T (smaller profiling case)")
+    ap.add_argument("--routed", type=int, default=None, help="override the routed expert count")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -274,6 +278,9 @@ def main():
 
     build.build()
     cfg = synth.CONFIGS[args.workload]
+    if args.tokens is not None or args.routed is not None:
+        cfg = synth.variant(cfg, T=args.tokens or cfg.T, n_routed=args.routed or cfg.n_routed,
+                            name=f"{cfg.name}[T={args.tokens or cfg.T},E_r={args.routed or cfg.n_routed}]")
     impl = {"auto": _lib.MOE_FFN_AUTO, "simt": _lib.MOE_FFN_SIMT, "tcgen05": _lib.MOE_FFN_TCGEN05}[args.ffn]
     d = synth.make_inputs(cfg, dist.device)
     stream = torch.cuda.current_stream(dist.device)
@@ -311,17 +318,21 @@ def main():
     if st != _lib.MOE_OK:
         raise SystemExit(f"layer reported {_lib.status_string(st)}")
 
-    # unfused GPU baseline (shared expert as its own dense pass), same process
-    unfused = MoELayer(cfg, d, fuse_shared=False, impl=impl)
-    ms_unf = time_steps(lambda: unfused.forward(d["x"], out), args.steps, args.warmup, dist, stream)
-    del unfused
+    if args.quick:
+        ms_unf = ms_e2e = float("nan")
+        x_host = out_host = d["x"]
+    else:
+        # unfused GPU baseline (shared expert as its own dense pass), same process
+        unfused = MoELayer(cfg, d, fuse_shared=False, impl=impl)
+        ms_unf = time_steps(lambda: unfused.forward(d["x"], out), args.steps, args.warmup, dist, stream)
+        del unfused
 
-    # end to end through the public API with pinned host buffers
-    x_host = d["x"].cpu().pin_memory()
-    out_host = torch.empty_like(x_host).pin_memory()
-    x_dev = torch.empty_like(d["x"])
-    ms_e2e = time_steps(lambda: fused.forward_host(x_host, out_host, x_dev, out), args.steps,
-                        args.warmup, dist, stream)
+        # end to end through the public API with pinned host buffers
+        x_host = d["x"].cpu().pin_memory()
+        out_host = torch.empty_like(x_host).pin_memory()
+        x_dev = torch.empty_like(d["x"])
+        ms_e2e = time_steps(lambda: fused.forward_host(x_host, out_host, x_dev, out), args.steps,
+                            args.warmup, dist, stream)
 
     N = dist.world
     ms_step = ms / args.steps
@@ -378,7 +389,7 @@ def main():
         "clocks": clk,
         "peaks": pk,
     }
-    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline and not args.quick:
         line["cpu_baseline"] = cpu_baseline(cfg, synth.to_host(d), args.cpu_seconds)
     if dist.rank == 0:
         print(json.dumps(line), flush=True)

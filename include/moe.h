@@ -177,6 +177,13 @@ void moe_profile_enable(int on);
 void moe_profile_reset(void);
 moe_status moe_profile_read(const char* name, int64_t* launches, double* total_ms);
 
+/* Failure-injection hook for tests of the bounded waits: the next n_calls
+ * grouped-FFN passes on the tensor-core path run with a TMA producer that never
+ * issues its loads and a wait limit of about 10 ms, so their waits run out; the
+ * kernels then drain, free TMEM, return, and leave MOE_ERR_TIMEOUT in the status
+ * word (the outputs of those calls are garbage). No GPU fault is involved. */
+void moe_inject_wait_timeout(int n_calls);
+
 #ifdef __cplusplus
 }
 #endif

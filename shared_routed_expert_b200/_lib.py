@@ -20,7 +20,7 @@ DTYPES = {"f32": MOE_F32, "bf16": MOE_BF16, "e4m3": MOE_E4M3}
 EXPORTS = ("moe_workspace_size", "moe_route_topk", "moe_permute", "moe_grouped_ffn",
            "moe_combine", "moe_forward", "moe_quant_rows_e4m3", "moe_get_status",
            "moe_clear_status", "moe_status_string", "moe_launch_count", "moe_profile_enable",
-           "moe_profile_reset", "moe_profile_read")
+           "moe_profile_reset", "moe_profile_read", "moe_inject_wait_timeout")
 
 
 class MoeError(RuntimeError):
@@ -74,6 +74,8 @@ def lib() -> C.CDLL:
         L.moe_profile_reset.argtypes = []
         L.moe_profile_read.restype = i
         L.moe_profile_read.argtypes = [C.c_char_p, C.POINTER(C.c_int64), C.POINTER(C.c_double)]
+        L.moe_inject_wait_timeout.restype = None
+        L.moe_inject_wait_timeout.argtypes = [i]
         _lib = L
     return _lib
 
@@ -178,6 +180,10 @@ def moe_profile_enable(on: bool):
 
 def moe_profile_reset():
     lib().moe_profile_reset()
+
+
+def moe_inject_wait_timeout(n_calls: int):
+    lib().moe_inject_wait_timeout(int(n_calls))
 
 
 def moe_profile_read(name: str):

@@ -415,6 +415,8 @@ const char* moe_status_string(moe_status s) {
 
 uint64_t moe_launch_count(void) { return g_launches.load(); }
 
+void moe_inject_wait_timeout(int n_calls) { ffn_tc_inject_stall(n_calls > 0 ? n_calls : 0); }
+
 void moe_profile_enable(int on) { g_prof_on.store(on != 0); }
 
 void moe_profile_reset(void) {

@@ -1,6 +1,468 @@
-// Placeholder until the tcgen05 grouped GEMMs land.
+// Grouped SwiGLU expert FFN on the 5th-generation tensor cores (tcgen05).
+//
+// "Optimizing GLM4-MoE for production" (Novita AI), section 1: the shared
+// expert has the same tensor shapes and computation flow as the routed ones,
+// so it joins them as one more group of the same grouped GEMM (expert index
+// n_routed, rows = every token) and one pass computes all S slots.
+//
+// Two persistent kernels per layer, one CTA per SM:
+//   GEMM1: G = Xp[rows of e] . W13[e]^T; the epilogue applies SwiGLU
+//          h = silu(G_gate) * G_up and stores bf16 h [R, I]
+//   GEMM2: Y = h[rows of e] . W2[e]^T, stored bf16 [R, H]
+// E4M3 layers run kind::f8f6f4 with per-row activation scales and
+// per-output-channel weight scales applied in the epilogue (they factor out of
+// the K-sum).
+//
+// CTA layout (192 threads): warp 0 = TMA producer, warp 1 = TMEM allocator and
+// single-thread MMA issuer, warps 2-5 = epilogue (warp w reads TMEM lanes
+// 32*(w%4)..+31, i.e. rows of the 128-row tile). Stages hold 128 bytes of K per
+// row (64 bf16 or 128 E4M3 values) for a 128-row A tile and an N-row B tile,
+// written by TMA with the 128-byte swizzle. Two TMEM accumulators (columns 0
+// and 256) let the epilogue of one tile overlap the MMAs of the next.
+//
+// Tiles are ordered expert-major, then n-tile, then m-tile, so CTAs running at
+// the same time share each weight tile through L2. An m-tile never straddles
+// two experts: rows past the expert's end are computed on whatever TMA loads
+// there (zero past R) and masked at the store.
+//
+// Every mbarrier wait is bounded; a wait that runs out raises an abort flag
+// that makes the other roles leave their loops, records MOE_ERR_TIMEOUT in the
+// status word, drains the copies and MMAs in flight and frees TMEM.
+#include <cuda.h>
+
+#include <atomic>
+#include <mutex>
+
 #include "kernels.cuh"
+#include "tc_ptx.cuh"
+
 namespace sre {
-bool ffn_tc_supported(const FfnArgs&) { return false; }
-cudaError_t launch_ffn_tc(const FfnArgs&, cudaStream_t) { return cudaErrorNotSupported; }
+
+namespace {
+
+constexpr int TC_BM = 128;
+constexpr int TC_STAGES = 4;
+constexpr int TC_THREADS = 192;
+constexpr int TC_ROWB = 128;                       // bytes of K per row per stage
+constexpr int TC_ABYTES = TC_BM * TC_ROWB;         // 16 KB
+constexpr int TC_MAXE = 260;
+constexpr uint32_t TC_TMEM_COLS = 512;
+
+struct TcParams {
+    int E, H, I;
+    int n_tiles_n;          // n-tiles per m-tile
+    int bn_out;             // output columns per n-tile (GEMM1: I columns; GEMM2: H columns)
+    int k_blocks;           // K / (128 bytes per row)
+    const int32_t* offsets; // [E+1]
+    const int32_t* tile_off;// [E+1]
+    uint16_t* out;          // GEMM1: h [R, I]; GEMM2: y [R, H] (bf16)
+    int out_ld;
+    const float* row_scale; // E4M3: per-row activation scale [R]
+    const float* col_scale; // E4M3: per-output-channel weight scale (s13 [E, 2I] or s2 [E, H])
+    DevStatus* status;
+    long long wait_limit;   // SM clock cycles per wait
+    int inject_stall;       // testing hook: the producer never issues its loads
+};
+
+struct TileInfo {
+    int e, row0, row_end, n0;
+};
+
+__device__ __forceinline__ TileInfo decode_tile(int id, const int* s_tile, const int* s_off, int E, int NT,
+                                                int bn_out) {
+    int lo = 0, hi = E - 1;   // largest e with s_tile[e] * NT <= id
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_tile[mid] * NT <= id) lo = mid; else hi = mid - 1;
+    }
+    const int e = lo;
+    const int mte = s_tile[e + 1] - s_tile[e];
+    const int local = id - s_tile[e] * NT;
+    const int nt = local / mte;
+    const int mt = local - nt * mte;
+    TileInfo t;
+    t.e = e;
+    t.row0 = s_off[e] + mt * TC_BM;
+    t.row_end = s_off[e + 1];
+    t.n0 = nt * bn_out;
+    return t;
+}
+
+// kBN: MMA N (GEMM1: gate half + up half; GEMM2: 256 output columns)
+template <bool kFp8, bool kGemm1, int kBN>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const TcParams p) {
+    constexpr int BBYTES = kBN * TC_ROWB;
+    constexpr int STAGE_TX = TC_ABYTES + BBYTES;
+    constexpr int HALF = kBN / 2;
+    constexpr int KEL = kFp8 ? 128 : 64;            // K elements per stage
+    constexpr uint32_t IDESC = ptx::instr_desc(TC_BM, kBN, kFp8 ? 0u : 1u);
+
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint64_t full_bar[TC_STAGES], empty_bar[TC_STAGES], tfull_bar[2], tempty_bar[2], drain_bar;
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_abort;
+    __shared__ int s_off[TC_MAXE], s_tile[TC_MAXE];
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t raw = ptx::smem_u32(smem_raw);
+    uint8_t* base = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+    uint8_t* sA = base;
+    uint8_t* sB = base + TC_STAGES * TC_ABYTES;
+    volatile int* abort_flag = &s_abort;
+
+    for (int i = threadIdx.x; i <= p.E; i += blockDim.x) {
+        s_off[i] = p.offsets[i];
+        s_tile[i] = p.tile_off[i];
+    }
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < TC_STAGES; ++s) {
+            ptx::mbar_init(&full_bar[s], 1);
+            ptx::mbar_init(&empty_bar[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(&tfull_bar[b], 1);
+            ptx::mbar_init(&tempty_bar[b], 128);
+        }
+        ptx::mbar_init(&drain_bar, 1);
+        s_abort = 0;
+        ptx::fence_mbar_init();
+        ptx::prefetch_tmap(&tmA);
+        ptx::prefetch_tmap(&tmB);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(&s_tmem, TC_TMEM_COLS);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = s_tmem;
+    const int total = s_tile[p.E] * p.n_tiles_n;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- producer
+        if (lane == 0 && !p.inject_stall) {
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+                const TileInfo t = decode_tile(tile, s_tile, s_off, p.E, p.n_tiles_n, p.bn_out);
+                bool ok = true;
+                for (int kb = 0; kb < p.k_blocks; ++kb) {
+                    if (!ptx::mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, p.wait_limit, p.status, 1u)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::mbar_arrive_expect_tx(&full_bar[stage], STAGE_TX);
+                    const int kx = kb * KEL;
+                    ptx::tma_load_2d(sA + stage * TC_ABYTES, &tmA, &full_bar[stage], kx, t.row0);
+                    if constexpr (kGemm1) {
+                        ptx::tma_load_3d(sB + stage * BBYTES, &tmB, &full_bar[stage], kx, t.n0, 2 * t.e);
+                        ptx::tma_load_3d(sB + stage * BBYTES + HALF * TC_ROWB, &tmB, &full_bar[stage], kx, t.n0,
+                                         2 * t.e + 1);
+                    } else {
+                        ptx::tma_load_2d(sB + stage * BBYTES, &tmB, &full_bar[stage], kx, t.e * p.H + t.n0);
+                    }
+                    if (++stage == TC_STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+            }
+            if (*abort_flag) {
+                // let every copy in flight land before the CTA can exit: each
+                // stage's last armed phase completes when its bytes arrive
+                for (int s = 0; s < TC_STAGES; ++s) {
+                    // stages below `stage` were armed in the current round (phase),
+                    // the others in the previous one (phase ^ 1) if ever
+                    const uint32_t par = (s < stage) ? phase : (phase ^ 1u);
+                    const long long t0 = clock64();
+                    while (!ptx::mbar_try_wait(&full_bar[s], par) && clock64() - t0 < p.wait_limit) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+                if (!ptx::mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, abort_flag, p.wait_limit, p.status, 2u)) break;
+                ptx::tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * 256);
+                bool ok = true;
+                for (int kb = 0; kb < p.k_blocks; ++kb) {
+                    if (!ptx::mbar_wait(&full_bar[stage], phase, abort_flag, p.wait_limit, p.status, 3u)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    const uint32_t a_addr = ptx::smem_u32(sA + stage * TC_ABYTES);
+                    const uint32_t b_addr = ptx::smem_u32(sB + stage * BBYTES);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint64_t ad = ptx::smem_desc_sw128(a_addr + k * 32);
+                        const uint64_t bd = ptx::smem_desc_sw128(b_addr + k * 32);
+                        if constexpr (kFp8) ptx::mma_f8(d_tmem, ad, bd, IDESC, (kb | k) != 0);
+                        else ptx::mma_f16(d_tmem, ad, bd, IDESC, (kb | k) != 0);
+                    }
+                    ptx::mma_commit(&empty_bar[stage]);
+                    if (++stage == TC_STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                ptx::mma_commit(&tfull_bar[acc]);
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
+            }
+            // every MMA this thread issued has finished before TMEM is freed
+            ptx::mma_commit(&drain_bar);
+            const long long t0 = clock64();
+            while (!ptx::mbar_try_wait(&drain_bar, 0) && clock64() - t0 < p.wait_limit) {
+            }
+        }
+    } else {
+        // ---------------------------------------------------------------- epilogue
+        const int sub = warp & 3;
+        const int r_local = sub * 32 + lane;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            const TileInfo t = decode_tile(tile, s_tile, s_off, p.E, p.n_tiles_n, p.bn_out);
+            // one lane waits, the warp follows its verdict: tcgen05.ld below needs the whole warp
+            int ok = 0;
+            if (lane == 0) ok = ptx::mbar_wait(&tfull_bar[acc], acc_phase, abort_flag, p.wait_limit, p.status, 4u);
+            ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            const int row = t.row0 + r_local;
+            const bool valid = row < t.row_end;
+            const uint32_t tb = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + static_cast<uint32_t>(acc * 256);
+            const float rs = (kFp8 && valid) ? p.row_scale[row] : 1.0f;
+            uint16_t* orow = p.out + static_cast<size_t>(valid ? row : 0) * p.out_ld + t.n0;
+            if constexpr (kGemm1) {
+#pragma unroll 1
+                for (int c = 0; c < HALF / 32; ++c) {
+                    uint32_t g[32], u[32];
+                    ptx::tmem_ld_32x32b_x32(tb + c * 32, g);
+                    ptx::tmem_ld_32x32b_x32(tb + HALF + c * 32, u);
+                    ptx::tmem_ld_wait(g);
+                    ptx::tmem_ld_wait(u);
+                    if (valid) {
+                        const float* sg = kFp8 ? p.col_scale + static_cast<size_t>(t.e) * 2 * p.I + t.n0 + c * 32 : nullptr;
+                        const float* su = kFp8 ? sg + p.I : nullptr;
+                        uint32_t packed[16];
+#pragma unroll
+                        for (int j = 0; j < 32; j += 2) {
+                            float g0 = __uint_as_float(g[j]), g1 = __uint_as_float(g[j + 1]);
+                            float u0 = __uint_as_float(u[j]), u1 = __uint_as_float(u[j + 1]);
+                            if constexpr (kFp8) {
+                                g0 = g0 * rs * sg[j];
+                                g1 = g1 * rs * sg[j + 1];
+                                u0 = u0 * rs * su[j];
+                                u1 = u1 * rs * su[j + 1];
+                            }
+                            packed[j >> 1] = pack_bf16x2(silu_f32(g0) * u0, silu_f32(g1) * u1);
+                        }
+                        uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+                    }
+                }
+            } else {
+#pragma unroll 1
+                for (int c = 0; c < kBN / 32; ++c) {
+                    uint32_t v[32];
+                    ptx::tmem_ld_32x32b_x32(tb + c * 32, v);
+                    ptx::tmem_ld_wait(v);
+                    if (valid) {
+                        const float* sc = kFp8 ? p.col_scale + static_cast<size_t>(t.e) * p.H + t.n0 + c * 32 : nullptr;
+                        uint32_t packed[16];
+#pragma unroll
+                        for (int j = 0; j < 32; j += 2) {
+                            float a0 = __uint_as_float(v[j]), a1 = __uint_as_float(v[j + 1]);
+                            if constexpr (kFp8) {
+                                a0 = a0 * rs * sc[j];
+                                a1 = a1 * rs * sc[j + 1];
+                            }
+                            packed[j >> 1] = pack_bf16x2(a0, a1);
+                        }
+                        uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+                    }
+                }
+            }
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(&tempty_bar[acc]);
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1u;
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem_base, TC_TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------ host side
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return static_cast<EncodeTiledFn>(nullptr);
+        return reinterpret_cast<EncodeTiledFn>(ptr);
+    }();
+    return fn;
+}
+
+// rank-2/3 K-major map with a {128 bytes of K, box_rows[, 1]} box and 128-byte swizzle
+bool make_map(CUtensorMap* m, const void* ptr, bool fp8, int rank, const cuuint64_t* dims,
+              const cuuint64_t* strides_bytes, cuuint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return false;
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(fp8 ? 128 : 64), box_rows, 1};
+    const cuuint32_t es[3] = {1, 1, 1};
+    const CUresult r = fn(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                          static_cast<cuuint32_t>(rank), const_cast<void*>(ptr), dims, strides_bytes, box, es,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int num_sms() {
+    int dev = 0, n = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+int gemm1_half(int I) {
+    if (I % 128 == 0) return 128;
+    if (I % 96 == 0) return 96;
+    return 64;
+}
+
+std::atomic<int> g_inject{0};
+
+template <bool kFp8, bool kGemm1, int kBN>
+cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const TcParams& p, cudaStream_t st,
+                       const char* name) {
+    constexpr int smem = TC_STAGES * (TC_ABYTES + kBN * TC_ROWB) + 1024;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(grouped_gemm_kernel<kFp8, kGemm1, kBN>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    ProfileScope ps(name, st);
+    grouped_gemm_kernel<kFp8, kGemm1, kBN><<<num_sms(), TC_THREADS, smem, st>>>(a, b, p);
+    note_launch();
+    return cudaGetLastError();
+}
+
+template <bool kFp8>
+cudaError_t launch_gemm1(const CUtensorMap& a, const CUtensorMap& b, const TcParams& p, int half,
+                         cudaStream_t st) {
+    if (half == 128) return launch_one<kFp8, true, 256>(a, b, p, st, "gemm1_tc");
+    if (half == 96) return launch_one<kFp8, true, 192>(a, b, p, st, "gemm1_tc");
+    return launch_one<kFp8, true, 128>(a, b, p, st, "gemm1_tc");
+}
+
+}  // namespace
+
+void ffn_tc_inject_stall(int n_launches) { g_inject.store(n_launches); }
+
+bool ffn_tc_supported(const FfnArgs& a) {
+    if (a.act_dtype != MOE_BF16) return false;
+    if (a.w_dtype != MOE_BF16 && a.w_dtype != MOE_E4M3) return false;
+    if (a.H % 256 != 0 || a.I % 64 != 0) return false;
+    if (a.E + 1 > TC_MAXE) return false;
+    if (encode_fn() == nullptr) return false;
+    return true;
+}
+
+cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
+    if (a.R == 0) return cudaSuccess;
+    const bool fp8 = a.w_dtype == MOE_E4M3;
+    const int esz = fp8 ? 1 : 2;
+    const int half = gemm1_half(a.I);
+    const int kel = fp8 ? 128 : 64;
+    int inject = 0;
+    {
+        int cur = g_inject.load();
+        while (cur > 0 && !g_inject.compare_exchange_weak(cur, cur - 1)) {
+        }
+        inject = cur > 0 ? 1 : 0;
+    }
+
+    // GEMM1: A = Xp [R, H]; B = W13 viewed as [2E][I][H] (gate/up halves separately clipped at I)
+    CUtensorMap ta, tb;
+    {
+        const cuuint64_t ad[2] = {static_cast<cuuint64_t>(a.H), static_cast<cuuint64_t>(a.R)};
+        const cuuint64_t as[1] = {static_cast<cuuint64_t>(a.H) * esz};
+        const cuuint64_t bd[3] = {static_cast<cuuint64_t>(a.H), static_cast<cuuint64_t>(a.I),
+                                  static_cast<cuuint64_t>(2 * a.E)};
+        const cuuint64_t bs[2] = {static_cast<cuuint64_t>(a.H) * esz, static_cast<cuuint64_t>(a.I) * a.H * esz};
+        if (!make_map(&ta, a.xp, fp8, 2, ad, as, TC_BM) || !make_map(&tb, a.w13, fp8, 3, bd, bs, half))
+            return cudaErrorInvalidValue;
+    }
+    TcParams p;
+    p.E = a.E; p.H = a.H; p.I = a.I;
+    p.n_tiles_n = ceil_div(a.I, half);
+    p.bn_out = half;
+    p.k_blocks = ceil_div(a.H, kel);
+    p.offsets = a.offsets;
+    p.tile_off = a.tile_off;
+    p.out = static_cast<uint16_t*>(a.h);
+    p.out_ld = a.I;
+    p.row_scale = fp8 ? a.xp_scale : nullptr;
+    p.col_scale = fp8 ? a.s13 : nullptr;
+    p.status = a.status;
+    p.wait_limit = inject ? (20ll << 20) : (4ll << 30);
+    p.inject_stall = inject;
+    cudaError_t err = fp8 ? launch_gemm1<true>(ta, tb, p, half, st) : launch_gemm1<false>(ta, tb, p, half, st);
+    if (err != cudaSuccess) return err;
+
+    const void* hA = a.h;
+    if (fp8) {
+        err = launch_quant_rows(a.R, a.I, static_cast<const uint16_t*>(a.h), a.hq, a.h_scale, st);
+        if (err != cudaSuccess) return err;
+        hA = a.hq;
+    }
+    // GEMM2: A = h [R, I]; B = W2 viewed as [E*H][I]
+    {
+        const cuuint64_t ad[2] = {static_cast<cuuint64_t>(a.I), static_cast<cuuint64_t>(a.R)};
+        const cuuint64_t as[1] = {static_cast<cuuint64_t>(a.I) * esz};
+        const cuuint64_t bd[2] = {static_cast<cuuint64_t>(a.I), static_cast<cuuint64_t>(a.E) * a.H};
+        const cuuint64_t bs[1] = {static_cast<cuuint64_t>(a.I) * esz};
+        if (!make_map(&ta, hA, fp8, 2, ad, as, TC_BM) || !make_map(&tb, a.w2, fp8, 2, bd, bs, 256))
+            return cudaErrorInvalidValue;
+    }
+    p.n_tiles_n = a.H / 256;
+    p.bn_out = 256;
+    p.k_blocks = ceil_div(a.I, kel);
+    p.out = static_cast<uint16_t*>(a.y);
+    p.out_ld = a.H;
+    p.row_scale = fp8 ? a.h_scale : nullptr;
+    p.col_scale = fp8 ? a.s2 : nullptr;
+    return fp8 ? launch_one<true, false, 256>(ta, tb, p, st, "gemm2_tc")
+               : launch_one<false, false, 256>(ta, tb, p, st, "gemm2_tc");
+}
+
 }  // namespace sre

@@ -58,6 +58,9 @@ cudaError_t launch_ffn_simt(const FfnArgs& a, cudaStream_t stream);
 // ---- expert FFN, tcgen05 tensor-core path (ffn_tc.cu)
 bool ffn_tc_supported(const FfnArgs& a);
 cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t stream);
+// testing hook: the next n grouped-FFN calls on the tensor-core path run with a
+// producer that never issues its loads and a ~10 ms wait limit
+void ffn_tc_inject_stall(int n_calls);
 
 // ---- combine (combine.cu)
 // out[t] = sum_k w[t,k] * y[inv[t*S+k]] (+ add_w * add[t] if add != null)

@@ -1,0 +1,30 @@
+"""Failure detection on the GPU without a GPU fault: a tensor-core GEMM whose
+producer never issues its loads runs its bounded waits out, returns, frees its
+tensor memory and leaves MOE_ERR_TIMEOUT in the status word; the context stays
+usable and the next call is correct."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from shared_routed_expert_b200 import MoELayer, _lib, build, synth
+from tests.parity_util import rel_err, to_f64, tol_of
+
+pytestmark = pytest.mark.gpu
+
+
+def test_wait_timeout_is_reported_and_the_context_survives():
+    build.build()
+    cfg = synth.variant(synth.CONFIGS["prefill_bf16"], T=64, H=512, I=128, n_routed=8, top_k=2)
+    inp = synth.make_inputs(cfg)
+    d = synth.to_device(inp, "cuda")
+    layer = MoELayer(cfg, d)
+    _lib.moe_inject_wait_timeout(1)
+    layer.forward(d["x"])
+    assert layer.status() == _lib.MOE_ERR_TIMEOUT
+    # the status word was cleared by the read; the next pass is clean and right
+    out = layer.forward(d["x"])
+    assert layer.status() == _lib.MOE_OK
+    ref = oracle.Layer(cfg, inp).forward()["out"]
+    assert rel_err(to_f64(out), ref) <= tol_of(cfg)
+    torch.cuda.synchronize()

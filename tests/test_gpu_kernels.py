@@ -182,3 +182,32 @@ def test_grouped_ffn_rows_match_oracle(name, impl):
     rows = list(range(0, T * S, 7)) + [T * S - 1]
     ref = np.stack([Ly.expert_ffn(int(ids.ravel()[perm[r]]), xs[perm[r] // S]) for r in rows])
     assert rel_err(yg[rows], ref) <= tol_of(cfg)
+
+
+@pytest.mark.parametrize("w_dtype", ["bf16", "e4m3"])
+@pytest.mark.parametrize("impl", [MOE_FFN_SIMT, MOE_FFN_TCGEN05], ids=["simt", "tcgen05"])
+def test_grouped_ffn_ragged_group_sizes(w_dtype, impl):
+    """Expert groups of 0, 1, 127, 128, 129 and 300 rows: empty groups, single
+    rows and tails one row either side of the 128-row tile."""
+    base = synth.CONFIGS["prefill_bf16" if w_dtype == "bf16" else "prefill_fp8"]
+    cfg = synth.variant(base, T=137, H=512, I=128, n_routed=5, top_k=4)   # S = 5, R = 685
+    counts = np.array([0, 1, 127, 128, 129, 300], np.int32)
+    assert counts.sum() == cfg.rows
+    offsets = np.r_[0, np.cumsum(counts)].astype(np.int32)
+    perm = np.random.default_rng(11).permutation(cfg.rows).astype(np.int32)
+    inp = synth.make_inputs(cfg)
+    d = synth.to_device(inp, DEV)
+    s = _lib.make_shape(cfg)
+    ws = _lib.alloc_workspace(s, True)
+    y = torch.full((cfg.rows, cfg.H), float("nan"), dtype=torch.bfloat16, device=DEV)
+    _lib.moe_grouped_ffn(s, d["x"], torch.from_numpy(perm).to(DEV), torch.from_numpy(offsets).to(DEV),
+                         d["w13"], d["s13"], d["w2"], d["s2"], y, ws, impl=impl)
+    assert _lib.moe_get_status(ws) == _lib.MOE_OK
+    yg = to_f64(y)
+    assert np.all(np.isfinite(yg))        # every row written exactly by its own group
+    Ly = oracle.Layer(cfg, inp)
+    xs = inp["x"].float().numpy()
+    expert_of = np.repeat(np.arange(6), counts)
+    rows = [0, 1, 127, 128, 129, 255, 256, 257, 384, 385, 600, 684]
+    ref = np.stack([Ly.expert_ffn(int(expert_of[r]), xs[perm[r] // cfg.slots]) for r in rows])
+    assert rel_err(yg[rows], ref) <= tol_of(cfg)

@@ -50,9 +50,9 @@ def test_forward_small_matches_oracle(name):
     d = synth.to_device(inp, DEV)
     ref = oracle.Layer(cfg, inp).forward()
     fused = _run(cfg, d, True)
-    assert rel_err(fused, ref["out_rnd"]) <= tol_of(cfg)
+    assert rel_err(fused, ref["out"]) <= tol_of(cfg)
     unfused = _run(cfg, d, False)
-    assert rel_err(unfused, ref["out_rnd"]) <= tol_of(cfg)
+    assert rel_err(unfused, ref["out"]) <= tol_of(cfg)
     # fused and unfused GPU paths agree with each other as well
     assert rel_err(fused, unfused) <= tol_of(cfg)
 
@@ -73,7 +73,7 @@ def test_zero_router_routes_everything_to_the_lowest_ids():
     ref = oracle.Layer(cfg, inp).forward()
     assert np.all(ref["ids"][:, :2] == [0, 1])
     got = _run(cfg, synth.to_device(inp, DEV))
-    assert rel_err(got, ref["out_rnd"]) <= tol_of(cfg)
+    assert rel_err(got, ref["out"]) <= tol_of(cfg)
 
 
 WORKLOADS = ["prefill_bf16", "decode_bf16", "prefill_fp8", "skewed_fp8"]
@@ -104,7 +104,7 @@ def test_full_size_workload(name):
     ref = oracle.Layer(cfg, host).forward(tokens=tok)
     got = to_f64(out)[tok]
     assert np.all(np.isfinite(to_f64(out)))
-    assert rel_err(got, ref["out_rnd"]) <= tol_of(cfg)
+    assert rel_err(got, ref["out"]) <= tol_of(cfg)
     del layer, d, host
     torch.cuda.empty_cache()
 
