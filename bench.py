@@ -148,7 +148,8 @@ def time_steps(fn, steps: int, warmup: int, dist: Dist, stream) -> float:
 
 
 KERNELS = ["route_logits", "route_topk", "permute_hist", "permute_scan", "permute_scatter",
-           "quant_rows", "gather", "gemm1_tc", "gemm2_tc", "gemm1_simt", "gemm2_simt", "combine"]
+           "quant_rows", "gather", "gemm1_tc", "gemm2_tc", "gemm1_simt", "gemm2_simt", "combine",
+           "round_out"]
 
 
 def kernel_table(steps: int) -> dict:
@@ -165,22 +166,55 @@ def kernel_table(steps: int) -> dict:
 
 
 def algorithmic(cfg, kernel: str, counts: np.ndarray | None):
-    """(bound, work per launch, unit) of one kernel launch for this workload."""
+    """(flops, bytes) one launch of `kernel` must do for this workload: flops of
+    the dense contraction it performs (None if it is not one), and the bytes it
+    must move at least once (touched experts' weights, its own inputs/outputs)."""
     R, T, H, I, Er = cfg.rows, cfg.T, cfg.H, cfg.I, cfg.n_routed
     wb = 1 if cfg.w_dtype == "e4m3" else (4 if cfg.w_dtype == "f32" else 2)
     ab = 4 if cfg.act_dtype == "f32" else 2
+    xb = 1 if wb == 1 else ab                      # bytes per GEMM input activation
     touched = int((counts > 0).sum()) if counts is not None else cfg.n_experts
     if kernel.startswith("gemm1"):
-        return "tensor", 2.0 * R * 2 * I * H, touched * 2 * I * H * wb + R * H * (1 if wb == 1 else ab) + R * I * ab
+        return 2.0 * R * 2 * I * H, touched * 2 * I * H * wb + R * H * xb + R * I * ab
     if kernel.startswith("gemm2"):
-        return "tensor", 2.0 * R * I * H, touched * H * I * wb + R * I * (1 if wb == 1 else ab) + R * H * ab
+        # combine fused in: reads h, writes fp32 partial sums of [T, H] (L2-resident)
+        return 2.0 * R * I * H, touched * H * I * wb + R * I * xb + T * H * 4
     if kernel == "route_logits":
-        return "alu", 2.0 * T * Er * H, T * H * ab + Er * H * 4
+        return None, T * H * ab + Er * H * 4 + (H // 256) * T * Er * 4
     if kernel == "combine":
-        return "hbm", None, R * H * ab + T * H * ab + R * 4 * 2
+        return None, R * H * ab + T * H * ab + R * 4 * 2
     if kernel == "gather":
-        return "hbm", None, 2 * R * H * (1 if wb == 1 else ab)
-    return "hbm", None, None
+        return None, 2 * R * H * xb
+    if kernel == "round_out":
+        return None, T * H * (4 + ab)
+    return None, None
+
+
+def roofline_of(cfg, kernel: str, ms_per_launch: float, counts, pk) -> dict:
+    flops, nbytes = algorithmic(cfg, kernel, counts)
+    t = ms_per_launch / 1000.0
+    tpk = pk["bf16_tflops"] * (2.0 if cfg.w_dtype == "e4m3" else 1.0)
+    src = f"{pk['source']} bf16 burst" + (" x2 (E4M3/bf16 nominal ratio)" if cfg.w_dtype == "e4m3" else "")
+    if kernel == "route_logits":
+        # fp32 CUDA-core FMAs in a fixed order (2 flop each)
+        fl = 2.0 * cfg.T * cfg.n_routed * cfg.H
+        peak = 148 * 128 * 2 * 1.965e9 / 1e12
+        return {"kernel": kernel, "bound": "alu", "achieved": fl / t / 1e12, "peak": peak,
+                "unit": "TFLOP/s", "frac": fl / t / 1e12 / peak, "traffic": None,
+                "peak_source": "148 SMs x 128 fp32 lanes x 2 flop x 1965 MHz"}
+    t_tensor = flops / (tpk * 1e12) if flops else 0.0
+    t_hbm = nbytes / (pk["hbm_gbs"] * 1e9) if nbytes else 0.0
+    if flops and t_tensor >= t_hbm:
+        ach = flops / t / 1e12
+        return {"kernel": kernel, "bound": "tensor", "achieved": ach, "peak": tpk, "unit": "TFLOP/s",
+                "frac": ach / tpk, "traffic": None, "peak_source": src,
+                "hbm_frac": nbytes / t / 1e9 / pk["hbm_gbs"]}
+    ach = (nbytes or 0) / t / 1e9
+    out = {"kernel": kernel, "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+           "frac": ach / pk["hbm_gbs"], "traffic": None, "peak_source": pk["source"]}
+    if flops:
+        out["tensor_frac"] = flops / t / 1e12 / tpk
+    return out
 
 
 # ------------------------------------------------------------------ CPU oracle baseline
@@ -347,22 +381,9 @@ def main():
     roof = None
     if tab:
         top = max(tab, key=lambda k: tab[k]["total_ms"])
-        bound, fl, by = algorithmic(cfg, top, counts)
-        t_launch = tab[top]["ms_per_launch"] / 1000.0
-        if bound == "tensor":
-            ach = fl / t_launch / 1e12
-            roof = {"kernel": top, "bound": "tensor", "achieved": ach, "peak": tensor_peak,
-                    "unit": "TFLOP/s", "frac": ach / tensor_peak, "traffic": None,
-                    "peak_source": f"{pk['source']} bf16 burst" + (" x2 (E4M3 nominal ratio)" if wb == 1 else "")}
-        elif bound == "alu":
-            alu_peak = 148 * 128 * 2 * 1.965e9 / 1e12
-            ach = fl / t_launch / 1e12
-            roof = {"kernel": top, "bound": "alu", "achieved": ach, "peak": alu_peak, "unit": "TFLOP/s",
-                    "frac": ach / alu_peak, "traffic": None, "peak_source": "148 SM x 128 FP32 lanes x 2 x 1965 MHz"}
-        else:
-            ach = (by or 0) / t_launch / 1e9
-            roof = {"kernel": top, "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                    "frac": ach / pk["hbm_gbs"], "traffic": None, "peak_source": pk["source"]}
+        roof = roofline_of(cfg, top, tab[top]["ms_per_launch"], counts, pk)
+        for k in tab:
+            tab[k]["roofline"] = roofline_of(cfg, k, tab[k]["ms_per_launch"], counts, pk)
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": N, "steps": args.steps,

@@ -62,9 +62,9 @@ int act_bytes(int dt) { return dt == MOE_F32 ? 4 : 2; }
 
 struct Layout {
     size_t status, partials, ids, wts, counts, offsets, tile_off, perm, inv, chunk;
-    size_t xq, xscale, xp, xp_scale, h, hq, h_scale, y;
+    size_t xq, xscale, xp, xp_scale, h, hq, h_scale, out_acc;
     // unfused only: the shared expert's dense pass
-    size_t sh_off, sh_tile, sh_h, sh_hq, sh_hscale, sh_y;
+    size_t sh_off, sh_tile, sh_h, sh_hq, sh_hscale;
     size_t total;
 };
 
@@ -113,7 +113,8 @@ Layout layout_of(const moe_shape& s, const Dims& d) {
         L.hq = take(static_cast<size_t>(d.R) * d.I);
         L.h_scale = take(static_cast<size_t>(d.R) * 4);
     }
-    L.y = take(static_cast<size_t>(d.R) * d.H * ab);
+    // fp32 combine accumulator [T, H] (fp32 layers accumulate into `out` itself)
+    if (s.act_dtype != MOE_F32) L.out_acc = take(static_cast<size_t>(d.T) * d.H * 4);
     if (!d.fused && d.shared) {
         L.sh_off = take(2 * 4);
         L.sh_tile = take(2 * 4);
@@ -122,7 +123,6 @@ Layout layout_of(const moe_shape& s, const Dims& d) {
             L.sh_hq = take(static_cast<size_t>(d.T) * d.I);
             L.sh_hscale = take(static_cast<size_t>(d.T) * 4);
         }
-        L.sh_y = take(static_cast<size_t>(d.T) * d.H * ab);
     }
     L.total = off;
     return L;
@@ -198,6 +198,11 @@ FfnArgs ffn_args(const moe_shape& s, const Dims& d, const Layout& L, void* ws, c
     a.hq = s.w_dtype == MOE_E4M3 ? at<uint8_t>(ws, L.hq) : nullptr;
     a.h_scale = s.w_dtype == MOE_E4M3 ? at<float>(ws, L.h_scale) : nullptr;
     a.y = y;
+    a.out_acc = nullptr;
+    a.perm = nullptr;
+    a.S = 1;
+    a.slot_w = nullptr;
+    a.w_const = 0.0f;
     a.max_mtiles = d.R / kTileM + d.E;
     a.status = at<DevStatus>(ws, L.status);
     return a;
@@ -245,7 +250,7 @@ moe_status moe_route_topk(const moe_shape* shape, const void* x, const float* ro
     if (shape->T == 0) return MOE_OK;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     return cuda_status(launch_route(*shape, x, router_w, router_bias, ids, weights, logits,
-                                    at<float>(ws, L.partials), shape->shared_id, st));
+                                    at<float>(ws, L.partials), shape->shared_id, nullptr, st));
 }
 
 moe_status moe_permute(const moe_shape* shape, const int32_t* ids, int32_t* counts,
@@ -330,21 +335,31 @@ moe_status moe_forward(const moe_shape* shape, const void* x, const float* route
 
     int32_t* ids = at<int32_t>(ws, L.ids);
     float* wts = at<float>(ws, L.wts);
+    // fp32 accumulator of the fused combine: zeroed by the top-K kernel, filled by
+    // GEMM2's epilogue, rounded once at the end (fp32 layers accumulate in `out`)
+    const bool f32_out = shape->act_dtype == MOE_F32;
+    float* acc = f32_out ? static_cast<float*>(out) : at<float>(ws, L.out_acc);
     const int route_shared = fused ? shape->shared_id : -1;
     cudaError_t err = launch_route(*shape, x, router_w, router_bias, ids, wts, nullptr,
-                                   at<float>(ws, L.partials), route_shared, st);
+                                   at<float>(ws, L.partials), route_shared, acc, st);
     if (err == cudaSuccess)
         err = launch_permute(d.R, d.E, ids, at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets),
                              at<int32_t>(ws, L.perm), at<int32_t>(ws, L.inv),
                              at<int32_t>(ws, L.tile_off), at<int32_t>(ws, L.chunk),
                              at<DevStatus>(ws, L.status), st);
     if (err == cudaSuccess) err = gather_inputs(*shape, d, L, ws, x, at<int32_t>(ws, L.perm), st);
-    void* y = at<void>(ws, L.y);
-    if (err == cudaSuccess) err = run_ffn(ffn_args(*shape, d, L, ws, w13, s13, w2, s2, y), ffn_impl, st);
+    if (err == cudaSuccess) {
+        FfnArgs a = ffn_args(*shape, d, L, ws, w13, s13, w2, s2, nullptr);
+        a.out_acc = acc;
+        a.perm = at<int32_t>(ws, L.perm);
+        a.S = d.S;
+        a.slot_w = wts;
+        err = run_ffn(a, ffn_impl, st);
+    }
 
-    const void* add = nullptr;
     if (err == cudaSuccess && !fused) {
-        // Unfused: the shared expert as its own dense pass over x (rows = tokens).
+        // Unfused: the shared expert as its own dense pass over x (rows = tokens),
+        // added into the same accumulator with weight shared_weight.
         const int esz = fp8 ? 1 : act_bytes(shape->w_dtype);
         const size_t sid = static_cast<size_t>(shape->shared_id);
         FfnArgs a;
@@ -361,18 +376,21 @@ moe_status moe_forward(const moe_shape* shape, const void* x, const float* route
         a.h = at<void>(ws, L.sh_h);
         a.hq = fp8 ? at<uint8_t>(ws, L.sh_hq) : nullptr;
         a.h_scale = fp8 ? at<float>(ws, L.sh_hscale) : nullptr;
-        a.y = at<void>(ws, L.sh_y);
+        a.y = nullptr;
+        a.out_acc = acc;
+        a.perm = nullptr;
+        a.S = 1;
+        a.slot_w = nullptr;
+        a.w_const = shape->shared_weight;
         a.max_mtiles = ceil_div(d.T, kTileM);
         a.status = at<DevStatus>(ws, L.status);
         dense_offsets_kernel<<<1, 1, 0, st>>>(d.T, at<int32_t>(ws, L.sh_off), at<int32_t>(ws, L.sh_tile));
         note_launch();
         err = cudaGetLastError();
         if (err == cudaSuccess) err = run_ffn(a, ffn_impl, st);
-        add = a.y;
     }
-    if (err == cudaSuccess)
-        err = launch_combine(d.T, d.S, d.H, shape->act_dtype, y, at<int32_t>(ws, L.inv), wts, add,
-                             shape->shared_weight, out, st);
+    if (err == cudaSuccess && !f32_out)
+        err = launch_round_rows(d.T, d.H, acc, static_cast<uint16_t*>(out), st);
     return cuda_status(err);
 }
 

@@ -5,9 +5,12 @@
 // slot K of every token (weight shared_weight), so one weighted sum over the
 // S = K + 1 slots gives the layer output:
 //     out[t] = sum_{k<S} w[t,k] * y[inv[t*S + k]]
-// accumulated in fp32 in slot order and rounded once to the output dtype.
-// The unfused layer passes its separately computed shared-expert output as
-// `add` (weight add_w), added after the routed slots.
+// accumulated in fp32 in slot order and rounded once to the output dtype
+// (the moe_combine entry point, over expert rows y). moe_forward does the same
+// sum inside the down-projection's epilogue and only needs round_rows here.
+// `add` (weight add_w) is an optional extra [T, H] term added last.
+#include <algorithm>
+
 #include "kernels.cuh"
 
 namespace sre {
@@ -96,7 +99,29 @@ __global__ void __launch_bounds__(CB_THREADS) combine_f32_kernel(int T, int S, i
     }
 }
 
+// out = bf16(acc), 8 elements per thread-step
+__global__ void __launch_bounds__(256) round_rows_kernel(size_t n8, const float4* __restrict__ acc,
+                                                         uint4* __restrict__ out) {
+    for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n8;
+         i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+        const float4 a = acc[2 * i], b = acc[2 * i + 1];
+        out[i] = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y),
+                            pack_bf16x2(b.z, b.w));
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_round_rows(int T, int H, const float* acc, uint16_t* out, cudaStream_t stream) {
+    if (T == 0) return cudaSuccess;
+    const size_t n8 = static_cast<size_t>(T) * H / 8;
+    const int blocks = static_cast<int>(std::min<size_t>((n8 + 255) / 256, 148 * 8));
+    ProfileScope ps("round_out", stream);
+    round_rows_kernel<<<blocks, 256, 0, stream>>>(n8, reinterpret_cast<const float4*>(acc),
+                                                   reinterpret_cast<uint4*>(out));
+    note_launch();
+    return cudaGetLastError();
+}
 
 cudaError_t launch_combine(int T, int S, int H, int act_dtype, const void* y, const int32_t* inv,
                            const float* w, const void* add, float add_w, void* out,

@@ -202,12 +202,21 @@ __global__ void __launch_bounds__(256) simt_gemm2_kernel(FfnArgs a) {
         const int row = row0 + ty * 4 + i;
         if (row >= row_end) continue;
         const float hs = (WDT == MOE_E4M3) ? a.h_scale[row] : 1.0f;
+        float wrow = 1.0f;
+        float* arow = nullptr;
+        if (a.out_acc != nullptr) {
+            const int f = a.perm != nullptr ? a.perm[row] : row;
+            wrow = a.slot_w != nullptr ? a.slot_w[f] : a.w_const;
+            arow = a.out_acc + static_cast<size_t>(f / a.S) * H;
+        }
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int n = n0 + tx * 8 + j;
             float v = acc[i][j];
             if (WDT == MOE_E4M3) v = v * hs * a.s2[static_cast<size_t>(e) * H + n];
-            if (HDT == MOE_F32)
+            if (arow != nullptr)
+                atomicAdd(arow + n, v * wrow);
+            else if (HDT == MOE_F32)
                 static_cast<float*>(a.y)[static_cast<size_t>(row) * H + n] = v;
             else
                 static_cast<uint16_t*>(a.y)[static_cast<size_t>(row) * H + n] = f32_to_bf16(v);

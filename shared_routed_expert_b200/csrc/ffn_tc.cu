@@ -8,7 +8,10 @@
 // Two persistent kernels per layer, one CTA per SM:
 //   GEMM1: G = Xp[rows of e] . W13[e]^T; the epilogue applies SwiGLU
 //          h = silu(G_gate) * G_up and stores bf16 h [R, I]
-//   GEMM2: Y = h[rows of e] . W2[e]^T, stored bf16 [R, H]
+//   GEMM2: Y = h[rows of e] . W2[e]^T, either stored bf16 [R, H] or - the
+//          layer's combine fused in - scaled by the row's slot weight and
+//          added into an fp32 [T, H] accumulator with vector reductions at L2
+//          (fp32 sums; the order of the S additions per output is not fixed)
 // E4M3 layers run kind::f8f6f4 with per-row activation scales and
 // per-output-channel weight scales applied in the epilogue (they factor out of
 // the K-sum).
@@ -59,6 +62,13 @@ struct TcParams {
     int out_ld;
     const float* row_scale; // E4M3: per-row activation scale [R]
     const float* col_scale; // E4M3: per-output-channel weight scale (s13 [E, 2I] or s2 [E, H])
+    // GEMM2 combine mode (out_acc != null): out_acc[f / S] += w * y_row with
+    // f = perm[row] (or row), w = slot_w[f] (or w_const); no y rows are written
+    float* out_acc;
+    const int32_t* perm;
+    int S;
+    const float* slot_w;
+    float w_const;
     DevStatus* status;
     long long wait_limit;   // SM clock cycles per wait
     int inject_stall;       // testing hook: the producer never issues its loads
@@ -272,6 +282,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     }
                 }
             } else {
+                float wrow = 1.0f;
+                float* arow = nullptr;
+                if (p.out_acc != nullptr && valid) {
+                    const int f = p.perm != nullptr ? p.perm[row] : row;
+                    wrow = p.slot_w != nullptr ? p.slot_w[f] : p.w_const;
+                    arow = p.out_acc + static_cast<size_t>(f / p.S) * p.H + t.n0;
+                }
 #pragma unroll 1
                 for (int c = 0; c < kBN / 32; ++c) {
                     uint32_t v[32];
@@ -279,20 +296,25 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     ptx::tmem_ld_wait(v);
                     if (valid) {
                         const float* sc = kFp8 ? p.col_scale + static_cast<size_t>(t.e) * p.H + t.n0 + c * 32 : nullptr;
-                        uint32_t packed[16];
+                        float a[32];
 #pragma unroll
-                        for (int j = 0; j < 32; j += 2) {
-                            float a0 = __uint_as_float(v[j]), a1 = __uint_as_float(v[j + 1]);
-                            if constexpr (kFp8) {
-                                a0 = a0 * rs * sc[j];
-                                a1 = a1 * rs * sc[j + 1];
-                            }
-                            packed[j >> 1] = pack_bf16x2(a0, a1);
+                        for (int j = 0; j < 32; ++j) {
+                            a[j] = __uint_as_float(v[j]);
+                            if constexpr (kFp8) a[j] = a[j] * rs * sc[j];
                         }
-                        uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+                        if (arow != nullptr) {
 #pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+                            for (int q = 0; q < 8; ++q)
+                                ptx::red_add_v4(arow + c * 32 + 4 * q, a[4 * q] * wrow, a[4 * q + 1] * wrow,
+                                                a[4 * q + 2] * wrow, a[4 * q + 3] * wrow);
+                        } else {
+                            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+                            for (int q = 0; q < 4; ++q)
+                                dst[q] = make_uint4(pack_bf16x2(a[8 * q], a[8 * q + 1]), pack_bf16x2(a[8 * q + 2], a[8 * q + 3]),
+                                                    pack_bf16x2(a[8 * q + 4], a[8 * q + 5]),
+                                                    pack_bf16x2(a[8 * q + 6], a[8 * q + 7]));
+                        }
                     }
                 }
             }
@@ -433,6 +455,11 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
     p.out_ld = a.I;
     p.row_scale = fp8 ? a.xp_scale : nullptr;
     p.col_scale = fp8 ? a.s13 : nullptr;
+    p.out_acc = nullptr;
+    p.perm = nullptr;
+    p.S = 1;
+    p.slot_w = nullptr;
+    p.w_const = 0.0f;
     p.status = a.status;
     p.wait_limit = inject ? (20ll << 20) : (4ll << 30);
     p.inject_stall = inject;
@@ -461,6 +488,11 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
     p.out_ld = a.H;
     p.row_scale = fp8 ? a.h_scale : nullptr;
     p.col_scale = fp8 ? a.s2 : nullptr;
+    p.out_acc = a.out_acc;
+    p.perm = a.perm;
+    p.S = a.S;
+    p.slot_w = a.slot_w;
+    p.w_const = a.w_const;
     return fp8 ? launch_one<true, false, 256>(ta, tb, p, st, "gemm2_tc")
                : launch_one<false, false, 256>(ta, tb, p, st, "gemm2_tc");
 }

@@ -17,9 +17,10 @@ struct ProfileScope {
 // ---- router (route.cu)
 int router_split_count(int T, int H);
 size_t router_partial_floats(int T, int H, int E);
+// zero_rows (optional): [T, H] fp32 rows the top-K kernel clears (the combine accumulator)
 cudaError_t launch_route(const moe_shape& s, const void* x, const float* wr, const float* bias,
                          int32_t* ids, float* wts, float* logits, float* partials, int shared_id,
-                         cudaStream_t st);
+                         float* zero_rows, cudaStream_t st);
 
 // ---- permutation (permute.cu)
 constexpr int kPermChunk = 512;      // flat slots per scatter chunk
@@ -49,7 +50,15 @@ struct FfnArgs {
     const void* w2;  const float* s2;
     void* h;                      // [R, I] act dtype (bf16 or f32)
     uint8_t* hq; float* h_scale;  // [R, I] codes, [R] (E4M3)
-    void* y;                      // [R, H] act dtype
+    void* y;                      // [R, H] act dtype (row-output mode)
+    // combine mode (out_acc != null): instead of writing y, GEMM2 adds
+    // w * y_row into out_acc[token] (fp32, [T, H]); token = f / S with
+    // f = perm[row] (perm == null: f = row); w = slot_w[f] (slot_w == null: w_const)
+    float* out_acc;
+    const int32_t* perm;
+    int S;
+    const float* slot_w;
+    float w_const;
     int max_mtiles;               // upper bound of sum_e ceil(count_e / kTileM)
     DevStatus* status;
 };
@@ -63,6 +72,8 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t stream);
 void ffn_tc_inject_stall(int n_calls);
 
 // ---- combine (combine.cu)
+// out[t] = bf16(acc[t]) for the fp32 combine accumulator
+cudaError_t launch_round_rows(int T, int H, const float* acc, uint16_t* out, cudaStream_t stream);
 // out[t] = sum_k w[t,k] * y[inv[t*S+k]] (+ add_w * add[t] if add != null)
 cudaError_t launch_combine(int T, int S, int H, int act_dtype, const void* y, const int32_t* inv,
                            const float* w, const void* add, float add_w, void* out,

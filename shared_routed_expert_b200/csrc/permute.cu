@@ -9,8 +9,9 @@
 //
 // Three kernels, no atomics on the order-defining path:
 //   hist:    per 512-slot chunk, per-expert counts (shared-memory histogram)
-//   scan:    one block; per expert an ordered walk over chunks gives each
-//            chunk's base row; counts, offsets and the GEMM tile prefix
+//   scan:    one block; warp-parallel scans over chunks (per expert) and over
+//            experts give each chunk's first row per expert, the counts, the
+//            offsets and the GEMM tile prefix
 //   scatter: one warp per chunk walks its slots in order, 32 at a time;
 //            __match_any_sync ranks equal experts inside a group.
 #include "kernels.cuh"
@@ -19,86 +20,123 @@ namespace sre {
 
 namespace {
 
-__global__ void __launch_bounds__(256) perm_hist_kernel(const int32_t* __restrict__ ids, int R, int E,
-                                                        int32_t* __restrict__ chunk_hist,
+// per 512-slot chunk c: counts of each expert -> chunk_hist[e][c] (expert-major)
+__global__ void __launch_bounds__(128) perm_hist_kernel(const int32_t* __restrict__ ids, int R, int E,
+                                                        int n_chunks, int32_t* __restrict__ chunk_hist,
                                                         DevStatus* status) {
     extern __shared__ int32_t hist[];
     for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
     __syncthreads();
     const int base = blockIdx.x * kPermChunk;
-    for (int i = threadIdx.x; i < kPermChunk; i += blockDim.x) {
+#pragma unroll
+    for (int i = threadIdx.x; i < kPermChunk; i += 128) {
         const int f = base + i;
-        if (f >= R) break;
-        const int e = ids[f];
-        if (e < 0 || e >= E) {
-            report(status, MOE_ERR_DEVICE, static_cast<unsigned>(f));
-            continue;
+        if (f < R) {
+            const int e = ids[f];
+            if (e < 0 || e >= E) report(status, MOE_ERR_DEVICE, static_cast<unsigned>(f));
+            else atomicAdd(&hist[e], 1);
         }
-        atomicAdd(&hist[e], 1);
     }
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x)
-        chunk_hist[static_cast<size_t>(blockIdx.x) * E + e] = hist[e];
+        chunk_hist[static_cast<size_t>(e) * n_chunks + blockIdx.x] = hist[e];
 }
 
-// single block, >= E threads (E <= 1024)
-__global__ void perm_scan_kernel(int n_chunks, int E, int32_t* __restrict__ chunk_hist,
-                                 int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
-                                 int32_t* __restrict__ tile_off) {
+__device__ __forceinline__ int warp_inclusive_scan(int v, int lane) {
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xFFFFFFFFu, v, off);
+        if (lane >= off) v += o;
+    }
+    return v;
+}
+
+// One block of 1024 threads. Warp w owns experts w, w+32, ...:
+//   counts[e] = sum over chunks; offsets = exclusive scan over experts;
+//   chunk_hist[e][c] <- offsets[e] + sum_{c' < c} chunk_hist[e][c'] (each chunk's first row)
+// Also the GEMM tile prefix tile_off[e] = sum_{e' < e} ceil(counts[e'] / kTileM).
+__global__ void __launch_bounds__(1024) perm_scan_kernel(int n_chunks, int E, int32_t* __restrict__ chunk_hist,
+                                                         int32_t* __restrict__ counts,
+                                                         int32_t* __restrict__ offsets,
+                                                         int32_t* __restrict__ tile_off) {
     __shared__ int32_t s_cnt[1024];
     __shared__ int32_t s_off[1025];
-    const int e = threadIdx.x;
-    int run = 0;
-    if (e < E) {
-        for (int c = 0; c < n_chunks; ++c) {
-            const size_t i = static_cast<size_t>(c) * E + e;
-            const int v = chunk_hist[i];
-            chunk_hist[i] = run;
-            run += v;
-        }
-        counts[e] = run;
-        s_cnt[e] = run;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int e = warp; e < E; e += 32) {
+        const int32_t* row = chunk_hist + static_cast<size_t>(e) * n_chunks;
+        int sum = 0;
+        for (int c = lane; c < n_chunks; c += 32) sum += row[c];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, off);
+        if (lane == 0) s_cnt[e] = sum;
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-        int acc = 0, tacc = 0;
-        for (int j = 0; j < E; ++j) {
-            s_off[j] = acc;
-            offsets[j] = acc;
-            tile_off[j] = tacc;
-            acc += s_cnt[j];
-            tacc += ceil_div(s_cnt[j], kTileM);
+    if (warp == 0) {
+        int carry = 0, tcarry = 0;
+        for (int e0 = 0; e0 < E; e0 += 32) {
+            const int e = e0 + lane;
+            const int c = (e < E) ? s_cnt[e] : 0;
+            const int tc = ceil_div(c, kTileM);
+            const int inc = warp_inclusive_scan(c, lane);
+            const int tinc = warp_inclusive_scan(tc, lane);
+            if (e < E) {
+                s_off[e] = carry + inc - c;
+                counts[e] = c;
+                offsets[e] = carry + inc - c;
+                tile_off[e] = tcarry + tinc - tc;
+            }
+            carry += __shfl_sync(0xFFFFFFFFu, inc, 31);
+            tcarry += __shfl_sync(0xFFFFFFFFu, tinc, 31);
         }
-        s_off[E] = acc;
-        offsets[E] = acc;
-        tile_off[E] = tacc;
+        if (lane == 0) {
+            s_off[E] = carry;
+            offsets[E] = carry;
+            tile_off[E] = tcarry;
+        }
     }
     __syncthreads();
-    if (e < E) {
-        const int o = s_off[e];
-        for (int c = 0; c < n_chunks; ++c) chunk_hist[static_cast<size_t>(c) * E + e] += o;
+    for (int e = warp; e < E; e += 32) {
+        int32_t* row = chunk_hist + static_cast<size_t>(e) * n_chunks;
+        int carry = s_off[e];
+        for (int c0 = 0; c0 < n_chunks; c0 += 32) {
+            const int c = c0 + lane;
+            const int v = (c < n_chunks) ? row[c] : 0;
+            const int inc = warp_inclusive_scan(v, lane);
+            if (c < n_chunks) row[c] = carry + inc - v;
+            carry += __shfl_sync(0xFFFFFFFFu, inc, 31);
+        }
     }
 }
 
-// one warp per chunk
+// One warp per chunk: the chunk's ids are loaded first (all loads in flight
+// at once), then ranked 32 at a time in slot order; __match_any_sync groups
+// equal experts, the rank inside a group is the count of lower lanes.
+constexpr int kPermPerLane = kPermChunk / 32;
 __global__ void __launch_bounds__(32) perm_scatter_kernel(const int32_t* __restrict__ ids, int R, int E,
+                                                          int n_chunks,
                                                           const int32_t* __restrict__ chunk_base,
                                                           int32_t* __restrict__ perm,
                                                           int32_t* __restrict__ inv) {
     extern __shared__ int32_t next[];
     const int lane = threadIdx.x;
-    for (int e = lane; e < E; e += 32) next[e] = chunk_base[static_cast<size_t>(blockIdx.x) * E + e];
-    __syncwarp();
+    for (int e = lane; e < E; e += 32) next[e] = chunk_base[static_cast<size_t>(e) * n_chunks + blockIdx.x];
     const int base = blockIdx.x * kPermChunk;
-    const unsigned lt = (1u << lane) - 1u;
-    for (int g = 0; g < kPermChunk; g += 32) {
-        const int f = base + g + lane;
+    int my[kPermPerLane];
+#pragma unroll
+    for (int g = 0; g < kPermPerLane; ++g) {
+        const int f = base + g * 32 + lane;
         int e = (f < R) ? ids[f] : -1;
-        if (e < 0 || e >= E) e = -1;
+        my[g] = (e < 0 || e >= E) ? -1 : e;
+    }
+    __syncwarp();
+    const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+    for (int g = 0; g < kPermPerLane; ++g) {
+        const int f = base + g * 32 + lane;
+        const int e = my[g];
         const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
-        int row = 0;
         if (e >= 0) {
-            row = next[e] + __popc(peers & lt);
+            const int row = next[e] + __popc(peers & lt);
             perm[row] = f;
             inv[f] = row;
         }
@@ -180,18 +218,17 @@ cudaError_t launch_permute(int R, int E, const int32_t* ids, int32_t* counts, in
     const size_t hsm = static_cast<size_t>(E) * sizeof(int32_t);
     if (n_chunks > 0) {
         ProfileScope ps("permute_hist", stream);
-        perm_hist_kernel<<<n_chunks, 256, hsm, stream>>>(ids, R, E, scratch, st);
+        perm_hist_kernel<<<n_chunks, 128, hsm, stream>>>(ids, R, E, n_chunks, scratch, st);
         note_launch();
     }
     {
         ProfileScope ps("permute_scan", stream);
-        perm_scan_kernel<<<1, ceil_div(E, 32) * 32, 0, stream>>>(n_chunks, E, scratch, counts,
-                                                                 offsets, tile_off);
+        perm_scan_kernel<<<1, 1024, 0, stream>>>(n_chunks, E, scratch, counts, offsets, tile_off);
         note_launch();
     }
     if (n_chunks > 0) {
         ProfileScope ps("permute_scatter", stream);
-        perm_scatter_kernel<<<n_chunks, 32, hsm, stream>>>(ids, R, E, scratch, perm, inv);
+        perm_scatter_kernel<<<n_chunks, 32, hsm, stream>>>(ids, R, E, n_chunks, scratch, perm, inv);
         note_launch();
     }
     return cudaGetLastError();

@@ -162,6 +162,13 @@ __device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[32]) {
     for (int i = 0; i < 32; ++i) asm volatile("" : "+r"(r[i]));
 }
 
+// ------------------------------------------------------------------ global reductions
+// out[0..3] += v (fp32, relaxed, performed at L2); out must be 16-byte aligned
+__device__ __forceinline__ void red_add_v4(float* out, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(out), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+
 // ------------------------------------------------------------------ descriptors
 // Shared-memory matrix descriptor of a K-major tile whose rows are 128 bytes
 // long, stored with the 128-byte swizzle in 1024-byte groups of 8 rows (the
