@@ -47,19 +47,27 @@ def peaks():
 # ------------------------------------------------------------------ distributed plumbing
 
 class Dist:
-    def __init__(self, gpus: int):
+    """One process per GPU (torchrun env). NCCL on GPUs; gloo when no GPU is
+    visible (the CPU tests of this host logic). Only the timing barrier and the
+    max-over-ranks of the step time are collectives."""
+
+    def __init__(self, gpus: int, backend: str | None = None):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
         self.pg = None
+        cuda = torch.cuda.is_available()
+        self.backend = backend or ("nccl" if cuda else "gloo")
+        self.device = torch.device("cuda", self.local) if self.backend == "nccl" else torch.device("cpu")
         if self.world > 1:
             import datetime
             import torch.distributed as dist
-            torch.cuda.set_device(self.local)
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                    device_id=torch.device("cuda", self.local))
+            kw = {}
+            if self.backend == "nccl":
+                torch.cuda.set_device(self.local)
+                kw["device_id"] = self.device
+            dist.init_process_group(self.backend, timeout=datetime.timedelta(seconds=120), **kw)
             self.pg = dist
-        self.device = torch.device("cuda", self.local)
 
     def barrier(self):
         if self.pg is not None:
@@ -127,6 +135,11 @@ class Clocks:
 
 
 # ------------------------------------------------------------------ timing
+
+def tokens_per_s(n_ranks: int, tokens_per_rank: int, steps: int, max_ms: float) -> float:
+    """Whole-job throughput: every rank's tokens over the slowest rank's time."""
+    return n_ranks * tokens_per_rank * steps / (max_ms / 1000.0)
+
 
 def time_steps(fn, steps: int, warmup: int, dist: Dist, stream) -> float:
     """Device time of `steps` back-to-back calls (ms), max over ranks."""
@@ -370,7 +383,7 @@ def main():
 
     N = dist.world
     ms_step = ms / args.steps
-    value = N * cfg.T * args.steps / (ms / 1000.0)
+    value = tokens_per_s(N, cfg.T, args.steps, ms)
     pk = peaks()
     flops = cfg.gemm_flops() + cfg.router_flops()
     wb = 1 if cfg.w_dtype == "e4m3" else 2

@@ -138,16 +138,14 @@ moe_status moe_combine(const moe_shape* shape, const void* y, const int32_t* inv
                        const float* weights, void* out, void* stream);
 
 /* The whole layer. fuse_shared = 1: the fused top-(K+1) pass (route -> permute
- * -> grouped FFN over all E experts, with the weighted aggregation done in the
- * down-projection's epilogue). fuse_shared = 0: the unfused layer of the
+ * -> grouped FFN over all E experts -> weighted aggregation). fuse_shared = 0: the unfused layer of the
  * pseudocode in section 2.1 of "GLM4-MoE生产环境优化：SGLang降低65%首Token延迟":
  * routed top-K pass plus a separate dense pass of the shared expert added with
  * weight shared_weight (the GPU baseline the fusion is measured against; needs
  * shared_id >= 0).
- * The aggregation adds w * y for each of a token's slots into an fp32
- * accumulator and rounds once to act_dtype at the end. The order of those fp32
- * additions is not fixed, so the last bits of `out` may differ between runs;
- * routing, counts and the permutation are deterministic.
+ * The expert rows are kept as fp16 scaled by a power of two per 32 columns
+ * (11 significant bits) and aggregated in fp32 in slot order, rounded once to
+ * act_dtype; the result is deterministic.
  *   x [T, H], router_w [n_routed, H], router_bias [n_routed] or NULL,
  *   w13 [E, 2I, H], s13, w2 [E, H, I], s2 as in moe_grouped_ffn, out [T, H].
  * Needs moe_workspace_size(shape, fuse_shared) bytes of ws. */

@@ -62,9 +62,9 @@ int act_bytes(int dt) { return dt == MOE_F32 ? 4 : 2; }
 
 struct Layout {
     size_t status, partials, ids, wts, counts, offsets, tile_off, perm, inv, chunk;
-    size_t xq, xscale, xp, xp_scale, h, hq, h_scale, out_acc;
+    size_t xq, xscale, xp, xp_scale, h, hq, h_scale, y, yexp;
     // unfused only: the shared expert's dense pass
-    size_t sh_off, sh_tile, sh_h, sh_hq, sh_hscale;
+    size_t sh_off, sh_tile, sh_h, sh_hq, sh_hscale, sh_y, sh_yexp;
     size_t total;
 };
 
@@ -113,8 +113,9 @@ Layout layout_of(const moe_shape& s, const Dims& d) {
         L.hq = take(static_cast<size_t>(d.R) * d.I);
         L.h_scale = take(static_cast<size_t>(d.R) * 4);
     }
-    // fp32 combine accumulator [T, H] (fp32 layers accumulate into `out` itself)
-    if (s.act_dtype != MOE_F32) L.out_acc = take(static_cast<size_t>(d.T) * d.H * 4);
+    // expert rows: fp32 for fp32 layers, else scaled fp16 + one exponent byte per 32 columns
+    L.y = take(static_cast<size_t>(d.R) * d.H * ab);
+    if (s.act_dtype != MOE_F32) L.yexp = take(static_cast<size_t>(d.R) * (d.H / 32));
     if (!d.fused && d.shared) {
         L.sh_off = take(2 * 4);
         L.sh_tile = take(2 * 4);
@@ -123,6 +124,8 @@ Layout layout_of(const moe_shape& s, const Dims& d) {
             L.sh_hq = take(static_cast<size_t>(d.T) * d.I);
             L.sh_hscale = take(static_cast<size_t>(d.T) * 4);
         }
+        L.sh_y = take(static_cast<size_t>(d.T) * d.H * ab);
+        if (s.act_dtype != MOE_F32) L.sh_yexp = take(static_cast<size_t>(d.T) * (d.H / 32));
     }
     L.total = off;
     return L;
@@ -184,11 +187,32 @@ moe_status check_impl(int impl, const moe_shape& s) {
     return MOE_OK;
 }
 
-FfnArgs ffn_args(const moe_shape& s, const Dims& d, const Layout& L, void* ws, const void* w13,
-                 const float* s13, const void* w2, const float* s2, void* y) {
+// Quantises x per token to E4M3 for E4M3 layers; returns the token matrix the
+// grouped pass reads (x itself otherwise).
+cudaError_t prepare_tokens(const moe_shape& s, const Dims& d, const Layout& L, void* ws, const void* x,
+                           const void** xt, const float** xt_scale, cudaStream_t st) {
+    if (s.w_dtype == MOE_E4M3) {
+        *xt = at<uint8_t>(ws, L.xq);
+        *xt_scale = at<float>(ws, L.xscale);
+        return launch_quant_rows(d.T, d.H, static_cast<const uint16_t*>(x), at<uint8_t>(ws, L.xq),
+                                 at<float>(ws, L.xscale), st);
+    }
+    *xt = x;
+    *xt_scale = nullptr;
+    return cudaSuccess;
+}
+
+FfnArgs ffn_args(const moe_shape& s, const Dims& d, const Layout& L, void* ws, const void* xt,
+                 const float* xt_scale, const int32_t* perm, const void* w13, const float* s13,
+                 const void* w2, const float* s2, void* y) {
     FfnArgs a;
     a.R = d.R; a.H = d.H; a.I = d.I; a.E = d.E;
     a.act_dtype = s.act_dtype; a.w_dtype = s.w_dtype;
+    a.xt = xt;
+    a.xt_scale = xt_scale;
+    a.T = d.T;
+    a.perm = perm;
+    a.S = d.S;
     a.xp = at<void>(ws, L.xp);
     a.xp_scale = at<float>(ws, L.xp_scale);
     a.offsets = at<int32_t>(ws, L.offsets);
@@ -198,29 +222,10 @@ FfnArgs ffn_args(const moe_shape& s, const Dims& d, const Layout& L, void* ws, c
     a.hq = s.w_dtype == MOE_E4M3 ? at<uint8_t>(ws, L.hq) : nullptr;
     a.h_scale = s.w_dtype == MOE_E4M3 ? at<float>(ws, L.h_scale) : nullptr;
     a.y = y;
-    a.out_acc = nullptr;
-    a.perm = nullptr;
-    a.S = 1;
-    a.slot_w = nullptr;
-    a.w_const = 0.0f;
+    a.yexp = nullptr;
     a.max_mtiles = d.R / kTileM + d.E;
     a.status = at<DevStatus>(ws, L.status);
     return a;
-}
-
-// Gathers x rows for the grouped pass (quantising x per token first for E4M3).
-cudaError_t gather_inputs(const moe_shape& s, const Dims& d, const Layout& L, void* ws, const void* x,
-                          const int32_t* perm, cudaStream_t st) {
-    cudaError_t err;
-    if (s.w_dtype == MOE_E4M3) {
-        err = launch_quant_rows(d.T, d.H, static_cast<const uint16_t*>(x), at<uint8_t>(ws, L.xq),
-                                at<float>(ws, L.xscale), st);
-        if (err != cudaSuccess) return err;
-        return launch_gather_rows(d.R, d.S, d.H, 1, at<uint8_t>(ws, L.xq), at<float>(ws, L.xscale),
-                                  perm, at<void>(ws, L.xp), at<float>(ws, L.xp_scale), st);
-    }
-    return launch_gather_rows(d.R, d.S, d.H, act_bytes(s.act_dtype), x, nullptr, perm,
-                              at<void>(ws, L.xp), nullptr, st);
 }
 
 }  // namespace
@@ -250,7 +255,7 @@ moe_status moe_route_topk(const moe_shape* shape, const void* x, const float* ro
     if (shape->T == 0) return MOE_OK;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     return cuda_status(launch_route(*shape, x, router_w, router_bias, ids, weights, logits,
-                                    at<float>(ws, L.partials), shape->shared_id, nullptr, st));
+                                    at<float>(ws, L.partials), shape->shared_id, st));
 }
 
 moe_status moe_permute(const moe_shape* shape, const int32_t* ids, int32_t* counts,
@@ -295,8 +300,11 @@ moe_status moe_grouped_ffn(const moe_shape* shape, const void* x, const int32_t*
         note_launch();
         err = cudaGetLastError();
     }
-    if (err == cudaSuccess) err = gather_inputs(*shape, d, L, ws, x, perm, st);
-    if (err == cudaSuccess) err = run_ffn(ffn_args(*shape, d, L, ws, w13, s13, w2, s2, y), ffn_impl, st);
+    const void* xt = nullptr;
+    const float* xt_scale = nullptr;
+    if (err == cudaSuccess) err = prepare_tokens(*shape, d, L, ws, x, &xt, &xt_scale, st);
+    if (err == cudaSuccess)
+        err = run_ffn(ffn_args(*shape, d, L, ws, xt, xt_scale, perm, w13, s13, w2, s2, y), ffn_impl, st);
     return cuda_status(err);
 }
 
@@ -335,38 +343,40 @@ moe_status moe_forward(const moe_shape* shape, const void* x, const float* route
 
     int32_t* ids = at<int32_t>(ws, L.ids);
     float* wts = at<float>(ws, L.wts);
-    // fp32 accumulator of the fused combine: zeroed by the top-K kernel, filled by
-    // GEMM2's epilogue, rounded once at the end (fp32 layers accumulate in `out`)
-    const bool f32_out = shape->act_dtype == MOE_F32;
-    float* acc = f32_out ? static_cast<float*>(out) : at<float>(ws, L.out_acc);
+    const bool f32_act = shape->act_dtype == MOE_F32;
     const int route_shared = fused ? shape->shared_id : -1;
     cudaError_t err = launch_route(*shape, x, router_w, router_bias, ids, wts, nullptr,
-                                   at<float>(ws, L.partials), route_shared, acc, st);
+                                   at<float>(ws, L.partials), route_shared, st);
     if (err == cudaSuccess)
         err = launch_permute(d.R, d.E, ids, at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets),
                              at<int32_t>(ws, L.perm), at<int32_t>(ws, L.inv),
                              at<int32_t>(ws, L.tile_off), at<int32_t>(ws, L.chunk),
                              at<DevStatus>(ws, L.status), st);
-    if (err == cudaSuccess) err = gather_inputs(*shape, d, L, ws, x, at<int32_t>(ws, L.perm), st);
+    const void* xt = nullptr;
+    const float* xt_scale = nullptr;
+    if (err == cudaSuccess) err = prepare_tokens(*shape, d, L, ws, x, &xt, &xt_scale, st);
     if (err == cudaSuccess) {
-        FfnArgs a = ffn_args(*shape, d, L, ws, w13, s13, w2, s2, nullptr);
-        a.out_acc = acc;
-        a.perm = at<int32_t>(ws, L.perm);
-        a.S = d.S;
-        a.slot_w = wts;
+        FfnArgs a = ffn_args(*shape, d, L, ws, xt, xt_scale, at<int32_t>(ws, L.perm), w13, s13, w2, s2,
+                             at<void>(ws, L.y));
+        a.yexp = f32_act ? nullptr : at<int8_t>(ws, L.yexp);
         err = run_ffn(a, ffn_impl, st);
     }
 
     if (err == cudaSuccess && !fused) {
-        // Unfused: the shared expert as its own dense pass over x (rows = tokens),
-        // added into the same accumulator with weight shared_weight.
+        // Unfused: the shared expert as its own dense pass over x (rows = tokens);
+        // the combine adds it with weight shared_weight.
         const int esz = fp8 ? 1 : act_bytes(shape->w_dtype);
         const size_t sid = static_cast<size_t>(shape->shared_id);
         FfnArgs a;
         a.R = d.T; a.H = d.H; a.I = d.I; a.E = 1;
         a.act_dtype = shape->act_dtype; a.w_dtype = shape->w_dtype;
-        a.xp = fp8 ? static_cast<const void*>(at<uint8_t>(ws, L.xq)) : x;
-        a.xp_scale = fp8 ? at<float>(ws, L.xscale) : nullptr;
+        a.xt = xt;
+        a.xt_scale = xt_scale;
+        a.T = d.T;
+        a.perm = nullptr;          // rows are the tokens in order
+        a.S = 1;
+        a.xp = nullptr;
+        a.xp_scale = nullptr;
         a.offsets = at<int32_t>(ws, L.sh_off);
         a.tile_off = at<int32_t>(ws, L.sh_tile);
         a.w13 = static_cast<const char*>(w13) + sid * 2 * d.I * d.H * esz;
@@ -376,12 +386,8 @@ moe_status moe_forward(const moe_shape* shape, const void* x, const float* route
         a.h = at<void>(ws, L.sh_h);
         a.hq = fp8 ? at<uint8_t>(ws, L.sh_hq) : nullptr;
         a.h_scale = fp8 ? at<float>(ws, L.sh_hscale) : nullptr;
-        a.y = nullptr;
-        a.out_acc = acc;
-        a.perm = nullptr;
-        a.S = 1;
-        a.slot_w = nullptr;
-        a.w_const = shape->shared_weight;
+        a.y = at<void>(ws, L.sh_y);
+        a.yexp = f32_act ? nullptr : at<int8_t>(ws, L.sh_yexp);
         a.max_mtiles = ceil_div(d.T, kTileM);
         a.status = at<DevStatus>(ws, L.status);
         dense_offsets_kernel<<<1, 1, 0, st>>>(d.T, at<int32_t>(ws, L.sh_off), at<int32_t>(ws, L.sh_tile));
@@ -389,8 +395,17 @@ moe_status moe_forward(const moe_shape* shape, const void* x, const float* route
         err = cudaGetLastError();
         if (err == cudaSuccess) err = run_ffn(a, ffn_impl, st);
     }
-    if (err == cudaSuccess && !f32_out)
-        err = launch_round_rows(d.T, d.H, acc, static_cast<uint16_t*>(out), st);
+    if (err == cudaSuccess) {
+        const int32_t* inv = at<int32_t>(ws, L.inv);
+        if (f32_act)
+            err = launch_combine(d.T, d.S, d.H, MOE_F32, at<void>(ws, L.y), inv, wts,
+                                 fused ? nullptr : at<void>(ws, L.sh_y), shape->shared_weight, out, st);
+        else
+            err = launch_combine_f16s(d.T, d.S, d.H, at<uint16_t>(ws, L.y), at<int8_t>(ws, L.yexp), inv, wts,
+                                      fused ? nullptr : at<uint16_t>(ws, L.sh_y),
+                                      fused ? nullptr : at<int8_t>(ws, L.sh_yexp), shape->shared_weight,
+                                      static_cast<uint16_t*>(out), st);
+    }
     return cuda_status(err);
 }
 

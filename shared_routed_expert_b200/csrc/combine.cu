@@ -6,11 +6,11 @@
 // S = K + 1 slots gives the layer output:
 //     out[t] = sum_{k<S} w[t,k] * y[inv[t*S + k]]
 // accumulated in fp32 in slot order and rounded once to the output dtype
-// (the moe_combine entry point, over expert rows y). moe_forward does the same
-// sum inside the down-projection's epilogue and only needs round_rows here.
-// `add` (weight add_w) is an optional extra [T, H] term added last.
-#include <algorithm>
-
+// The moe_combine entry point runs it over bf16/fp32 expert rows; moe_forward
+// over the scaled-fp16 rows its down-projection writes (11 significant bits,
+// so that storing the rows adds ~2^-12 relative error per slot instead of
+// bf16's 2^-9). `add` (weight add_w) is an optional [T, H] term added last:
+// the unfused layer's separately computed shared expert.
 #include "kernels.cuh"
 
 namespace sre {
@@ -99,26 +99,69 @@ __global__ void __launch_bounds__(CB_THREADS) combine_f32_kernel(int T, int S, i
     }
 }
 
-// out = bf16(acc), 8 elements per thread-step
-__global__ void __launch_bounds__(256) round_rows_kernel(size_t n8, const float4* __restrict__ acc,
-                                                         uint4* __restrict__ out) {
-    for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n8;
-         i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-        const float4 a = acc[2 * i], b = acc[2 * i + 1];
-        out[i] = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y),
-                            pack_bf16x2(b.z, b.w));
+// Scaled-fp16 rows (see the GEMM2 epilogue): value = fp16 * 2^k, one k per 32
+// columns. Each thread owns 8-column vectors of the token's row (4 threads per
+// exponent byte).
+__global__ void __launch_bounds__(CB_THREADS) combine_f16s_kernel(int T, int S, int H,
+                                                                  const uint4* __restrict__ y,
+                                                                  const int8_t* __restrict__ yexp,
+                                                                  const int32_t* __restrict__ inv,
+                                                                  const float* __restrict__ w,
+                                                                  const uint4* __restrict__ add,
+                                                                  const int8_t* __restrict__ addexp,
+                                                                  float add_w, uint4* __restrict__ out) {
+    const int t = blockIdx.x;
+    const int nv = H / 8, ne = H / 32;
+    __shared__ int32_t s_row[64];
+    __shared__ float s_w[64];
+    for (int k = threadIdx.x; k < S; k += blockDim.x) {
+        s_row[k] = inv[static_cast<size_t>(t) * S + k];
+        s_w[k] = w[static_cast<size_t>(t) * S + k];
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < nv; i += blockDim.x) {
+        float acc[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
+        for (int k = 0; k < S; ++k) {
+            const size_t r = static_cast<size_t>(s_row[k]);
+            const uint4 q = y[r * nv + i];
+            const float wk = s_w[k] * exp2_int(yexp[r * ne + (i >> 2)]);
+            const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float2 f = unpack_f16x2(u[j]);
+                acc[2 * j] = __fmaf_rn(wk, f.x, acc[2 * j]);
+                acc[2 * j + 1] = __fmaf_rn(wk, f.y, acc[2 * j + 1]);
+            }
+        }
+        if (add != nullptr) {
+            const uint4 q = add[static_cast<size_t>(t) * nv + i];
+            const float wk = add_w * exp2_int(addexp[static_cast<size_t>(t) * ne + (i >> 2)]);
+            const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float2 f = unpack_f16x2(u[j]);
+                acc[2 * j] = __fmaf_rn(wk, f.x, acc[2 * j]);
+                acc[2 * j + 1] = __fmaf_rn(wk, f.y, acc[2 * j + 1]);
+            }
+        }
+        out[static_cast<size_t>(t) * nv + i] =
+            make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
+                       pack_bf16x2(acc[6], acc[7]));
     }
 }
 
 }  // namespace
 
-cudaError_t launch_round_rows(int T, int H, const float* acc, uint16_t* out, cudaStream_t stream) {
+cudaError_t launch_combine_f16s(int T, int S, int H, const uint16_t* y16, const int8_t* yexp,
+                                const int32_t* inv, const float* w, const uint16_t* add16,
+                                const int8_t* addexp, float add_w, uint16_t* out, cudaStream_t stream) {
     if (T == 0) return cudaSuccess;
-    const size_t n8 = static_cast<size_t>(T) * H / 8;
-    const int blocks = static_cast<int>(std::min<size_t>((n8 + 255) / 256, 148 * 8));
-    ProfileScope ps("round_out", stream);
-    round_rows_kernel<<<blocks, 256, 0, stream>>>(n8, reinterpret_cast<const float4*>(acc),
-                                                   reinterpret_cast<uint4*>(out));
+    ProfileScope ps("combine", stream);
+    combine_f16s_kernel<<<T, CB_THREADS, 0, stream>>>(T, S, H, reinterpret_cast<const uint4*>(y16), yexp, inv,
+                                                      w, reinterpret_cast<const uint4*>(add16), addexp, add_w,
+                                                      reinterpret_cast<uint4*>(out));
     note_launch();
     return cudaGetLastError();
 }

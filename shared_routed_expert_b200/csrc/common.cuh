@@ -3,6 +3,7 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_fp8.h>
 #include <stdint.h>
 
@@ -49,6 +50,28 @@ __device__ __forceinline__ float e4m3_to_f32(uint8_t c) {
 // round to nearest even, saturate to +-448 (cvt.rn.satfinite)
 __device__ __forceinline__ uint8_t f32_to_e4m3(float f) {
     return static_cast<uint8_t>(__nv_cvt_float_to_fp8(f, __NV_SATFINITE, __NV_E4M3));
+}
+
+// Power-of-two exponent k for a chunk whose largest magnitude is amax, so that
+// amax * 2^-k lies in [2^14, 2^15) (fp16 keeps 11 significant bits there and
+// cannot overflow). k is clamped to [-100, 113]; amax = 0 gives k = 0.
+__device__ __forceinline__ int f16_chunk_exp(float amax) {
+    if (!(amax > 0.0f)) return 0;
+    const int ex = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu) - 127;
+    return max(-100, min(113, ex - 14));
+}
+
+__device__ __forceinline__ float exp2_int(int k) {   // 2^k for k in [-126, 127]
+    return __uint_as_float(static_cast<uint32_t>(127 + k) << 23);
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float a, float b) {
+    __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ float2 unpack_f16x2(uint32_t v) {
+    return __half22float2(*reinterpret_cast<__half2*>(&v));
 }
 
 __device__ __forceinline__ float silu_f32(float g) { return g / (1.0f + __expf(-g)); }

@@ -197,37 +197,63 @@ __global__ void __launch_bounds__(256) simt_gemm2_kernel(FfnArgs a) {
         }
         __syncthreads();
     }
+    // Scaled-fp16 rows: the 32-column chunk of a row is spread over 4 lanes
+    // (tx = 4c..4c+3), so its amax is reduced over lane bits 0-1. Every lane
+    // runs the shuffles; only valid rows store.
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int row = row0 + ty * 4 + i;
-        if (row >= row_end) continue;
-        const float hs = (WDT == MOE_E4M3) ? a.h_scale[row] : 1.0f;
-        float wrow = 1.0f;
-        float* arow = nullptr;
-        if (a.out_acc != nullptr) {
-            const int f = a.perm != nullptr ? a.perm[row] : row;
-            wrow = a.slot_w != nullptr ? a.slot_w[f] : a.w_const;
-            arow = a.out_acc + static_cast<size_t>(f / a.S) * H;
-        }
+        const bool valid = row < row_end;
+        const float hs = (WDT == MOE_E4M3 && valid) ? a.h_scale[row] : 1.0f;
+        float v[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int n = n0 + tx * 8 + j;
-            float v = acc[i][j];
-            if (WDT == MOE_E4M3) v = v * hs * a.s2[static_cast<size_t>(e) * H + n];
-            if (arow != nullptr)
-                atomicAdd(arow + n, v * wrow);
-            else if (HDT == MOE_F32)
-                static_cast<float*>(a.y)[static_cast<size_t>(row) * H + n] = v;
-            else
-                static_cast<uint16_t*>(a.y)[static_cast<size_t>(row) * H + n] = f32_to_bf16(v);
+            v[j] = acc[i][j];
+            if (WDT == MOE_E4M3 && valid) v[j] = v[j] * hs * a.s2[static_cast<size_t>(e) * H + n];
+        }
+        if (a.yexp != nullptr) {
+            float amax = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[j]));
+            amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+            amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+            const int k = f16_chunk_exp(amax);
+            const float down = exp2_int(-k);
+            if (valid) {
+                uint16_t* dst = static_cast<uint16_t*>(a.y) + static_cast<size_t>(row) * H + n0 + tx * 8;
+                *reinterpret_cast<uint4*>(dst) =
+                    make_uint4(pack_f16x2(v[0] * down, v[1] * down), pack_f16x2(v[2] * down, v[3] * down),
+                               pack_f16x2(v[4] * down, v[5] * down), pack_f16x2(v[6] * down, v[7] * down));
+                if ((tx & 3) == 0) a.yexp[static_cast<size_t>(row) * (H / 32) + (n0 + tx * 8) / 32] = static_cast<int8_t>(k);
+            }
+        } else if (valid) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int n = n0 + tx * 8 + j;
+                if (HDT == MOE_F32)
+                    static_cast<float*>(a.y)[static_cast<size_t>(row) * H + n] = v[j];
+                else
+                    static_cast<uint16_t*>(a.y)[static_cast<size_t>(row) * H + n] = f32_to_bf16(v[j]);
+            }
         }
     }
 }
 
 }  // namespace
 
-cudaError_t launch_ffn_simt(const FfnArgs& a, cudaStream_t stream) {
-    if (a.R == 0 || a.max_mtiles == 0) return cudaSuccess;
+cudaError_t launch_ffn_simt(const FfnArgs& in, cudaStream_t stream) {
+    if (in.R == 0 || in.max_mtiles == 0) return cudaSuccess;
+    FfnArgs a = in;
+    if (a.perm != nullptr) {
+        // rows of the grouped pass gathered from the token matrix
+        const int eb = (a.w_dtype == MOE_E4M3) ? 1 : (a.act_dtype == MOE_F32 ? 4 : 2);
+        cudaError_t err = launch_gather_rows(a.R, a.S, a.H, eb, a.xt, a.xt_scale, a.perm, a.xp, a.xp_scale, stream);
+        if (err != cudaSuccess) return err;
+    } else {
+        a.xp = const_cast<void*>(a.xt);           // row r is token r
+        a.xp_scale = const_cast<float*>(a.xt_scale);
+    }
     const dim3 g1(a.max_mtiles, a.I / 32), g2(a.max_mtiles, a.H / 64);
     {
         ProfileScope ps("gemm1_simt", stream);

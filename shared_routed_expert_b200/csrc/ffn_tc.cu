@@ -8,10 +8,10 @@
 // Two persistent kernels per layer, one CTA per SM:
 //   GEMM1: G = Xp[rows of e] . W13[e]^T; the epilogue applies SwiGLU
 //          h = silu(G_gate) * G_up and stores bf16 h [R, I]
-//   GEMM2: Y = h[rows of e] . W2[e]^T, either stored bf16 [R, H] or - the
-//          layer's combine fused in - scaled by the row's slot weight and
-//          added into an fp32 [T, H] accumulator with vector reductions at L2
-//          (fp32 sums; the order of the S additions per output is not fixed)
+//   GEMM2: Y = h[rows of e] . W2[e]^T, stored as bf16 rows [R, H] (the
+//          moe_grouped_ffn entry point) or, inside moe_forward, as fp16 rows
+//          scaled by a power of two per 32 columns (11 significant bits, same
+//          bytes as bf16) for the fp32 weighted combine that follows
 // E4M3 layers run kind::f8f6f4 with per-row activation scales and
 // per-output-channel weight scales applied in the epilogue (they factor out of
 // the K-sum).
@@ -62,13 +62,8 @@ struct TcParams {
     int out_ld;
     const float* row_scale; // E4M3: per-row activation scale [R]
     const float* col_scale; // E4M3: per-output-channel weight scale (s13 [E, 2I] or s2 [E, H])
-    // GEMM2 combine mode (out_acc != null): out_acc[f / S] += w * y_row with
-    // f = perm[row] (or row), w = slot_w[f] (or w_const); no y rows are written
-    float* out_acc;
-    const int32_t* perm;
-    int S;
-    const float* slot_w;
-    float w_const;
+    // GEMM2 with yexp != null: rows stored as fp16(v * 2^-k), k per 32 columns in yexp
+    int8_t* yexp;
     DevStatus* status;
     long long wait_limit;   // SM clock cycles per wait
     int inject_stall;       // testing hook: the producer never issues its loads
@@ -98,6 +93,32 @@ __device__ __forceinline__ TileInfo decode_tile(int id, const int* s_tile, const
     return t;
 }
 
+// One warp's 32 rows x 32 columns of 16-bit results (lane = row, packed[] = its
+// 64 bytes) go to global memory through a 2 KB shared-memory slice: written
+// with the 16-byte chunks of row r XOR-swizzled by (r >> 1) & 3 (conflict-free),
+// read back so that 4 lanes cover one row's 64 contiguous bytes (8 rows per
+// instruction); rows at or past row_end are not stored.
+__device__ __forceinline__ void stage_store(uint8_t* slice, const uint32_t (&packed)[16], int lane, uint16_t* out,
+                                            int ld, int row0, int row_end, int col0) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int pc = q ^ ((lane >> 1) & 3);
+        *reinterpret_cast<uint4*>(slice + lane * 64 + pc * 16) =
+            make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+    }
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int r = j * 8 + (lane >> 2);
+        const int c = lane & 3;
+        const uint4 v = *reinterpret_cast<const uint4*>(slice + r * 64 + ((c ^ ((r >> 1) & 3)) * 16));
+        const int grow = row0 + r;
+        if (grow < row_end)
+            *reinterpret_cast<uint4*>(out + static_cast<size_t>(grow) * ld + col0 + c * 8) = v;
+    }
+    __syncwarp();
+}
+
 // kBN: MMA N (GEMM1: gate half + up half; GEMM2: 256 output columns)
 template <bool kFp8, bool kGemm1, int kBN>
 __global__ void __launch_bounds__(TC_THREADS, 1)
@@ -120,6 +141,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     uint8_t* base = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
     uint8_t* sA = base;
     uint8_t* sB = base + TC_STAGES * TC_ABYTES;
+    uint8_t* sStage = sB + TC_STAGES * BBYTES;      // 4 epilogue warps x 2 KB
     volatile int* abort_flag = &s_abort;
 
     for (int i = threadIdx.x; i <= p.E; i += blockDim.x) {
@@ -153,32 +175,37 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
     if (warp == 0) {
         // ---------------------------------------------------------------- producer
-        if (lane == 0 && !p.inject_stall) {
+        // The whole warp walks the tiles; lane 0 waits and issues every load.
+        if (!p.inject_stall) {
             int stage = 0;
             uint32_t phase = 0;
             for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
                 const TileInfo t = decode_tile(tile, s_tile, s_off, p.E, p.n_tiles_n, p.bn_out);
-                bool ok = true;
-                for (int kb = 0; kb < p.k_blocks; ++kb) {
-                    if (!ptx::mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, p.wait_limit, p.status, 1u)) {
-                        ok = false;
-                        break;
+                int ok = 1;
+                if (lane == 0) {
+                    for (int kb = 0; kb < p.k_blocks; ++kb) {
+                        if (!ptx::mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, p.wait_limit, p.status, 1u)) {
+                            ok = 0;
+                            break;
+                        }
+                        ptx::mbar_arrive_expect_tx(&full_bar[stage], STAGE_TX);
+                        const int kx = kb * KEL;
+                        ptx::tma_load_2d(sA + stage * TC_ABYTES, &tmA, &full_bar[stage], kx, t.row0);
+                        if constexpr (kGemm1) {
+                            ptx::tma_load_3d(sB + stage * BBYTES, &tmB, &full_bar[stage], kx, t.n0, 2 * t.e);
+                            ptx::tma_load_3d(sB + stage * BBYTES + HALF * TC_ROWB, &tmB, &full_bar[stage], kx, t.n0,
+                                             2 * t.e + 1);
+                        } else {
+                            ptx::tma_load_2d(sB + stage * BBYTES, &tmB, &full_bar[stage], kx, t.e * p.H + t.n0);
+                        }
+                        if (++stage == TC_STAGES) { stage = 0; phase ^= 1u; }
                     }
-                    ptx::mbar_arrive_expect_tx(&full_bar[stage], STAGE_TX);
-                    const int kx = kb * KEL;
-                    ptx::tma_load_2d(sA + stage * TC_ABYTES, &tmA, &full_bar[stage], kx, t.row0);
-                    if constexpr (kGemm1) {
-                        ptx::tma_load_3d(sB + stage * BBYTES, &tmB, &full_bar[stage], kx, t.n0, 2 * t.e);
-                        ptx::tma_load_3d(sB + stage * BBYTES + HALF * TC_ROWB, &tmB, &full_bar[stage], kx, t.n0,
-                                         2 * t.e + 1);
-                    } else {
-                        ptx::tma_load_2d(sB + stage * BBYTES, &tmB, &full_bar[stage], kx, t.e * p.H + t.n0);
-                    }
-                    if (++stage == TC_STAGES) { stage = 0; phase ^= 1u; }
                 }
+                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+                __syncwarp();
                 if (!ok) break;
             }
-            if (*abort_flag) {
+            if (lane == 0 && *abort_flag) {
                 // let every copy in flight land before the CTA can exit: each
                 // stage's last armed phase completes when its bytes arrive
                 for (int s = 0; s < TC_STAGES; ++s) {
@@ -250,7 +277,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             const bool valid = row < t.row_end;
             const uint32_t tb = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + static_cast<uint32_t>(acc * 256);
             const float rs = (kFp8 && valid) ? p.row_scale[row] : 1.0f;
-            uint16_t* orow = p.out + static_cast<size_t>(valid ? row : 0) * p.out_ld + t.n0;
+            // 16-bit outputs leave through this warp's 2 KB staging slice so that
+            // global stores cover whole 64-byte row segments (see stage_store)
+            uint8_t* stage_w = sStage + (warp - 2) * 2048;
+            const int wrow0 = t.row0 + sub * 32;        // first tile row of this warp
             if constexpr (kGemm1) {
 #pragma unroll 1
                 for (int c = 0; c < HALF / 32; ++c) {
@@ -259,64 +289,59 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     ptx::tmem_ld_32x32b_x32(tb + HALF + c * 32, u);
                     ptx::tmem_ld_wait(g);
                     ptx::tmem_ld_wait(u);
-                    if (valid) {
-                        const float* sg = kFp8 ? p.col_scale + static_cast<size_t>(t.e) * 2 * p.I + t.n0 + c * 32 : nullptr;
-                        const float* su = kFp8 ? sg + p.I : nullptr;
-                        uint32_t packed[16];
+                    const float* sg = (kFp8 && valid) ? p.col_scale + static_cast<size_t>(t.e) * 2 * p.I + t.n0 + c * 32 : nullptr;
+                    const float* su = (kFp8 && valid) ? sg + p.I : nullptr;
+                    uint32_t packed[16];
 #pragma unroll
-                        for (int j = 0; j < 32; j += 2) {
-                            float g0 = __uint_as_float(g[j]), g1 = __uint_as_float(g[j + 1]);
-                            float u0 = __uint_as_float(u[j]), u1 = __uint_as_float(u[j + 1]);
-                            if constexpr (kFp8) {
+                    for (int j = 0; j < 32; j += 2) {
+                        float g0 = __uint_as_float(g[j]), g1 = __uint_as_float(g[j + 1]);
+                        float u0 = __uint_as_float(u[j]), u1 = __uint_as_float(u[j + 1]);
+                        if constexpr (kFp8) {
+                            if (valid) {
                                 g0 = g0 * rs * sg[j];
                                 g1 = g1 * rs * sg[j + 1];
                                 u0 = u0 * rs * su[j];
                                 u1 = u1 * rs * su[j + 1];
                             }
-                            packed[j >> 1] = pack_bf16x2(silu_f32(g0) * u0, silu_f32(g1) * u1);
                         }
-                        uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+                        packed[j >> 1] = pack_bf16x2(silu_f32(g0) * u0, silu_f32(g1) * u1);
                     }
+                    stage_store(stage_w, packed, lane, p.out, p.out_ld, wrow0, t.row_end, t.n0 + c * 32);
                 }
             } else {
-                float wrow = 1.0f;
-                float* arow = nullptr;
-                if (p.out_acc != nullptr && valid) {
-                    const int f = p.perm != nullptr ? p.perm[row] : row;
-                    wrow = p.slot_w != nullptr ? p.slot_w[f] : p.w_const;
-                    arow = p.out_acc + static_cast<size_t>(f / p.S) * p.H + t.n0;
-                }
+                uint64_t exps = 0;
 #pragma unroll 1
                 for (int c = 0; c < kBN / 32; ++c) {
                     uint32_t v[32];
                     ptx::tmem_ld_32x32b_x32(tb + c * 32, v);
                     ptx::tmem_ld_wait(v);
-                    if (valid) {
-                        const float* sc = kFp8 ? p.col_scale + static_cast<size_t>(t.e) * p.H + t.n0 + c * 32 : nullptr;
-                        float a[32];
+                    const float* sc = (kFp8 && valid) ? p.col_scale + static_cast<size_t>(t.e) * p.H + t.n0 + c * 32 : nullptr;
+                    float a[32];
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            a[j] = __uint_as_float(v[j]);
-                            if constexpr (kFp8) a[j] = a[j] * rs * sc[j];
-                        }
-                        if (arow != nullptr) {
-#pragma unroll
-                            for (int q = 0; q < 8; ++q)
-                                ptx::red_add_v4(arow + c * 32 + 4 * q, a[4 * q] * wrow, a[4 * q + 1] * wrow,
-                                                a[4 * q + 2] * wrow, a[4 * q + 3] * wrow);
-                        } else {
-                            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-                            for (int q = 0; q < 4; ++q)
-                                dst[q] = make_uint4(pack_bf16x2(a[8 * q], a[8 * q + 1]), pack_bf16x2(a[8 * q + 2], a[8 * q + 3]),
-                                                    pack_bf16x2(a[8 * q + 4], a[8 * q + 5]),
-                                                    pack_bf16x2(a[8 * q + 6], a[8 * q + 7]));
+                    for (int j = 0; j < 32; ++j) {
+                        a[j] = __uint_as_float(v[j]);
+                        if constexpr (kFp8) {
+                            if (valid) a[j] = a[j] * rs * sc[j];
                         }
                     }
+                    uint32_t packed[16];
+                    if (p.yexp != nullptr) {
+                        float amax = 0.0f;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(a[j]));
+                        const int k = f16_chunk_exp(amax);
+                        const float down = exp2_int(-k);
+#pragma unroll
+                        for (int j = 0; j < 32; j += 2) packed[j >> 1] = pack_f16x2(a[j] * down, a[j + 1] * down);
+                        exps |= static_cast<uint64_t>(static_cast<uint8_t>(static_cast<int8_t>(k))) << (8 * c);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; j += 2) packed[j >> 1] = pack_bf16x2(a[j], a[j + 1]);
+                    }
+                    stage_store(stage_w, packed, lane, p.out, p.out_ld, wrow0, t.row_end, t.n0 + c * 32);
                 }
+                if (p.yexp != nullptr && valid)
+                    *reinterpret_cast<uint64_t*>(p.yexp + static_cast<size_t>(row) * (p.H / 32) + t.n0 / 32) = exps;
             }
             ptx::tc_fence_before();
             ptx::mbar_arrive(&tempty_bar[acc]);
@@ -384,7 +409,7 @@ std::atomic<int> g_inject{0};
 template <bool kFp8, bool kGemm1, int kBN>
 cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const TcParams& p, cudaStream_t st,
                        const char* name) {
-    constexpr int smem = TC_STAGES * (TC_ABYTES + kBN * TC_ROWB) + 1024;
+    constexpr int smem = TC_STAGES * (TC_ABYTES + kBN * TC_ROWB) + 4 * 2048 + 1024;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
@@ -425,6 +450,16 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
     const int esz = fp8 ? 1 : 2;
     const int half = gemm1_half(a.I);
     const int kel = fp8 ? 128 : 64;
+    // rows of the grouped pass gathered from the token matrix (rows are the
+    // tokens themselves when perm is null)
+    const void* xp = a.xt;
+    const float* xp_scale = a.xt_scale;
+    if (a.perm != nullptr) {
+        const cudaError_t e = launch_gather_rows(a.R, a.S, a.H, esz, a.xt, a.xt_scale, a.perm, a.xp, a.xp_scale, st);
+        if (e != cudaSuccess) return e;
+        xp = a.xp;
+        xp_scale = a.xp_scale;
+    }
     int inject = 0;
     {
         int cur = g_inject.load();
@@ -433,7 +468,8 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
         inject = cur > 0 ? 1 : 0;
     }
 
-    // GEMM1: A = Xp [R, H]; B = W13 viewed as [2E][I][H] (gate/up halves separately clipped at I)
+    // GEMM1: A = Xp [R, H] (rows gathered by the gather kernel); B = W13 viewed as
+    // [2E][I][H] (gate/up halves separately clipped at I)
     CUtensorMap ta, tb;
     {
         const cuuint64_t ad[2] = {static_cast<cuuint64_t>(a.H), static_cast<cuuint64_t>(a.R)};
@@ -441,7 +477,7 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
         const cuuint64_t bd[3] = {static_cast<cuuint64_t>(a.H), static_cast<cuuint64_t>(a.I),
                                   static_cast<cuuint64_t>(2 * a.E)};
         const cuuint64_t bs[2] = {static_cast<cuuint64_t>(a.H) * esz, static_cast<cuuint64_t>(a.I) * a.H * esz};
-        if (!make_map(&ta, a.xp, fp8, 2, ad, as, TC_BM) || !make_map(&tb, a.w13, fp8, 3, bd, bs, half))
+        if (!make_map(&ta, xp, fp8, 2, ad, as, TC_BM) || !make_map(&tb, a.w13, fp8, 3, bd, bs, half))
             return cudaErrorInvalidValue;
     }
     TcParams p;
@@ -453,13 +489,9 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
     p.tile_off = a.tile_off;
     p.out = static_cast<uint16_t*>(a.h);
     p.out_ld = a.I;
-    p.row_scale = fp8 ? a.xp_scale : nullptr;
+    p.row_scale = fp8 ? xp_scale : nullptr;
     p.col_scale = fp8 ? a.s13 : nullptr;
-    p.out_acc = nullptr;
-    p.perm = nullptr;
-    p.S = 1;
-    p.slot_w = nullptr;
-    p.w_const = 0.0f;
+    p.yexp = nullptr;
     p.status = a.status;
     p.wait_limit = inject ? (20ll << 20) : (4ll << 30);
     p.inject_stall = inject;
@@ -488,11 +520,7 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
     p.out_ld = a.H;
     p.row_scale = fp8 ? a.h_scale : nullptr;
     p.col_scale = fp8 ? a.s2 : nullptr;
-    p.out_acc = a.out_acc;
-    p.perm = a.perm;
-    p.S = a.S;
-    p.slot_w = a.slot_w;
-    p.w_const = a.w_const;
+    p.yexp = a.yexp;
     return fp8 ? launch_one<true, false, 256>(ta, tb, p, st, "gemm2_tc")
                : launch_one<false, false, 256>(ta, tb, p, st, "gemm2_tc");
 }

@@ -17,10 +17,9 @@ struct ProfileScope {
 // ---- router (route.cu)
 int router_split_count(int T, int H);
 size_t router_partial_floats(int T, int H, int E);
-// zero_rows (optional): [T, H] fp32 rows the top-K kernel clears (the combine accumulator)
 cudaError_t launch_route(const moe_shape& s, const void* x, const float* wr, const float* bias,
                          int32_t* ids, float* wts, float* logits, float* partials, int shared_id,
-                         float* zero_rows, cudaStream_t st);
+                         cudaStream_t st);
 
 // ---- permutation (permute.cu)
 constexpr int kPermChunk = 512;      // flat slots per scatter chunk
@@ -42,23 +41,26 @@ cudaError_t launch_quant_rows(int rows, int cols, const uint16_t* in, uint8_t* c
 struct FfnArgs {
     int R, H, I, E;               // rows, hidden, intermediate, experts in this pass
     int act_dtype, w_dtype;
-    const void* xp;               // [R, H] gathered activations (act dtype, or E4M3 codes)
-    const float* xp_scale;        // [R] (E4M3)
+    // activations: the token matrix and how rows map to it
+    const void* xt;               // [T, H] x (act dtype) or its E4M3 codes
+    const float* xt_scale;        // [T] per-token E4M3 scale
+    int T;
+    const int32_t* perm;          // [R] row -> flat slot t*S + k; null: row r is token r
+    int S;
+    // CUDA-core path only: rows gathered from xt into xp before the GEMMs
+    void* xp;                     // [R, H] (act dtype, or E4M3 codes)
+    float* xp_scale;              // [R] (E4M3)
     const int32_t* offsets;       // [E+1]
     const int32_t* tile_off;      // [E+1] m-tile prefix (kTileM rows)
     const void* w13; const float* s13;
     const void* w2;  const float* s2;
     void* h;                      // [R, I] act dtype (bf16 or f32)
     uint8_t* hq; float* h_scale;  // [R, I] codes, [R] (E4M3)
-    void* y;                      // [R, H] act dtype (row-output mode)
-    // combine mode (out_acc != null): instead of writing y, GEMM2 adds
-    // w * y_row into out_acc[token] (fp32, [T, H]); token = f / S with
-    // f = perm[row] (perm == null: f = row); w = slot_w[f] (slot_w == null: w_const)
-    float* out_acc;
-    const int32_t* perm;
-    int S;
-    const float* slot_w;
-    float w_const;
+    void* y;                      // [R, H] expert rows: act dtype, or fp16 when yexp != null
+    // scaled-fp16 rows (yexp != null): y holds fp16(v * 2^-k) and
+    // yexp[r * H/32 + c] = k (int8), one power-of-two exponent per 32 columns,
+    // chosen so the chunk's largest |v| maps into [2^14, 2^15)
+    int8_t* yexp;
     int max_mtiles;               // upper bound of sum_e ceil(count_e / kTileM)
     DevStatus* status;
 };
@@ -72,11 +74,13 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t stream);
 void ffn_tc_inject_stall(int n_calls);
 
 // ---- combine (combine.cu)
-// out[t] = bf16(acc[t]) for the fp32 combine accumulator
-cudaError_t launch_round_rows(int T, int H, const float* acc, uint16_t* out, cudaStream_t stream);
 // out[t] = sum_k w[t,k] * y[inv[t*S+k]] (+ add_w * add[t] if add != null)
 cudaError_t launch_combine(int T, int S, int H, int act_dtype, const void* y, const int32_t* inv,
                            const float* w, const void* add, float add_w, void* out,
                            cudaStream_t stream);
+// same over scaled-fp16 rows (y16/yexp, add16/addexp as produced by the GEMM2 epilogue), bf16 out
+cudaError_t launch_combine_f16s(int T, int S, int H, const uint16_t* y16, const int8_t* yexp,
+                                const int32_t* inv, const float* w, const uint16_t* add16,
+                                const int8_t* addexp, float add_w, uint16_t* out, cudaStream_t stream);
 
 }  // namespace sre

@@ -150,8 +150,7 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ P, 
                                                    int K, int renormalize, int shared_id,
                                                    float shared_weight, int32_t* __restrict__ ids,
                                                    float* __restrict__ wts,
-                                                   float* __restrict__ logits_out,
-                                                   float* __restrict__ zero_rows, int H) {
+                                                   float* __restrict__ logits_out) {
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (warp >= T) return;
@@ -220,10 +219,6 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ P, 
         ids[static_cast<size_t>(t) * S + K] = shared_id;
         wts[static_cast<size_t>(t) * S + K] = shared_weight;
     }
-    if (zero_rows != nullptr) {
-        float4* z = reinterpret_cast<float4*>(zero_rows + static_cast<size_t>(t) * H);
-        for (int i = lane; i < H / 4; i += 32) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
 }
 
 }  // namespace
@@ -239,7 +234,7 @@ size_t router_partial_floats(int T, int H, int E) {
 
 cudaError_t launch_route(const moe_shape& s, const void* x, const float* wr, const float* bias,
                          int32_t* ids, float* wts, float* logits, float* partials, int shared_id,
-                         float* zero_rows, cudaStream_t st) {
+                         cudaStream_t st) {
     const int T = s.T, H = s.H, E = s.n_routed;
     const int split = router_split_count(T, H);
     dim3 grid(ceil_div(T, RT_BT), ceil_div(E, RT_BE), split);
@@ -255,8 +250,7 @@ cudaError_t launch_route(const moe_shape& s, const void* x, const float* wr, con
         ProfileScope ps("route_topk", st);
         topk_kernel<<<ceil_div(T * 32, 256), 256, 0, st>>>(partials, split, bias, T, E, s.top_k,
                                                           s.renormalize, shared_id,
-                                                          s.shared_weight, ids, wts, logits,
-                                                          zero_rows, H);
+                                                          s.shared_weight, ids, wts, logits);
         note_launch();
     }
     return cudaGetLastError();

@@ -130,3 +130,15 @@ def test_launch_counter_and_profile():
     assert _lib.moe_launch_count() - n0 >= 6
     n, ms = _lib.moe_profile_read("combine")
     assert n == 1 and ms > 0
+
+
+@pytest.mark.parametrize("name", ["bf16_small", "fp8_i192_zipf"])
+def test_forward_is_bit_deterministic(name):
+    """Routing, the permutation and the slot-ordered fp32 combine are all fixed
+    in order: two passes over the same inputs give the same bits."""
+    cfg = SMALL[name]
+    d = synth.to_device(synth.make_inputs(cfg), DEV)
+    layer = MoELayer(cfg, d)
+    a = layer.forward(d["x"]).clone()
+    b = layer.forward(d["x"]).clone()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
