@@ -181,6 +181,30 @@ void moe_profile_enable(int on);
 void moe_profile_reset(void);
 moe_status moe_profile_read(const char* name, int64_t* launches, double* total_ms);
 
+/* moe_permute without a workspace, for callers that cannot allocate device
+ * memory themselves: code whose device buffers all come from a host framework
+ * that owns every allocation and gives plugins no allocator; code that must not
+ * call cudaMalloc where it enqueues work (it may synchronise the device, and is
+ * not allowed while a stream is being captured); callers with a fixed device
+ * footprint. The method on the pages has no counterpart of this call; it is a
+ * deployment convenience.
+ * Arguments and results are those of moe_permute (ids [T, S] in, counts [E],
+ * offsets [E+1], perm [R], inv [R] out, all caller-owned device buffers); the
+ * kernels are the same. Their scratch lives in one 1 MiB array in the library's
+ * device globals, which every GPU that loads the library holds until the
+ * process exits. Limit: ceil(T*S / 512) * E <= 261888 (for 161 experts and 9
+ * slots, T <= 92501); larger calls return MOE_ERR_UNSUPPORTED before enqueuing
+ * anything. The library allocates nothing in this call.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture. All calls share the array and it keeps the last call's contents, so
+ * calls that overlap on the GPU (other streams, other host threads) race and
+ * must be serialised by the caller. Out-of-range ids are dropped as in
+ * moe_permute, but not reported: this call has no status word the caller can
+ * read. */
+moe_status moe_permute_noalloc(const moe_shape* shape, const int32_t* ids, int32_t* counts,
+                               int32_t* offsets, int32_t* perm, int32_t* inv, void* stream);
+
 /* Failure-injection hook for tests of the bounded waits: the next n_calls
  * grouped-FFN passes on the tensor-core path run with a TMA producer that never
  * issues its loads and a wait limit of about 10 ms, so their waits run out; the

@@ -20,7 +20,8 @@ DTYPES = {"f32": MOE_F32, "bf16": MOE_BF16, "e4m3": MOE_E4M3}
 EXPORTS = ("moe_workspace_size", "moe_route_topk", "moe_permute", "moe_grouped_ffn",
            "moe_combine", "moe_forward", "moe_quant_rows_e4m3", "moe_get_status",
            "moe_clear_status", "moe_status_string", "moe_launch_count", "moe_profile_enable",
-           "moe_profile_reset", "moe_profile_read", "moe_inject_wait_timeout")
+           "moe_profile_reset", "moe_profile_read", "moe_inject_wait_timeout",
+           "moe_permute_noalloc")
 
 
 class MoeError(RuntimeError):
@@ -74,6 +75,8 @@ def lib() -> C.CDLL:
         L.moe_profile_reset.argtypes = []
         L.moe_profile_read.restype = i
         L.moe_profile_read.argtypes = [C.c_char_p, C.POINTER(C.c_int64), C.POINTER(C.c_double)]
+        L.moe_permute_noalloc.restype = i
+        L.moe_permute_noalloc.argtypes = [S, p, p, p, p, p, p]
         L.moe_inject_wait_timeout.restype = None
         L.moe_inject_wait_timeout.argtypes = [i]
         _lib = L
@@ -155,6 +158,13 @@ def moe_forward(shape, x, router_w, router_bias, w13, s13, w2, s2, fuse_shared, 
     _check("moe_forward", lib().moe_forward(
         C.byref(shape), _p(x), _p(router_w), _p(router_bias), _p(w13), _p(s13), _p(w2), _p(s2),
         int(fuse_shared), _p(out), _p(ws), ws.numel(), impl, _stream(stream)))
+
+
+def moe_permute_noalloc(shape, ids, counts, offsets, perm, inv, stream=None):
+    """moe_permute for callers that cannot allocate: the library's own fixed
+    device scratch replaces the workspace (see include/moe.h)."""
+    _check("moe_permute_noalloc", lib().moe_permute_noalloc(
+        C.byref(shape), _p(ids), _p(counts), _p(offsets), _p(perm), _p(inv), _stream(stream)))
 
 
 def moe_quant_rows_e4m3(rows, cols, inp, codes, scales, stream=None):
