@@ -306,7 +306,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="prefill_bf16", choices=list(synth.CONFIGS))
-    ap.add_argument("--ffn", default="auto", choices=["auto", "simt", "tcgen05"])
+    ap.add_argument("--ffn", default="auto", choices=["auto", "simt", "tcgen05", "tcgen05_m128", "tcgen05_m256"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--quick", action="store_true",
@@ -328,7 +328,8 @@ def main():
     if args.tokens is not None or args.routed is not None:
         cfg = synth.variant(cfg, T=args.tokens or cfg.T, n_routed=args.routed or cfg.n_routed,
                             name=f"{cfg.name}[T={args.tokens or cfg.T},E_r={args.routed or cfg.n_routed}]")
-    impl = {"auto": _lib.MOE_FFN_AUTO, "simt": _lib.MOE_FFN_SIMT, "tcgen05": _lib.MOE_FFN_TCGEN05}[args.ffn]
+    impl = {"auto": _lib.MOE_FFN_AUTO, "simt": _lib.MOE_FFN_SIMT, "tcgen05": _lib.MOE_FFN_TCGEN05,
+            "tcgen05_m128": _lib.MOE_FFN_TCGEN05_M128, "tcgen05_m256": _lib.MOE_FFN_TCGEN05_M256}[args.ffn]
     d = synth.make_inputs(cfg, dist.device)
     stream = torch.cuda.current_stream(dist.device)
     fused = MoELayer(cfg, d, fuse_shared=True, impl=impl)
@@ -374,13 +375,26 @@ def main():
         ms_unf = time_steps(lambda: unfused.forward(d["x"], out), args.steps, args.warmup, dist, stream)
         del unfused
 
-        # end to end through the public API with pinned host buffers
+        # end to end through the public API with pinned host buffers: every step
+        # uploads its x and downloads its out; the pipelined submission overlaps
+        # one step's copies with its neighbours' compute
         x_host = d["x"].cpu().pin_memory()
-        out_host = torch.empty_like(x_host).pin_memory()
-        x_dev = torch.empty_like(d["x"])
-        ms_e2e = time_steps(lambda: fused.forward_host(x_host, out_host, x_dev, out), args.steps,
-                            args.warmup, dist, stream)
-
+        out_hosts = [torch.empty_like(x_host).pin_memory() for _ in range(2)]
+        for i in range(args.warmup):
+            fused.submit_host(x_host, out_hosts[i % 2])
+        fused.sync_host()
+        dist.barrier()
+        h2d, comp, d2h = fused.host_streams()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(h2d)
+        for i in range(args.steps):
+            fused.submit_host(x_host, out_hosts[i % 2])
+        e1.record(d2h)           # after the last download, which depends on every earlier step
+        fused.sync_host()
+        dist.barrier()
+        ms_e2e = dist.max(e0.elapsed_time(e1))
+        out_host = out_hosts[0]
     N = dist.world
     ms_step = ms / args.steps
     value = tokens_per_s(N, cfg.T, args.steps, ms)

@@ -74,8 +74,15 @@ typedef struct moe_shape {
 } moe_shape;
 
 /* Kernel choice for the expert GEMMs. AUTO picks the tcgen05 tensor-core
- * kernels for bf16/E4M3 weights and the CUDA-core kernels for fp32. */
-typedef enum moe_ffn_impl { MOE_FFN_AUTO = 0, MOE_FFN_SIMT = 1, MOE_FFN_TCGEN05 = 2 } moe_ffn_impl;
+ * kernels for bf16/E4M3 weights and the CUDA-core kernels for fp32. TCGEN05
+ * picks the tensor-core work unit itself: 256 rows (two 128-row tiles of one
+ * expert sharing each weight tile) for bf16 weights when groups average >= 192
+ * rows, else 128;
+ * TCGEN05_M128 / TCGEN05_M256 force one of them. */
+typedef enum moe_ffn_impl {
+    MOE_FFN_AUTO = 0, MOE_FFN_SIMT = 1, MOE_FFN_TCGEN05 = 2,
+    MOE_FFN_TCGEN05_M128 = 3, MOE_FFN_TCGEN05_M256 = 4
+} moe_ffn_impl;
 
 /* Bytes of workspace moe_forward needs for this shape (fused or not). The
  * other entry points need at most this much. Returns 0 for an invalid shape. */

@@ -71,5 +71,59 @@ class MoELayer:
             out_host.copy_(out_dev, non_blocking=True)
         return out_host
 
+    # ---- pipelined host-buffer submission -------------------------------------
+    # Batches that arrive in pinned host memory: each submit enqueues the upload
+    # on one copy stream, the layer on the compute stream and the download on a
+    # second copy stream, with `depth` device slots so that the copies of one
+    # batch overlap the layer of its neighbours. Every batch still makes its own
+    # host->device and device->host trip.
+
+    def _pipeline(self, depth: int, T: int):
+        key = (depth, T)
+        if getattr(self, "_pipe_key", None) != key:
+            dev = self.device
+            self._pipe = {
+                "h2d": torch.cuda.Stream(dev), "d2h": torch.cuda.Stream(dev),
+                "comp": torch.cuda.Stream(dev),
+                "x": [torch.empty(T, self.cfg.H, dtype=self.act_dtype, device=dev) for _ in range(depth)],
+                "out": [torch.empty(T, self.cfg.H, dtype=self.act_dtype, device=dev) for _ in range(depth)],
+                "up": [torch.cuda.Event() for _ in range(depth)],      # upload done
+                "done": [torch.cuda.Event() for _ in range(depth)],    # layer done (x slot free)
+                "down": [torch.cuda.Event() for _ in range(depth)],    # download done (out slot free)
+                "used": [False] * depth, "next": 0, "depth": depth,
+            }
+            self._pipe_key = key
+        return self._pipe
+
+    def submit_host(self, x_host: torch.Tensor, out_host: torch.Tensor, depth: int = 2) -> None:
+        """Enqueue one batch: pinned x_host [T, H] in, pinned out_host [T, H] out.
+        Returns at once; call sync_host() before reading out_host."""
+        P = self._pipeline(depth, x_host.shape[0])
+        i = P["next"]
+        P["next"] = (i + 1) % P["depth"]
+        if P["used"][i]:
+            P["h2d"].wait_event(P["done"][i])       # the layer finished reading slot i's x
+            P["comp"].wait_event(P["down"][i])      # the download finished reading slot i's out
+        P["used"][i] = True
+        with torch.cuda.stream(P["h2d"]):
+            P["x"][i].copy_(x_host, non_blocking=True)
+            P["up"][i].record(P["h2d"])
+        P["comp"].wait_event(P["up"][i])
+        self.forward(P["x"][i], P["out"][i], stream=P["comp"])
+        P["done"][i].record(P["comp"])
+        P["d2h"].wait_event(P["done"][i])
+        with torch.cuda.stream(P["d2h"]):
+            out_host.copy_(P["out"][i], non_blocking=True)
+            P["down"][i].record(P["d2h"])
+
+    def host_streams(self):
+        """(upload, compute, download) streams of the pipelined path."""
+        P = self._pipe
+        return P["h2d"], P["comp"], P["d2h"]
+
+    def sync_host(self) -> None:
+        for s in self.host_streams():
+            s.synchronize()
+
     def status(self) -> int:
         return moe_get_status(self.ws)

@@ -61,6 +61,7 @@ struct FfnArgs {
     // yexp[r * H/32 + c] = k (int8), one power-of-two exponent per 32 columns,
     // chosen so the chunk's largest |v| maps into [2^14, 2^15)
     int8_t* yexp;
+    int unit_rows;                // tensor-core work unit: 0 auto, 128 or 256 rows
     int max_mtiles;               // upper bound of sum_e ceil(count_e / kTileM)
     DevStatus* status;
 };

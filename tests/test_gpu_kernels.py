@@ -9,7 +9,8 @@ import torch
 
 import oracle
 from shared_routed_expert_b200 import _lib, build, synth
-from shared_routed_expert_b200._lib import MOE_FFN_SIMT, MOE_FFN_TCGEN05
+from shared_routed_expert_b200._lib import (MOE_FFN_SIMT, MOE_FFN_TCGEN05, MOE_FFN_TCGEN05_M128,
+                                            MOE_FFN_TCGEN05_M256)
 from tests.parity_util import oracle_logits, rel_err, to_f64, tol_of
 
 pytestmark = pytest.mark.gpu
@@ -157,11 +158,15 @@ FFN_CASES = {
 }
 
 
+IMPLS = [MOE_FFN_SIMT, MOE_FFN_TCGEN05_M128, MOE_FFN_TCGEN05_M256]
+IMPL_IDS = ["simt", "tcgen05_m128", "tcgen05_m256"]
+
+
 @pytest.mark.parametrize("name", list(FFN_CASES))
-@pytest.mark.parametrize("impl", [MOE_FFN_SIMT, MOE_FFN_TCGEN05], ids=["simt", "tcgen05"])
+@pytest.mark.parametrize("impl", IMPLS, ids=IMPL_IDS)
 def test_grouped_ffn_rows_match_oracle(name, impl):
     cfg = FFN_CASES[name]
-    if impl == MOE_FFN_TCGEN05 and cfg.w_dtype == "f32":
+    if impl != MOE_FFN_SIMT and cfg.w_dtype == "f32":
         pytest.skip("tensor-core path is for bf16/E4M3 weights")
     inp = synth.make_inputs(cfg)
     d = synth.to_device(inp, DEV)
@@ -185,7 +190,7 @@ def test_grouped_ffn_rows_match_oracle(name, impl):
 
 
 @pytest.mark.parametrize("w_dtype", ["bf16", "e4m3"])
-@pytest.mark.parametrize("impl", [MOE_FFN_SIMT, MOE_FFN_TCGEN05], ids=["simt", "tcgen05"])
+@pytest.mark.parametrize("impl", IMPLS, ids=IMPL_IDS)
 def test_grouped_ffn_ragged_group_sizes(w_dtype, impl):
     """Expert groups of 0, 1, 127, 128, 129 and 300 rows: empty groups, single
     rows and tails one row either side of the 128-row tile."""

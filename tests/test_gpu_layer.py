@@ -61,7 +61,9 @@ def test_forward_small_matches_oracle(name):
 def test_forward_simt_and_tensor_core_paths_agree(name):
     cfg = SMALL[name]
     d = synth.to_device(synth.make_inputs(cfg), DEV)
-    assert rel_err(_run(cfg, d, True, MOE_FFN_SIMT), _run(cfg, d, True, MOE_FFN_AUTO)) <= tol_of(cfg)
+    simt = _run(cfg, d, True, MOE_FFN_SIMT)
+    for impl in (_lib.MOE_FFN_TCGEN05_M128, _lib.MOE_FFN_TCGEN05_M256):
+        assert rel_err(simt, _run(cfg, d, True, impl)) <= tol_of(cfg)
 
 
 def test_zero_router_routes_everything_to_the_lowest_ids():
@@ -142,3 +144,20 @@ def test_forward_is_bit_deterministic(name):
     a = layer.forward(d["x"]).clone()
     b = layer.forward(d["x"]).clone()
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_pipelined_host_submission_matches_forward():
+    """Host batches through submit_host (upload, layer, download on three
+    streams, two device slots) give exactly what forward gives, batch by batch."""
+    cfg = SMALL["bf16_small"]
+    d = synth.to_device(synth.make_inputs(cfg), DEV)
+    layer = MoELayer(cfg, d)
+    g = torch.Generator().manual_seed(9)
+    xs = [torch.randn(cfg.T, cfg.H, generator=g).to(torch.bfloat16).pin_memory() for _ in range(5)]
+    outs = [torch.empty_like(x).pin_memory() for x in xs]
+    for x, o in zip(xs, outs):
+        layer.submit_host(x, o)
+    layer.sync_host()
+    for x, o in zip(xs, outs):
+        ref = layer.forward(x.to(DEV)).cpu()
+        assert torch.equal(o.view(torch.int16), ref.view(torch.int16))
