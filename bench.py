@@ -332,6 +332,7 @@ def main():
                     help="only the fused device-timed region (for ncu launch lists and captures)")
     ap.add_argument("--tokens", type=int, default=None, help="override T (smaller profiling case)")
     ap.add_argument("--routed", type=int, default=None, help="override the routed expert count")
+    ap.add_argument("--inter", type=int, default=None, help="override I (smaller profiling case)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -344,9 +345,11 @@ def main():
 
     build.build()
     cfg = synth.CONFIGS[args.workload]
-    if args.tokens is not None or args.routed is not None:
+    if args.tokens is not None or args.routed is not None or args.inter is not None:
         cfg = synth.variant(cfg, T=args.tokens or cfg.T, n_routed=args.routed or cfg.n_routed,
-                            name=f"{cfg.name}[T={args.tokens or cfg.T},E_r={args.routed or cfg.n_routed}]")
+                            I=args.inter or cfg.I,
+                            name=f"{cfg.name}[T={args.tokens or cfg.T},E_r={args.routed or cfg.n_routed},"
+                                 f"I={args.inter or cfg.I}]")
     impl = {"auto": _lib.MOE_FFN_AUTO, "simt": _lib.MOE_FFN_SIMT, "tcgen05": _lib.MOE_FFN_TCGEN05,
             "tcgen05_m128": _lib.MOE_FFN_TCGEN05_M128, "tcgen05_m256": _lib.MOE_FFN_TCGEN05_M256}[args.ffn]
     d = synth.make_inputs(cfg, dist.device)

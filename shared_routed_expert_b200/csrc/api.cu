@@ -227,6 +227,7 @@ FfnArgs ffn_args(const moe_shape& s, const Dims& d, const Layout& L, void* ws, c
     a.y = y;
     a.yexp = nullptr;
     a.unit_rows = 0;
+    a.direct_e = -1;
     a.max_mtiles = d.R / kTileM + d.E;
     a.status = at<DevStatus>(ws, L.status);
     return a;
@@ -363,6 +364,9 @@ moe_status moe_forward(const moe_shape* shape, const void* x, const float* route
         FfnArgs a = ffn_args(*shape, d, L, ws, xt, xt_scale, at<int32_t>(ws, L.perm), w13, s13, w2, s2,
                              at<void>(ws, L.y));
         a.yexp = f32_act ? nullptr : at<int8_t>(ws, L.yexp);
+        // fused layout: the shared expert's group is every token in order (stable
+        // permutation, shared id last), so its rows need no gather
+        a.direct_e = (fused && d.shared) ? d.E - 1 : -1;
         err = run_ffn(a, ffn_impl, st);
     }
 
@@ -393,6 +397,7 @@ moe_status moe_forward(const moe_shape* shape, const void* x, const float* route
         a.y = at<void>(ws, L.sh_y);
         a.yexp = f32_act ? nullptr : at<int8_t>(ws, L.sh_yexp);
         a.unit_rows = 0;
+        a.direct_e = -1;
         a.max_mtiles = ceil_div(d.T, kTileM);
         a.status = at<DevStatus>(ws, L.status);
         dense_offsets_kernel<<<1, 1, 0, st>>>(d.T, at<int32_t>(ws, L.sh_off), at<int32_t>(ws, L.sh_tile));

@@ -248,7 +248,7 @@ cudaError_t launch_ffn_simt(const FfnArgs& in, cudaStream_t stream) {
     if (a.perm != nullptr) {
         // rows of the grouped pass gathered from the token matrix
         const int eb = (a.w_dtype == MOE_E4M3) ? 1 : (a.act_dtype == MOE_F32 ? 4 : 2);
-        cudaError_t err = launch_gather_rows(a.R, a.S, a.H, eb, a.xt, a.xt_scale, a.perm, a.xp, a.xp_scale, stream);
+        cudaError_t err = launch_gather_rows(a.R, a.S, a.H, eb, a.xt, a.xt_scale, a.perm, a.xp, a.xp_scale, nullptr, stream);
         if (err != cudaSuccess) return err;
     } else {
         a.xp = const_cast<void*>(a.xt);           // row r is token r

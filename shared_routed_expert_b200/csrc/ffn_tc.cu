@@ -45,9 +45,10 @@ namespace sre {
 namespace {
 
 constexpr int TC_BM = 128;
-constexpr int TC_STAGES = 4;
-constexpr int TC_ROWB = 128;                       // bytes of K per row per stage
-constexpr int TC_ABYTES = TC_BM * TC_ROWB;         // 16 KB
+constexpr int TC_RING_BYTES = 192 * 1024;          // shared memory for the stage ring
+#ifndef SRE_STAGE_ROW_BYTES
+#define SRE_STAGE_ROW_BYTES 128
+#endif
 constexpr int TC_MAXE = 260;
 constexpr uint32_t TC_TMEM_COLS = 512;
 
@@ -61,6 +62,8 @@ struct TcParams {
     uint16_t* out;          // GEMM1: h [R, I]; GEMM2: y [R, H] (bf16)
     int out_ld;
     const float* row_scale; // E4M3: per-row activation scale [R]
+    int direct_e;           // GEMM1: expert whose A rows are read from the token matrix (tmA2), or -1
+    const float* direct_scale;  // E4M3: per-token scale of that expert's rows
     const float* col_scale; // E4M3: per-output-channel weight scale (s13 [E, 2I] or s2 [E, H])
     // GEMM2 with yexp != null: rows stored as fp16(v * 2^-k), k per 32 columns in yexp
     int8_t* yexp;
@@ -133,16 +136,28 @@ __device__ __forceinline__ void stage_store(uint8_t* slice, const uint32_t (&pac
 // drain them 4 per accumulator. Otherwise a unit is one m-tile, the two TMEM
 // buffers alternate between units, and the 8 epilogue warps split each tile's
 // columns in two halves (two warps per TMEM sub-partition).
-template <bool kFp8, bool kGemm1, int kBN, bool kPair>
+// kRowB: bytes of K per row per stage (128: 128-byte swizzle; 64: 64-byte swizzle,
+// twice as many stages of half the size).
+template <int kRowB, int kBN, bool kPair>
+struct Ring {
+    static constexpr int A_TILE = TC_BM * kRowB;
+    static constexpr int STAGE = (kPair ? 2 : 1) * A_TILE + kBN * kRowB;
+    static constexpr int N = (TC_RING_BYTES / STAGE) > 8 ? 8 : (TC_RING_BYTES / STAGE);
+    static constexpr int SMEM = N * STAGE + 8 * 2048 + 1024;   // + epilogue staging + alignment
+};
+
+template <bool kFp8, bool kGemm1, int kBN, bool kPair, int kRowB>
 __global__ void __launch_bounds__(320, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                        const TcParams p) {
-    constexpr int NSTAGE = kPair ? 3 : TC_STAGES;
-    constexpr int A_TILES = kPair ? 2 : 1;
-    constexpr int ABYTES = A_TILES * TC_ABYTES;     // A bytes per stage
-    constexpr int BBYTES = kBN * TC_ROWB;
+                        const __grid_constant__ CUtensorMap tmA2, const TcParams p) {
+    using RG = Ring<kRowB, kBN, kPair>;
+    constexpr int NSTAGE = RG::N;
+    constexpr int TC_ABYTES = RG::A_TILE;           // one 128-row A tile per stage
+    constexpr int ABYTES = (kPair ? 2 : 1) * TC_ABYTES;
+    constexpr int BBYTES = kBN * kRowB;
     constexpr int HALF = kBN / 2;
-    constexpr int KEL = kFp8 ? 128 : 64;            // K elements per stage
+    constexpr int KEL = kFp8 ? kRowB : kRowB / 2;   // K elements per stage
+    constexpr int KSTEPS = kRowB / 32;              // MMAs (32 bytes of K each) per stage
     constexpr int EPI_WARPS = 8;
     constexpr uint32_t IDESC = ptx::instr_desc(TC_BM, kBN, kFp8 ? 0u : 1u);
 
@@ -195,6 +210,7 @@ __global__ void __launch_bounds__(320, 1)
         ptx::fence_mbar_init();
         ptx::prefetch_tmap(&tmA);
         ptx::prefetch_tmap(&tmB);
+        if (p.direct_e >= 0) ptx::prefetch_tmap(&tmA2);
     }
     if (warp == 1) {
         ptx::tmem_alloc(&s_tmem, TC_TMEM_COLS);
@@ -224,12 +240,16 @@ __global__ void __launch_bounds__(320, 1)
                         }
                         ptx::mbar_arrive_expect_tx(&full_bar[stage], tx);
                         const int kx = kb * KEL;
-                        ptx::tma_load_2d(sA + stage * ABYTES, &tmA, &full_bar[stage], kx, t.row0);
+                        // A rows: gathered copy, or the token matrix itself for the direct group
+                        const bool direct = t.e == p.direct_e;
+                        const CUtensorMap* am = direct ? &tmA2 : &tmA;
+                        const int ar = direct ? t.row0 - s_off[t.e] : t.row0;
+                        ptx::tma_load_2d(sA + stage * ABYTES, am, &full_bar[stage], kx, ar);
                         if (t.two)
-                            ptx::tma_load_2d(sA + stage * ABYTES + TC_ABYTES, &tmA, &full_bar[stage], kx, t.row0 + TC_BM);
+                            ptx::tma_load_2d(sA + stage * ABYTES + TC_ABYTES, am, &full_bar[stage], kx, ar + TC_BM);
                         if constexpr (kGemm1) {
                             ptx::tma_load_3d(sB + stage * BBYTES, &tmB, &full_bar[stage], kx, t.n0, 2 * t.e);
-                            ptx::tma_load_3d(sB + stage * BBYTES + HALF * TC_ROWB, &tmB, &full_bar[stage], kx, t.n0,
+                            ptx::tma_load_3d(sB + stage * BBYTES + HALF * kRowB, &tmB, &full_bar[stage], kx, t.n0,
                                              2 * t.e + 1);
                         } else {
                             ptx::tma_load_2d(sB + stage * BBYTES, &tmB, &full_bar[stage], kx, t.e * p.H + t.n0);
@@ -278,13 +298,13 @@ __global__ void __launch_bounds__(320, 1)
                     const uint32_t a_addr = ptx::smem_u32(sA + stage * ABYTES);
                     const uint32_t b_addr = ptx::smem_u32(sB + stage * BBYTES);
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const uint64_t ad = ptx::smem_desc_sw128(a_addr + k * 32);
-                        const uint64_t bd = ptx::smem_desc_sw128(b_addr + k * 32);
+                    for (int k = 0; k < KSTEPS; ++k) {
+                        const uint64_t ad = ptx::smem_desc_sw<kRowB>(a_addr + k * 32);
+                        const uint64_t bd = ptx::smem_desc_sw<kRowB>(b_addr + k * 32);
                         if constexpr (kFp8) ptx::mma_f8(d0, ad, bd, IDESC, (kb | k) != 0);
                         else ptx::mma_f16(d0, ad, bd, IDESC, (kb | k) != 0);
                         if (kPair && two) {
-                            const uint64_t ad1 = ptx::smem_desc_sw128(a_addr + TC_ABYTES + k * 32);
+                            const uint64_t ad1 = ptx::smem_desc_sw<kRowB>(a_addr + TC_ABYTES + k * 32);
                             if constexpr (kFp8) ptx::mma_f8(d1, ad1, bd, IDESC, (kb | k) != 0);
                             else ptx::mma_f16(d1, ad1, bd, IDESC, (kb | k) != 0);
                         }
@@ -331,7 +351,9 @@ __global__ void __launch_bounds__(320, 1)
             const bool valid = active && row < t.row_end;
             const uint32_t tb = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) +
                                 static_cast<uint32_t>(kPair ? eg * 256 : acc * 256);
-            const float rs = (kFp8 && valid) ? p.row_scale[row] : 1.0f;
+            float rs = 1.0f;
+            if (kFp8 && valid)
+                rs = (t.e == p.direct_e) ? p.direct_scale[row - s_off[t.e]] : p.row_scale[row];
             if (active) {
             // 16-bit outputs leave through this warp's 2 KB staging slice so that
             // global stores cover whole 64-byte row segments (see stage_store)
@@ -454,16 +476,18 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// rank-2/3 K-major map with a {128 bytes of K, box_rows[, 1]} box and 128-byte swizzle
+// rank-2/3 K-major map with a {row_bytes of K, box_rows[, 1]} box and the
+// swizzle of that width (128 or 64 bytes)
 bool make_map(CUtensorMap* m, const void* ptr, bool fp8, int rank, const cuuint64_t* dims,
-              const cuuint64_t* strides_bytes, cuuint32_t box_rows) {
+              const cuuint64_t* strides_bytes, cuuint32_t box_rows, int row_bytes) {
     EncodeTiledFn fn = encode_fn();
     if (fn == nullptr) return false;
-    const cuuint32_t box[3] = {static_cast<cuuint32_t>(fp8 ? 128 : 64), box_rows, 1};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(fp8 ? row_bytes : row_bytes / 2), box_rows, 1};
     const cuuint32_t es[3] = {1, 1, 1};
     const CUresult r = fn(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                           static_cast<cuuint32_t>(rank), const_cast<void*>(ptr), dims, strides_bytes, box, es,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -484,30 +508,29 @@ int gemm1_half(int I) {
 std::atomic<int> g_inject{0};
 
 template <bool kFp8, bool kGemm1, int kBN, bool kPair>
-cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const TcParams& p, cudaStream_t st,
-                       const char* name) {
-    constexpr int nstage = kPair ? 3 : TC_STAGES;
-    constexpr int smem = nstage * ((kPair ? 2 : 1) * TC_ABYTES + kBN * TC_ROWB) + 8 * 2048 + 1024;
-    constexpr int threads = 320;
+cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2, const TcParams& p,
+                       cudaStream_t st, const char* name) {
+    constexpr int kRowB = SRE_STAGE_ROW_BYTES;
+    constexpr int smem = Ring<kRowB, kBN, kPair>::SMEM;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(grouped_gemm_kernel<kFp8, kGemm1, kBN, kPair>,
+        attr_err = cudaFuncSetAttribute(grouped_gemm_kernel<kFp8, kGemm1, kBN, kPair, kRowB>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     });
     if (attr_err != cudaSuccess) return attr_err;
     ProfileScope ps(name, st);
-    grouped_gemm_kernel<kFp8, kGemm1, kBN, kPair><<<num_sms(), threads, smem, st>>>(a, b, p);
+    grouped_gemm_kernel<kFp8, kGemm1, kBN, kPair, kRowB><<<num_sms(), 320, smem, st>>>(a, b, a2, p);
     note_launch();
     return cudaGetLastError();
 }
 
 template <bool kFp8, bool kPair>
-cudaError_t launch_gemm1(const CUtensorMap& a, const CUtensorMap& b, const TcParams& p, int half,
-                         cudaStream_t st) {
-    if (half == 128) return launch_one<kFp8, true, 256, kPair>(a, b, p, st, "gemm1_tc");
-    if (half == 96) return launch_one<kFp8, true, 192, kPair>(a, b, p, st, "gemm1_tc");
-    return launch_one<kFp8, true, 128, kPair>(a, b, p, st, "gemm1_tc");
+cudaError_t launch_gemm1(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2, const TcParams& p,
+                         int half, cudaStream_t st) {
+    if (half == 128) return launch_one<kFp8, true, 256, kPair>(a, b, a2, p, st, "gemm1_tc");
+    if (half == 96) return launch_one<kFp8, true, 192, kPair>(a, b, a2, p, st, "gemm1_tc");
+    return launch_one<kFp8, true, 128, kPair>(a, b, a2, p, st, "gemm1_tc");
 }
 
 }  // namespace
@@ -528,13 +551,17 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
     const bool fp8 = a.w_dtype == MOE_E4M3;
     const int esz = fp8 ? 1 : 2;
     const int half = gemm1_half(a.I);
-    const int kel = fp8 ? 128 : 64;
+    constexpr int kRowBytes = SRE_STAGE_ROW_BYTES;
+    const int kel = fp8 ? kRowBytes : kRowBytes / 2;
     // rows of the grouped pass gathered from the token matrix (rows are the
     // tokens themselves when perm is null)
     const void* xp = a.xt;
     const float* xp_scale = a.xt_scale;
     if (a.perm != nullptr) {
-        const cudaError_t e = launch_gather_rows(a.R, a.S, a.H, esz, a.xt, a.xt_scale, a.perm, a.xp, a.xp_scale, st);
+        // the direct group's rows are not copied: GEMM1 reads them from xt
+        const int32_t* skip = a.direct_e >= 0 ? a.offsets + a.direct_e : nullptr;
+        const cudaError_t e = launch_gather_rows(a.R, a.S, a.H, esz, a.xt, a.xt_scale, a.perm, a.xp, a.xp_scale,
+                                                 skip, st);
         if (e != cudaSuccess) return e;
         xp = a.xp;
         xp_scale = a.xp_scale;
@@ -556,8 +583,16 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
         const cuuint64_t bd[3] = {static_cast<cuuint64_t>(a.H), static_cast<cuuint64_t>(a.I),
                                   static_cast<cuuint64_t>(2 * a.E)};
         const cuuint64_t bs[2] = {static_cast<cuuint64_t>(a.H) * esz, static_cast<cuuint64_t>(a.I) * a.H * esz};
-        if (!make_map(&ta, xp, fp8, 2, ad, as, TC_BM) || !make_map(&tb, a.w13, fp8, 3, bd, bs, half))
+        if (!make_map(&ta, xp, fp8, 2, ad, as, TC_BM, kRowBytes) || !make_map(&tb, a.w13, fp8, 3, bd, bs, half, kRowBytes))
             return cudaErrorInvalidValue;
+    }
+    // the direct group's A: the token matrix [T, H]
+    CUtensorMap ta2 = ta;
+    const int direct_e = (a.perm != nullptr) ? a.direct_e : -1;
+    if (direct_e >= 0) {
+        const cuuint64_t ad[2] = {static_cast<cuuint64_t>(a.H), static_cast<cuuint64_t>(a.T)};
+        const cuuint64_t as[1] = {static_cast<cuuint64_t>(a.H) * esz};
+        if (!make_map(&ta2, a.xt, fp8, 2, ad, as, TC_BM, kRowBytes)) return cudaErrorInvalidValue;
     }
     TcParams p;
     p.E = a.E; p.H = a.H; p.I = a.I;
@@ -569,6 +604,8 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
     p.out = static_cast<uint16_t*>(a.h);
     p.out_ld = a.I;
     p.row_scale = fp8 ? xp_scale : nullptr;
+    p.direct_e = direct_e;
+    p.direct_scale = fp8 ? a.xt_scale : nullptr;
     p.col_scale = fp8 ? a.s13 : nullptr;
     p.yexp = nullptr;
     p.status = a.status;
@@ -580,10 +617,10 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
     // faster with 128-row units (prefill_fp8 4.95 vs 6.04 ms, skewed_fp8 0.84 vs 0.99 ms).
     const bool pair = a.unit_rows == 256 ||
                       (a.unit_rows == 0 && a.w_dtype == MOE_BF16 && a.R >= 192 * a.E);
-    cudaError_t err = fp8 ? (pair ? launch_gemm1<true, true>(ta, tb, p, half, st)
-                                  : launch_gemm1<true, false>(ta, tb, p, half, st))
-                          : (pair ? launch_gemm1<false, true>(ta, tb, p, half, st)
-                                  : launch_gemm1<false, false>(ta, tb, p, half, st));
+    cudaError_t err = fp8 ? (pair ? launch_gemm1<true, true>(ta, tb, ta2, p, half, st)
+                                  : launch_gemm1<true, false>(ta, tb, ta2, p, half, st))
+                          : (pair ? launch_gemm1<false, true>(ta, tb, ta2, p, half, st)
+                                  : launch_gemm1<false, false>(ta, tb, ta2, p, half, st));
     if (err != cudaSuccess) return err;
 
     const void* hA = a.h;
@@ -598,7 +635,7 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
         const cuuint64_t as[1] = {static_cast<cuuint64_t>(a.I) * esz};
         const cuuint64_t bd[2] = {static_cast<cuuint64_t>(a.I), static_cast<cuuint64_t>(a.E) * a.H};
         const cuuint64_t bs[1] = {static_cast<cuuint64_t>(a.I) * esz};
-        if (!make_map(&ta, hA, fp8, 2, ad, as, TC_BM) || !make_map(&tb, a.w2, fp8, 2, bd, bs, 256))
+        if (!make_map(&ta, hA, fp8, 2, ad, as, TC_BM, kRowBytes) || !make_map(&tb, a.w2, fp8, 2, bd, bs, 256, kRowBytes))
             return cudaErrorInvalidValue;
     }
     p.n_tiles_n = a.H / 256;
@@ -607,13 +644,14 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
     p.out = static_cast<uint16_t*>(a.y);
     p.out_ld = a.H;
     p.row_scale = fp8 ? a.h_scale : nullptr;
+    p.direct_e = -1;
     p.col_scale = fp8 ? a.s2 : nullptr;
     p.yexp = a.yexp;
     if (fp8)
-        return pair ? launch_one<true, false, 256, true>(ta, tb, p, st, "gemm2_tc")
-                    : launch_one<true, false, 256, false>(ta, tb, p, st, "gemm2_tc");
-    return pair ? launch_one<false, false, 256, true>(ta, tb, p, st, "gemm2_tc")
-                : launch_one<false, false, 256, false>(ta, tb, p, st, "gemm2_tc");
+        return pair ? launch_one<true, false, 256, true>(ta, tb, ta, p, st, "gemm2_tc")
+                    : launch_one<true, false, 256, false>(ta, tb, ta, p, st, "gemm2_tc");
+    return pair ? launch_one<false, false, 256, true>(ta, tb, ta, p, st, "gemm2_tc")
+                : launch_one<false, false, 256, false>(ta, tb, ta, p, st, "gemm2_tc");
 }
 
 }  // namespace sre

@@ -29,10 +29,12 @@ size_t permute_scratch_ints(int R, int E);
 cudaError_t launch_permute(int R, int E, const int32_t* ids, int32_t* counts, int32_t* offsets,
                            int32_t* perm, int32_t* inv, int32_t* tile_off, int32_t* scratch,
                            DevStatus* st, cudaStream_t stream);
-// Xp[r] = x[perm[r] / S] (bf16 or fp32 rows, or E4M3 codes + per-row scale)
+// Xp[r] = x[perm[r] / S] (bf16 or fp32 rows, or E4M3 codes + per-row scale);
+// rows in [skip[0], skip[1]) are left out when skip != null (a group whose rows
+// the GEMM reads from x directly)
 cudaError_t launch_gather_rows(int R, int S, int H, int elem_bytes, const void* x,
                                const float* xscale, const int32_t* perm, void* xp, float* xpscale,
-                               cudaStream_t stream);
+                               const int32_t* skip, cudaStream_t stream);
 // per-row E4M3 quantisation of bf16 rows
 cudaError_t launch_quant_rows(int rows, int cols, const uint16_t* in, uint8_t* codes,
                               float* scales, cudaStream_t stream);
@@ -62,6 +64,8 @@ struct FfnArgs {
     // chosen so the chunk's largest |v| maps into [2^14, 2^15)
     int8_t* yexp;
     int unit_rows;                // tensor-core work unit: 0 auto, 128 or 256 rows
+    int direct_e;                 // expert whose rows are tokens 0..T-1 in order (A read from
+                                  // xt directly, not gathered), or -1
     int max_mtiles;               // upper bound of sum_e ceil(count_e / kTileM)
     DevStatus* status;
 };

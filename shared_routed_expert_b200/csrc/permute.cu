@@ -152,10 +152,12 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(int R, int S, int row_
                                                           const float* __restrict__ xscale,
                                                           const int32_t* __restrict__ perm,
                                                           uint4* __restrict__ xp,
-                                                          float* __restrict__ xpscale) {
+                                                          float* __restrict__ xpscale,
+                                                          const int32_t* __restrict__ skip) {
     const int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (r >= R) return;
+    if (skip != nullptr && r >= skip[0] && r < skip[1]) return;
     const int f = perm[r];
     if (f < 0 || f >= R) return;          // a slot dropped for a bad id leaves no row
     const int t = f / S;
@@ -236,12 +238,12 @@ cudaError_t launch_permute(int R, int E, const int32_t* ids, int32_t* counts, in
 
 cudaError_t launch_gather_rows(int R, int S, int H, int elem_bytes, const void* x,
                                const float* xscale, const int32_t* perm, void* xp, float* xpscale,
-                               cudaStream_t stream) {
+                               const int32_t* skip, cudaStream_t stream) {
     if (R == 0) return cudaSuccess;
     const int row_vecs = H * elem_bytes / 16;
     ProfileScope ps("gather", stream);
     gather_rows_kernel<<<ceil_div(R * 32, 256), 256, 0, stream>>>(
-        R, S, row_vecs, static_cast<const uint4*>(x), xscale, perm, static_cast<uint4*>(xp), xpscale);
+        R, S, row_vecs, static_cast<const uint4*>(x), xscale, perm, static_cast<uint4*>(xp), xpscale, skip);
     note_launch();
     return cudaGetLastError();
 }

@@ -170,20 +170,22 @@ __device__ __forceinline__ void red_add_v4(float* out, float a, float b, float c
 }
 
 // ------------------------------------------------------------------ descriptors
-// Shared-memory matrix descriptor of a K-major tile whose rows are 128 bytes
-// long, stored with the 128-byte swizzle in 1024-byte groups of 8 rows (the
-// layout a TMA load with CU_TENSOR_MAP_SWIZZLE_128B writes):
+// Shared-memory matrix descriptor of a K-major tile whose rows are kRowB = 128
+// or 64 bytes long, stored with the matching TMA swizzle (128-byte or 64-byte)
+// in groups of 8 rows (1024 or 512 bytes):
 //   bits  0-13 start address >> 4      bits 16-29 leading byte offset >> 4 (unused here: 1)
-//   bits 32-45 stride byte offset >> 4 (1024 B between 8-row groups)
-//   bits 46-47 descriptor version 1    bits 49-51 base offset 0 (1024-aligned tiles)
-//   bits 61-63 layout: 2 = 128-byte swizzle
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
+//   bits 32-45 stride byte offset >> 4 (bytes between 8-row groups)
+//   bits 46-47 descriptor version 1    bits 49-51 base offset 0 (tiles aligned to the group)
+//   bits 61-63 layout: 2 = 128-byte swizzle, 4 = 64-byte swizzle
+template <int kRowB>
+__device__ __forceinline__ uint64_t smem_desc_sw(uint32_t saddr) {
+    static_assert(kRowB == 128 || kRowB == 64, "128- or 64-byte rows");
     uint64_t d = 0;
     d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
     d |= static_cast<uint64_t>(1u) << 16;
-    d |= static_cast<uint64_t>(1024u >> 4) << 32;
+    d |= static_cast<uint64_t>((8u * kRowB) >> 4) << 32;
     d |= static_cast<uint64_t>(1u) << 46;
-    d |= static_cast<uint64_t>(2u) << 61;
+    d |= static_cast<uint64_t>(kRowB == 128 ? 2u : 4u) << 61;
     return d;
 }
 
