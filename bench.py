@@ -390,11 +390,19 @@ def main():
 
     if args.quick:
         ms_unf = ms_e2e = float("nan")
+        tab_unf = {}
         x_host = out_host = d["x"]
     else:
         # unfused GPU baseline (shared expert as its own dense pass), same process
         unfused = MoELayer(cfg, d, fuse_shared=False, impl=impl)
-        ms_unf = time_steps(lambda: unfused.forward(d["x"], out), args.steps, args.warmup, dist, stream)
+        for _ in range(args.warmup):
+            unfused.forward(d["x"], out)
+        torch.cuda.synchronize()
+        _lib.moe_profile_reset()
+        _lib.moe_profile_enable(True)
+        ms_unf = time_steps(lambda: unfused.forward(d["x"], out), args.steps, 0, dist, stream)
+        _lib.moe_profile_enable(False)
+        tab_unf = kernel_table(args.steps)
         del unfused
 
         # end to end through the public API with pinned host buffers: every step
@@ -450,7 +458,9 @@ def main():
         "hbm_gbs": alg_bytes / (ms_step / 1000.0) / 1e9,
         "hbm_frac": alg_bytes / (ms_step / 1000.0) / 1e9 / pk["hbm_gbs"],
         "unfused": {"value": N * cfg.T * args.steps / (ms_unf / 1000.0), "ms_per_step": ms_unf / args.steps,
-                    "fused_speedup": ms_unf / ms},
+                    "fused_speedup": ms_unf / ms,
+                    "kernels": {k: {"launches": v["launches"], "ms_per_step": v["total_ms"] / args.steps}
+                                for k, v in tab_unf.items()}},
         "e2e": {"value": N * cfg.T * args.steps / (ms_e2e / 1000.0), "unit": "tokens/s",
                 "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
                 "d2h_bytes_per_step": out_host.numel() * out_host.element_size()},
