@@ -211,15 +211,21 @@ def algorithmic(cfg, kernel: str, counts: np.ndarray | None):
 PROFILED_TRAFFIC_RATIO = {("gemm1_tc", "bf16", 256): 1.09, ("gemm2_tc", "bf16", 256): 0.97}
 
 
-def unit_rows(cfg, ffn: str) -> int:
+def unit_rows(cfg, ffn: str):
+    """Tensor-core work unit the run uses: 128, 256 (one CTA) or "pair256"
+    (256 rows over a CTA pair)."""
     if ffn == "tcgen05_m128":
         return 128
     if ffn == "tcgen05_m256":
         return 256
+    if ffn == "tcgen05_pair":
+        return "pair256"
+    if ffn == "tcgen05_wide":
+        return "pair256x512"
     return 256 if (cfg.w_dtype == "bf16" and cfg.rows >= 192 * cfg.n_experts) else 128
 
 
-def roofline_of(cfg, kernel: str, ms_per_launch: float, counts, pk, urows: int = 128) -> dict:
+def roofline_of(cfg, kernel: str, ms_per_launch: float, counts, pk, urows=128) -> dict:
     flops, nbytes = algorithmic(cfg, kernel, counts)
     ratio = PROFILED_TRAFFIC_RATIO.get((kernel, cfg.w_dtype, urows))
     traffic = int(ratio * nbytes) if (ratio and nbytes) else None
@@ -325,7 +331,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="prefill_bf16", choices=list(synth.CONFIGS))
-    ap.add_argument("--ffn", default="auto", choices=["auto", "simt", "tcgen05", "tcgen05_m128", "tcgen05_m256"])
+    ap.add_argument("--ffn", default="auto",
+                    choices=["auto", "simt", "tcgen05", "tcgen05_m128", "tcgen05_m256", "tcgen05_pair",
+                             "tcgen05_wide"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--quick", action="store_true",
@@ -351,7 +359,8 @@ def main():
                             name=f"{cfg.name}[T={args.tokens or cfg.T},E_r={args.routed or cfg.n_routed},"
                                  f"I={args.inter or cfg.I}]")
     impl = {"auto": _lib.MOE_FFN_AUTO, "simt": _lib.MOE_FFN_SIMT, "tcgen05": _lib.MOE_FFN_TCGEN05,
-            "tcgen05_m128": _lib.MOE_FFN_TCGEN05_M128, "tcgen05_m256": _lib.MOE_FFN_TCGEN05_M256}[args.ffn]
+            "tcgen05_m128": _lib.MOE_FFN_TCGEN05_M128, "tcgen05_m256": _lib.MOE_FFN_TCGEN05_M256,
+            "tcgen05_pair": _lib.MOE_FFN_TCGEN05_PAIR, "tcgen05_wide": _lib.MOE_FFN_TCGEN05_WIDE}[args.ffn]
     d = synth.make_inputs(cfg, dist.device)
     stream = torch.cuda.current_stream(dist.device)
     fused = MoELayer(cfg, d, fuse_shared=True, impl=impl)

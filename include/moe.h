@@ -78,10 +78,16 @@ typedef struct moe_shape {
  * picks the tensor-core work unit itself: 256 rows (two 128-row tiles of one
  * expert sharing each weight tile) for bf16 weights when groups average >= 192
  * rows, else 128;
- * TCGEN05_M128 / TCGEN05_M256 force one of them. */
+ * TCGEN05_M128 / TCGEN05_M256 force one of them; TCGEN05_PAIR forces 256-row
+ * units split over a pair of CTAs on the two SMs of a TPC (tcgen05 cta_group::2,
+ * each SM staging half of every weight tile); TCGEN05_WIDE the same with
+ * 256 x 512 tiles per pair (two N = 256 MMAs sharing each activation stage)
+ * where the output width allows (GEMM1: I % 256 == 0, GEMM2: H % 512 == 0;
+ * 256 x 256 pair tiles otherwise). */
 typedef enum moe_ffn_impl {
     MOE_FFN_AUTO = 0, MOE_FFN_SIMT = 1, MOE_FFN_TCGEN05 = 2,
-    MOE_FFN_TCGEN05_M128 = 3, MOE_FFN_TCGEN05_M256 = 4
+    MOE_FFN_TCGEN05_M128 = 3, MOE_FFN_TCGEN05_M256 = 4, MOE_FFN_TCGEN05_PAIR = 5,
+    MOE_FFN_TCGEN05_WIDE = 6
 } moe_ffn_impl;
 
 /* Bytes of workspace moe_forward needs for this shape (fused or not). The

@@ -174,18 +174,22 @@ __global__ void tile_prefix_kernel(int E, const int32_t* __restrict__ off, int32
 // for E4M3 layers.
 cudaError_t run_ffn(const FfnArgs& in, int impl, cudaStream_t st) {
     const bool tc_ok = ffn_tc_supported(in);
-    const bool tc_forced = impl == MOE_FFN_TCGEN05 || impl == MOE_FFN_TCGEN05_M128 || impl == MOE_FFN_TCGEN05_M256;
+    const bool tc_forced = impl == MOE_FFN_TCGEN05 || impl == MOE_FFN_TCGEN05_M128 ||
+                           impl == MOE_FFN_TCGEN05_M256 || impl == MOE_FFN_TCGEN05_PAIR ||
+                           impl == MOE_FFN_TCGEN05_WIDE;
     if (tc_forced || (impl == MOE_FFN_AUTO && in.w_dtype != MOE_F32 && tc_ok)) {
         if (!tc_ok) return cudaErrorNotSupported;
         FfnArgs a = in;
         a.unit_rows = impl == MOE_FFN_TCGEN05_M128 ? 128 : (impl == MOE_FFN_TCGEN05_M256 ? 256 : 0);
+        a.cta_pair = impl == MOE_FFN_TCGEN05_PAIR ? 1 : impl == MOE_FFN_TCGEN05_WIDE ? 2
+                   : (impl == MOE_FFN_AUTO || impl == MOE_FFN_TCGEN05) ? -1 : 0;
         return launch_ffn_tc(a, st);
     }
     return launch_ffn_simt(in, st);
 }
 
 moe_status check_impl(int impl, const moe_shape& s) {
-    if (impl < MOE_FFN_AUTO || impl > MOE_FFN_TCGEN05_M256) return MOE_ERR_INVALID_ARG;
+    if (impl < MOE_FFN_AUTO || impl > MOE_FFN_TCGEN05_WIDE) return MOE_ERR_INVALID_ARG;
     if (impl >= MOE_FFN_TCGEN05 && s.w_dtype == MOE_F32) return MOE_ERR_UNSUPPORTED;
     return MOE_OK;
 }
@@ -227,6 +231,7 @@ FfnArgs ffn_args(const moe_shape& s, const Dims& d, const Layout& L, void* ws, c
     a.y = y;
     a.yexp = nullptr;
     a.unit_rows = 0;
+    a.cta_pair = 0;
     a.direct_e = -1;
     a.max_mtiles = d.R / kTileM + d.E;
     a.status = at<DevStatus>(ws, L.status);
@@ -397,6 +402,7 @@ moe_status moe_forward(const moe_shape* shape, const void* x, const float* route
         a.y = at<void>(ws, L.sh_y);
         a.yexp = f32_act ? nullptr : at<int8_t>(ws, L.sh_yexp);
         a.unit_rows = 0;
+    a.cta_pair = 0;
         a.direct_e = -1;
         a.max_mtiles = ceil_div(d.T, kTileM);
         a.status = at<DevStatus>(ws, L.status);

@@ -128,6 +128,95 @@ __device__ __forceinline__ void stage_store(uint8_t* slice, const uint32_t (&pac
     __syncwarp();
 }
 
+// Epilogue of one unit for one warp: TMEM columns [c_begin, c_end) x 32 of the
+// lane group at `tb` (row = this lane's output row, valid if it is stored)
+// become bf16 h (GEMM1, SwiGLU applied) or bf16 / scaled-fp16 y rows (GEMM2),
+// leaving through this warp's staging slice (rows wrow0..wrow0+31).
+template <bool kFp8, bool kGemm1, int kBN>
+__device__ __forceinline__ void epilogue_rows(const TcParams& p, const TileInfo& t, uint32_t tb, int c_begin,
+                                              int c_end, uint8_t* stage_w, int lane, int row, bool valid,
+                                              float rs, int wrow0) {
+    constexpr int HALF = kBN / 2;
+    if constexpr (kGemm1) {
+#pragma unroll 1
+        for (int c = c_begin; c < c_end; ++c) {
+            uint32_t g[32], u[32];
+            ptx::tmem_ld_32x32b_x32(tb + c * 32, g);
+            ptx::tmem_ld_32x32b_x32(tb + HALF + c * 32, u);
+            ptx::tmem_ld_wait(g);
+            ptx::tmem_ld_wait(u);
+            const float* sg = (kFp8 && valid) ? p.col_scale + static_cast<size_t>(t.e) * 2 * p.I + t.n0 + c * 32 : nullptr;
+            const float* su = (kFp8 && valid) ? sg + p.I : nullptr;
+            uint32_t packed[16];
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+                float g0 = __uint_as_float(g[j]), g1 = __uint_as_float(g[j + 1]);
+                float u0 = __uint_as_float(u[j]), u1 = __uint_as_float(u[j + 1]);
+                if constexpr (kFp8) {
+                    if (valid) {
+                        g0 = g0 * rs * sg[j];
+                        g1 = g1 * rs * sg[j + 1];
+                        u0 = u0 * rs * su[j];
+                        u1 = u1 * rs * su[j + 1];
+                    }
+                }
+                packed[j >> 1] = pack_bf16x2(silu_f32(g0) * u0, silu_f32(g1) * u1);
+            }
+            stage_store(stage_w, packed, lane, p.out, p.out_ld, wrow0, t.row_end, t.n0 + c * 32);
+        }
+    } else {
+        // chunk c's TMEM load is in flight while chunk c-1 is converted and stored
+        uint64_t exps = 0;
+        auto process = [&](const uint32_t (&v)[32], int c) {
+            const float* sc = (kFp8 && valid) ? p.col_scale + static_cast<size_t>(t.e) * p.H + t.n0 + c * 32 : nullptr;
+            float a[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                a[j] = __uint_as_float(v[j]);
+                if constexpr (kFp8) {
+                    if (valid) a[j] = a[j] * rs * sc[j];
+                }
+            }
+            uint32_t packed[16];
+            if (p.yexp != nullptr) {
+                float amax = 0.0f;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(a[j]));
+                const int k = f16_chunk_exp(amax);
+                const float down = exp2_int(-k);
+#pragma unroll
+                for (int j = 0; j < 32; j += 2) packed[j >> 1] = pack_f16x2(a[j] * down, a[j + 1] * down);
+                exps |= static_cast<uint64_t>(static_cast<uint8_t>(static_cast<int8_t>(k))) << (8 * (c - c_begin));
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; j += 2) packed[j >> 1] = pack_bf16x2(a[j], a[j + 1]);
+            }
+            stage_store(stage_w, packed, lane, p.out, p.out_ld, wrow0, t.row_end, t.n0 + c * 32);
+        };
+        uint32_t va[32], vb[32];
+        ptx::tmem_ld_32x32b_x32(tb + c_begin * 32, va);
+        ptx::tmem_ld_wait(va);
+#pragma unroll 1
+        for (int c = c_begin; c < c_end; c += 2) {
+            const bool has_b = c + 1 < c_end;
+            if (has_b) ptx::tmem_ld_32x32b_x32(tb + (c + 1) * 32, vb);
+            process(va, c);
+            if (has_b) {
+                ptx::tmem_ld_wait(vb);
+                const bool has_a = c + 2 < c_end;
+                if (has_a) ptx::tmem_ld_32x32b_x32(tb + (c + 2) * 32, va);
+                process(vb, c + 1);
+                if (has_a) ptx::tmem_ld_wait(va);
+            }
+        }
+        if (p.yexp != nullptr && valid) {
+            int8_t* e = p.yexp + static_cast<size_t>(row) * (p.H / 32) + t.n0 / 32 + c_begin;
+            if (c_end - c_begin == 8) *reinterpret_cast<uint64_t*>(e) = exps;
+            else *reinterpret_cast<uint32_t*>(e) = static_cast<uint32_t>(exps);
+        }
+    }
+}
+
 // kBN: MMA N (GEMM1: gate half + up half; GEMM2: 256 output columns).
 // kPair: a work unit is two consecutive 128-row m-tiles of one expert that share
 // each weight (B) stage in shared memory (an M = 256 tile: every weight byte is
@@ -355,88 +444,11 @@ __global__ void __launch_bounds__(320, 1)
             if (kFp8 && valid)
                 rs = (t.e == p.direct_e) ? p.direct_scale[row - s_off[t.e]] : p.row_scale[row];
             if (active) {
-            // 16-bit outputs leave through this warp's 2 KB staging slice so that
-            // global stores cover whole 64-byte row segments (see stage_store)
-            uint8_t* stage_w = sStage + (warp - 2) * 2048;
-            const int wrow0 = t.row0 + (kPair ? eg * TC_BM : 0) + sub * 32;   // first unit row of this warp
-            if constexpr (kGemm1) {
-#pragma unroll 1
-                for (int c = c_begin; c < c_end; ++c) {
-                    uint32_t g[32], u[32];
-                    ptx::tmem_ld_32x32b_x32(tb + c * 32, g);
-                    ptx::tmem_ld_32x32b_x32(tb + HALF + c * 32, u);
-                    ptx::tmem_ld_wait(g);
-                    ptx::tmem_ld_wait(u);
-                    const float* sg = (kFp8 && valid) ? p.col_scale + static_cast<size_t>(t.e) * 2 * p.I + t.n0 + c * 32 : nullptr;
-                    const float* su = (kFp8 && valid) ? sg + p.I : nullptr;
-                    uint32_t packed[16];
-#pragma unroll
-                    for (int j = 0; j < 32; j += 2) {
-                        float g0 = __uint_as_float(g[j]), g1 = __uint_as_float(g[j + 1]);
-                        float u0 = __uint_as_float(u[j]), u1 = __uint_as_float(u[j + 1]);
-                        if constexpr (kFp8) {
-                            if (valid) {
-                                g0 = g0 * rs * sg[j];
-                                g1 = g1 * rs * sg[j + 1];
-                                u0 = u0 * rs * su[j];
-                                u1 = u1 * rs * su[j + 1];
-                            }
-                        }
-                        packed[j >> 1] = pack_bf16x2(silu_f32(g0) * u0, silu_f32(g1) * u1);
-                    }
-                    stage_store(stage_w, packed, lane, p.out, p.out_ld, wrow0, t.row_end, t.n0 + c * 32);
-                }
-            } else {
-                // chunk c's TMEM load is in flight while chunk c-1 is converted and stored
-                uint64_t exps = 0;
-                auto process = [&](const uint32_t (&v)[32], int c) {
-                    const float* sc = (kFp8 && valid) ? p.col_scale + static_cast<size_t>(t.e) * p.H + t.n0 + c * 32 : nullptr;
-                    float a[32];
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        a[j] = __uint_as_float(v[j]);
-                        if constexpr (kFp8) {
-                            if (valid) a[j] = a[j] * rs * sc[j];
-                        }
-                    }
-                    uint32_t packed[16];
-                    if (p.yexp != nullptr) {
-                        float amax = 0.0f;
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(a[j]));
-                        const int k = f16_chunk_exp(amax);
-                        const float down = exp2_int(-k);
-#pragma unroll
-                        for (int j = 0; j < 32; j += 2) packed[j >> 1] = pack_f16x2(a[j] * down, a[j + 1] * down);
-                        exps |= static_cast<uint64_t>(static_cast<uint8_t>(static_cast<int8_t>(k))) << (8 * (c - c_begin));
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 32; j += 2) packed[j >> 1] = pack_bf16x2(a[j], a[j + 1]);
-                    }
-                    stage_store(stage_w, packed, lane, p.out, p.out_ld, wrow0, t.row_end, t.n0 + c * 32);
-                };
-                uint32_t va[32], vb[32];
-                ptx::tmem_ld_32x32b_x32(tb + c_begin * 32, va);
-                ptx::tmem_ld_wait(va);
-#pragma unroll 1
-                for (int c = c_begin; c < c_end; c += 2) {
-                    const bool has_b = c + 1 < c_end;
-                    if (has_b) ptx::tmem_ld_32x32b_x32(tb + (c + 1) * 32, vb);
-                    process(va, c);
-                    if (has_b) {
-                        ptx::tmem_ld_wait(vb);
-                        const bool has_a = c + 2 < c_end;
-                        if (has_a) ptx::tmem_ld_32x32b_x32(tb + (c + 2) * 32, va);
-                        process(vb, c + 1);
-                        if (has_a) ptx::tmem_ld_wait(va);
-                    }
-                }
-                if (p.yexp != nullptr && valid) {
-                    int8_t* e = p.yexp + static_cast<size_t>(row) * (p.H / 32) + t.n0 / 32 + c_begin;
-                    if (c_end - c_begin == 8) *reinterpret_cast<uint64_t*>(e) = exps;
-                    else *reinterpret_cast<uint32_t*>(e) = static_cast<uint32_t>(exps);
-                }
-            }
+                // 16-bit outputs leave through this warp's 2 KB staging slice so that
+                // global stores cover whole 64-byte row segments (see stage_store)
+                uint8_t* stage_w = sStage + (warp - 2) * 2048;
+                const int wrow0 = t.row0 + (kPair ? eg * TC_BM : 0) + sub * 32;   // first unit row of this warp
+                epilogue_rows<kFp8, kGemm1, kBN>(p, t, tb, c_begin, c_end, stage_w, lane, row, valid, rs, wrow0);
             }
             ptx::tc_fence_before();
             ptx::mbar_arrive(&tempty_bar[acc]);
@@ -455,6 +467,294 @@ __global__ void __launch_bounds__(320, 1)
         __syncwarp();
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem_base, TC_TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------ CTA-pair kernel
+// 256-row units on a cluster of two CTAs (the two SMs of a TPC) with
+// tcgen05.mma.cta_group::2: CTA r holds A rows row0 + 128 r .. +127 and half
+// of the unit's B rows, and receives D rows 128 r .. +127 for all columns in
+// its own TMEM. Each weight byte is fetched once per 256 rows, as with
+// single-CTA 256-row units, but each SM stages only half of it.
+//
+// kNSUB = 1: one N = kBN MMA per K step; the two TMEM buffers (columns 0 and
+//   256) alternate between units, so the epilogue of one unit overlaps the
+//   MMAs of the next. B halves: GEMM1 the gate rows in rank 0 and the up rows
+//   in rank 1; GEMM2 output columns n0 + 128 r .. +127.
+// kNSUB = 2: two N = 256 MMAs per K step share the A stage (a 256 x 512 tile
+//   per pair: half the A traffic per FLOP, a quarter less staged per FLOP),
+//   filling all 512 TMEM columns; sub-tile j accumulates in columns 256 j.
+//   GEMM1: rank 0 stages gate rows n0 .. n0+255 and rank 1 the up rows, so
+//   sub-tile j holds gate and up of h columns n0 + 128 j .. +127; GEMM2: rank r
+//   stages output rows n0 + 256 j + 128 r .. +127 for sub-tile j, so sub-tile j
+//   holds output columns n0 + 256 j .. +255. Warps 2-5 drain sub-tile 0 and
+//   warps 6-9 sub-tile 1; the next unit's MMAs wait for both.
+//
+// Rank 0 arms its full barriers for the bytes of both CTAs and issues every
+// MMA; the commit that frees a stage or fills an accumulator arrives on the
+// barrier of that index in both CTAs. The epilogue threads of both CTAs arrive
+// on rank 0's TMEM-empty barriers. A wait that runs out raises the abort flag
+// of both CTAs.
+template <int kRowB, int kBN, int kNSUB>
+struct Ring2 {
+    static constexpr int A_TILE = TC_BM * kRowB;
+    static constexpr int B_SUB = (kBN / 2) * kRowB;           // one CTA's rows of one sub-tile
+    static constexpr int B_HALF = kNSUB * B_SUB;
+    static constexpr int STAGE = A_TILE + B_HALF;
+    static constexpr int N = (TC_RING_BYTES / STAGE) > 8 ? 8 : (TC_RING_BYTES / STAGE);
+    static constexpr int SMEM = N * STAGE + 8 * 2048 + 1024;
+};
+
+template <bool kFp8, bool kGemm1, int kBN, int kNSUB, int kRowB>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                             const __grid_constant__ CUtensorMap tmA2, const TcParams p) {
+    static_assert(kNSUB == 1 || kBN == 256, "two sub-tiles of N = 256");
+    using RG = Ring2<kRowB, kBN, kNSUB>;
+    constexpr int NSTAGE = RG::N;
+    constexpr int ABYTES = RG::A_TILE;
+    constexpr int BBYTES = RG::B_HALF;
+    constexpr int HALF = kBN / 2;
+    constexpr int KEL = kFp8 ? kRowB : kRowB / 2;
+    constexpr int KSTEPS = kRowB / 32;
+    constexpr int EPI_WARPS = 8;
+    constexpr uint32_t IDESC = ptx::instr_desc(2 * TC_BM, kBN, kFp8 ? 0u : 1u);
+
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint64_t full_bar[NSTAGE], empty_bar[NSTAGE], tfull_bar[2], tempty_bar[2], drain_bar;
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_abort;
+    __shared__ int s_off[TC_MAXE], s_unit[TC_MAXE];
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = ptx::cluster_ctarank();
+    const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+    const uint32_t raw = ptx::smem_u32(smem_raw);
+    uint8_t* base = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+    uint8_t* sA = base;
+    uint8_t* sB = base + NSTAGE * ABYTES;
+    uint8_t* sStage = sB + NSTAGE * BBYTES;
+    volatile int* abort_flag = &s_abort;
+    const uint32_t peer_abort = ptx::mapa(&s_abort, rank ^ 1u);
+
+    for (int i = threadIdx.x; i <= p.E; i += blockDim.x) s_off[i] = p.offsets[i];
+    if (warp == 0) {
+        // prefix of 256-row units per expert
+        int carry = 0;
+        for (int e0 = 0; e0 <= p.E; e0 += 32) {
+            const int e = e0 + lane;
+            const int pairs = (e < p.E) ? (p.tile_off[e + 1] - p.tile_off[e] + 1) >> 1 : 0;
+            int inc = pairs;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int o = __shfl_up_sync(0xFFFFFFFFu, inc, off);
+                if (lane >= off) inc += o;
+            }
+            if (e <= p.E) s_unit[e] = carry + inc - pairs;
+            carry += __shfl_sync(0xFFFFFFFFu, inc, 31);
+        }
+    }
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NSTAGE; ++s) {
+            ptx::mbar_init(&full_bar[s], 1);
+            ptx::mbar_init(&empty_bar[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(&tfull_bar[b], 1);
+            // epilogue threads of both CTAs that drain this buffer
+            ptx::mbar_init(&tempty_bar[b], 2 * (EPI_WARPS / kNSUB) * 32);
+        }
+        ptx::mbar_init(&drain_bar, 1);
+        s_abort = 0;
+        ptx::fence_mbar_init();
+        ptx::prefetch_tmap(&tmA);
+        ptx::prefetch_tmap(&tmB);
+        if (p.direct_e >= 0) ptx::prefetch_tmap(&tmA2);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc_pair(&s_tmem, TC_TMEM_COLS);
+        ptx::tmem_relinquish_pair();
+    }
+    ptx::tc_fence_before();
+    ptx::cluster_sync();        // rank 0's barriers exist before the peer's copies name them
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = s_tmem;
+    const int total = s_unit[p.E] * p.n_tiles_n;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- producers (both CTAs)
+        if (!p.inject_stall) {
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int u = cluster; u < total; u += nclusters) {
+                const TileInfo t = decode_unit<true>(u, s_unit, s_off, p.E, p.n_tiles_n, p.bn_out);
+                int ok = 1;
+                if (lane == 0) {
+                    // rank 1's A tile exists only when the unit has a second m-tile;
+                    // otherwise its rows of D are never stored and its MMA rows read
+                    // whatever the stage last held
+                    const bool load_a = rank == 0 || t.two;
+                    const uint32_t tx = (t.two ? 2 : 1) * ABYTES + 2 * BBYTES;
+                    const bool direct = t.e == p.direct_e;
+                    const CUtensorMap* am = direct ? &tmA2 : &tmA;
+                    const int ar = (direct ? t.row0 - s_off[t.e] : t.row0) + static_cast<int>(rank) * TC_BM;
+                    for (int kb = 0; kb < p.k_blocks; ++kb) {
+                        if (!ptx::mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, p.wait_limit, p.status, 1u)) {
+                            ok = 0;
+                            break;
+                        }
+                        const uint32_t fb = ptx::mapa(&full_bar[stage], 0);
+                        if (rank == 0) ptx::mbar_arrive_expect_tx(&full_bar[stage], tx);
+                        const int kx = kb * KEL;
+                        uint8_t* b_dst = sB + stage * BBYTES;
+                        if (load_a) ptx::tma_load_2d_pair(sA + stage * ABYTES, am, fb, kx, ar);
+                        if constexpr (kGemm1) {
+                            // one box of kNSUB * HALF gate (rank 0) or up (rank 1) rows
+                            ptx::tma_load_3d_pair(b_dst, &tmB, fb, kx, t.n0, 2 * t.e + static_cast<int>(rank));
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < kNSUB; ++j)
+                                ptx::tma_load_2d_pair(b_dst + j * RG::B_SUB, &tmB, fb, kx,
+                                                      t.e * p.H + t.n0 + j * kBN + static_cast<int>(rank) * HALF);
+                        }
+                        if (++stage == NSTAGE) { stage = 0; phase ^= 1u; }
+                    }
+                }
+                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+                __syncwarp();
+                if (!ok) break;
+            }
+            if (lane == 0 && *abort_flag) {
+                ptx::st_remote_u32(peer_abort, 1u);
+                if (rank == 0) {
+                    // every stage's last armed phase completes when both CTAs' bytes land
+                    for (int s = 0; s < NSTAGE; ++s) {
+                        const uint32_t par = (s < stage) ? phase : (phase ^ 1u);
+                        const long long t0 = clock64();
+                        while (!ptx::mbar_try_wait(&full_bar[s], par) && clock64() - t0 < p.wait_limit) {
+                        }
+                    }
+                } else {
+                    // rank 1 cannot see its copies land (they count on rank 0's
+                    // barriers): give any in flight ample time
+                    const long long t0 = clock64();
+                    while (clock64() - t0 < (1ll << 21)) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer (rank 0)
+        if (lane == 0 && rank == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;                // kNSUB = 1: buffer of this unit
+            uint32_t acc_phase = 0;     // parity of the buffer's current use
+            for (int u = cluster; u < total; u += nclusters) {
+                bool ok = true;
+#pragma unroll
+                for (int j = 0; j < kNSUB; ++j) {
+                    const int b = kNSUB == 1 ? acc : j;
+                    ok = ok && ptx::mbar_wait_cluster(&tempty_bar[b], acc_phase ^ 1u, abort_flag, p.wait_limit,
+                                                      p.status, 2u);
+                }
+                if (!ok) break;
+                ptx::tc_fence_after();
+                const uint32_t d = tmem_base + static_cast<uint32_t>(acc * 256);
+                for (int kb = 0; kb < p.k_blocks; ++kb) {
+                    if (!ptx::mbar_wait(&full_bar[stage], phase, abort_flag, p.wait_limit, p.status, 3u)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    const uint32_t a_addr = ptx::smem_u32(sA + stage * ABYTES);
+                    const uint32_t b_addr = ptx::smem_u32(sB + stage * BBYTES);
+#pragma unroll
+                    for (int k = 0; k < KSTEPS; ++k) {
+                        const uint64_t ad = ptx::smem_desc_sw<kRowB>(a_addr + k * 32);
+#pragma unroll
+                        for (int j = 0; j < kNSUB; ++j) {
+                            const uint64_t bd = ptx::smem_desc_sw<kRowB>(b_addr + j * RG::B_SUB + k * 32);
+                            const uint32_t dj = d + static_cast<uint32_t>(j * 256);
+                            if constexpr (kFp8) ptx::mma_f8_pair(dj, ad, bd, IDESC, (kb | k) != 0);
+                            else ptx::mma_f16_pair(dj, ad, bd, IDESC, (kb | k) != 0);
+                        }
+                    }
+                    ptx::mma_commit_pair(&empty_bar[stage], 0x3);
+                    if (++stage == NSTAGE) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+#pragma unroll
+                for (int j = 0; j < kNSUB; ++j) ptx::mma_commit_pair(&tfull_bar[kNSUB == 1 ? acc : j], 0x3);
+                if constexpr (kNSUB == 1) {
+                    acc ^= 1;
+                    if (acc == 0) acc_phase ^= 1u;
+                } else {
+                    acc_phase ^= 1u;
+                }
+            }
+            if (*abort_flag) ptx::st_remote_u32(peer_abort, 1u);
+            // every MMA has finished (in both CTAs' TMEM and shared memory) before teardown
+            ptx::mma_commit_pair(&drain_bar, 0x3);
+        }
+        if (lane == 0) {
+            const long long t0 = clock64();
+            while (!ptx::mbar_try_wait(&drain_bar, 0) && clock64() - t0 < p.wait_limit) {
+            }
+        }
+    } else {
+        // ---------------------------------------------------------------- epilogue (both CTAs)
+        const int sub = warp & 3;
+        const int eg = (warp - 2) >> 2;            // kNSUB = 1: column half; 2: sub-tile
+        constexpr int NCH = kGemm1 ? HALF / 32 : kBN / 32;
+        constexpr int PER = kNSUB == 1 ? (NCH + 1) / 2 : NCH;
+        const int c_begin = kNSUB == 1 ? eg * PER : 0;
+        const int c_end = min(NCH, c_begin + PER);
+        const int r_local = static_cast<int>(rank) * TC_BM + sub * 32 + lane;
+        const uint32_t tempty0 = ptx::mapa(&tempty_bar[0], 0);
+        const uint32_t tempty1 = ptx::mapa(&tempty_bar[1], 0);
+        uint8_t* stage_w = sStage + (warp - 2) * 2048;
+        int acc = kNSUB == 1 ? 0 : eg;
+        uint32_t acc_phase = 0;
+        for (int u = cluster; u < total; u += nclusters) {
+            TileInfo t = decode_unit<true>(u, s_unit, s_off, p.E, p.n_tiles_n, p.bn_out);
+            int ok = 0;
+            if (lane == 0) ok = ptx::mbar_wait(&tfull_bar[acc], acc_phase, abort_flag, p.wait_limit, p.status, 4u);
+            ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+            if (!ok) {
+                if (lane == 0) ptx::st_remote_u32(peer_abort, 1u);
+                break;
+            }
+            ptx::tc_fence_after();
+            if constexpr (kNSUB == 2) t.n0 += eg * (kGemm1 ? HALF : kBN);   // this sub-tile's output columns
+            const bool active = (rank == 0 || t.two) && c_begin < c_end;    // warp-uniform
+            const int row = t.row0 + r_local;
+            const bool valid = active && row < t.row_end;
+            const uint32_t tb = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + static_cast<uint32_t>(acc * 256);
+            float rs = 1.0f;
+            if (kFp8 && valid)
+                rs = (t.e == p.direct_e) ? p.direct_scale[row - s_off[t.e]] : p.row_scale[row];
+            if (active) {
+                const int wrow0 = t.row0 + static_cast<int>(rank) * TC_BM + sub * 32;
+                epilogue_rows<kFp8, kGemm1, kBN>(p, t, tb, c_begin, c_end, stage_w, lane, row, valid, rs, wrow0);
+            }
+            ptx::tc_fence_before();
+            ptx::mbar_arrive_remote(acc == 0 ? tempty0 : tempty1);
+            if constexpr (kNSUB == 1) {
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
+            } else {
+                acc_phase ^= 1u;
+            }
+        }
+    }
+
+    __syncwarp();
+    ptx::tc_fence_before();
+    ptx::cluster_sync();        // no CTA leaves while its peer may still name its memory
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc_pair(tmem_base, TC_TMEM_COLS);
     }
 }
 
@@ -525,12 +825,51 @@ cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const CUtenso
     return cudaGetLastError();
 }
 
+// CTA pairs: as many clusters of two as can be resident at once (a TPC with
+// one usable SM holds none), each walking the units persistently
+template <bool kFp8, bool kGemm1, int kBN, int kNSUB>
+cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2, const TcParams& p,
+                        cudaStream_t st, const char* name) {
+    constexpr int kRowB = SRE_STAGE_ROW_BYTES;
+    constexpr int smem = Ring2<kRowB, kBN, kNSUB>::SMEM;
+    auto kern = grouped_gemm_pair_kernel<kFp8, kGemm1, kBN, kNSUB, kRowB>;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    static int clusters = 0;
+    std::call_once(once, [kern] {
+        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (attr_err != cudaSuccess) return;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(num_sms() & ~1), 1, 1);
+        cfg.blockDim = dim3(320, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        int n = 0;
+        attr_err = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+        clusters = n;
+        if (attr_err == cudaSuccess && n < 1) attr_err = cudaErrorNotSupported;
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    ProfileScope ps(name, st);
+    kern<<<2 * clusters, 320, smem, st>>>(a, b, a2, p);
+    note_launch();
+    return cudaGetLastError();
+}
+
 template <bool kFp8, bool kPair>
 cudaError_t launch_gemm1(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2, const TcParams& p,
                          int half, cudaStream_t st) {
     if (half == 128) return launch_one<kFp8, true, 256, kPair>(a, b, a2, p, st, "gemm1_tc");
     if (half == 96) return launch_one<kFp8, true, 192, kPair>(a, b, a2, p, st, "gemm1_tc");
     return launch_one<kFp8, true, 128, kPair>(a, b, a2, p, st, "gemm1_tc");
+}
+
+template <bool kFp8>
+cudaError_t launch_gemm1_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2, const TcParams& p,
+                              int half, bool wide, cudaStream_t st) {
+    if (wide) return launch_pair<kFp8, true, 256, 2>(a, b, a2, p, st, "gemm1_tc");
+    if (half == 128) return launch_pair<kFp8, true, 256, 1>(a, b, a2, p, st, "gemm1_tc");
+    if (half == 96) return launch_pair<kFp8, true, 192, 1>(a, b, a2, p, st, "gemm1_tc");
+    return launch_pair<kFp8, true, 128, 1>(a, b, a2, p, st, "gemm1_tc");
 }
 
 }  // namespace
@@ -574,6 +913,13 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
         inject = cur > 0 ? 1 : 0;
     }
 
+    // CTA pairs (cta_pair > 0); 256 x 512 pair tiles (cta_pair == 2) where the
+    // output width divides into them (GEMM1: I % 256, GEMM2: H % 512)
+    const bool two_sm = a.cta_pair > 0;
+    const bool wide1 = a.cta_pair == 2 && half == 128 && a.I % 256 == 0;
+    const bool wide2 = a.cta_pair == 2 && a.H % 512 == 0;
+    const int bn1 = wide1 ? 2 * half : half;     // h columns per unit
+
     // GEMM1: A = Xp [R, H] (rows gathered by the gather kernel); B = W13 viewed as
     // [2E][I][H] (gate/up halves separately clipped at I)
     CUtensorMap ta, tb;
@@ -583,7 +929,7 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
         const cuuint64_t bd[3] = {static_cast<cuuint64_t>(a.H), static_cast<cuuint64_t>(a.I),
                                   static_cast<cuuint64_t>(2 * a.E)};
         const cuuint64_t bs[2] = {static_cast<cuuint64_t>(a.H) * esz, static_cast<cuuint64_t>(a.I) * a.H * esz};
-        if (!make_map(&ta, xp, fp8, 2, ad, as, TC_BM, kRowBytes) || !make_map(&tb, a.w13, fp8, 3, bd, bs, half, kRowBytes))
+        if (!make_map(&ta, xp, fp8, 2, ad, as, TC_BM, kRowBytes) || !make_map(&tb, a.w13, fp8, 3, bd, bs, bn1, kRowBytes))
             return cudaErrorInvalidValue;
     }
     // the direct group's A: the token matrix [T, H]
@@ -596,8 +942,8 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
     }
     TcParams p;
     p.E = a.E; p.H = a.H; p.I = a.I;
-    p.n_tiles_n = ceil_div(a.I, half);
-    p.bn_out = half;
+    p.n_tiles_n = ceil_div(a.I, bn1);
+    p.bn_out = bn1;
     p.k_blocks = ceil_div(a.H, kel);
     p.offsets = a.offsets;
     p.tile_off = a.tile_off;
@@ -617,10 +963,15 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
     // faster with 128-row units (prefill_fp8 4.95 vs 6.04 ms, skewed_fp8 0.84 vs 0.99 ms).
     const bool pair = a.unit_rows == 256 ||
                       (a.unit_rows == 0 && a.w_dtype == MOE_BF16 && a.R >= 192 * a.E);
-    cudaError_t err = fp8 ? (pair ? launch_gemm1<true, true>(ta, tb, ta2, p, half, st)
-                                  : launch_gemm1<true, false>(ta, tb, ta2, p, half, st))
-                          : (pair ? launch_gemm1<false, true>(ta, tb, ta2, p, half, st)
-                                  : launch_gemm1<false, false>(ta, tb, ta2, p, half, st));
+    cudaError_t err;
+    if (two_sm)
+        err = fp8 ? launch_gemm1_pair<true>(ta, tb, ta2, p, half, wide1, st)
+                  : launch_gemm1_pair<false>(ta, tb, ta2, p, half, wide1, st);
+    else
+        err = fp8 ? (pair ? launch_gemm1<true, true>(ta, tb, ta2, p, half, st)
+                          : launch_gemm1<true, false>(ta, tb, ta2, p, half, st))
+                  : (pair ? launch_gemm1<false, true>(ta, tb, ta2, p, half, st)
+                          : launch_gemm1<false, false>(ta, tb, ta2, p, half, st));
     if (err != cudaSuccess) return err;
 
     const void* hA = a.h;
@@ -635,11 +986,13 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
         const cuuint64_t as[1] = {static_cast<cuuint64_t>(a.I) * esz};
         const cuuint64_t bd[2] = {static_cast<cuuint64_t>(a.I), static_cast<cuuint64_t>(a.E) * a.H};
         const cuuint64_t bs[1] = {static_cast<cuuint64_t>(a.I) * esz};
-        if (!make_map(&ta, hA, fp8, 2, ad, as, TC_BM, kRowBytes) || !make_map(&tb, a.w2, fp8, 2, bd, bs, 256, kRowBytes))
+        // a CTA pair stages 128 of the 256 weight rows in each CTA
+        if (!make_map(&ta, hA, fp8, 2, ad, as, TC_BM, kRowBytes) ||
+            !make_map(&tb, a.w2, fp8, 2, bd, bs, two_sm ? 128 : 256, kRowBytes))
             return cudaErrorInvalidValue;
     }
-    p.n_tiles_n = a.H / 256;
-    p.bn_out = 256;
+    p.n_tiles_n = a.H / (wide2 ? 512 : 256);
+    p.bn_out = wide2 ? 512 : 256;
     p.k_blocks = ceil_div(a.I, kel);
     p.out = static_cast<uint16_t*>(a.y);
     p.out_ld = a.H;
@@ -647,6 +1000,12 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
     p.direct_e = -1;
     p.col_scale = fp8 ? a.s2 : nullptr;
     p.yexp = a.yexp;
+    if (wide2)
+        return fp8 ? launch_pair<true, false, 256, 2>(ta, tb, ta, p, st, "gemm2_tc")
+                   : launch_pair<false, false, 256, 2>(ta, tb, ta, p, st, "gemm2_tc");
+    if (two_sm)
+        return fp8 ? launch_pair<true, false, 256, 1>(ta, tb, ta, p, st, "gemm2_tc")
+                   : launch_pair<false, false, 256, 1>(ta, tb, ta, p, st, "gemm2_tc");
     if (fp8)
         return pair ? launch_one<true, false, 256, true>(ta, tb, ta, p, st, "gemm2_tc")
                     : launch_one<true, false, 256, false>(ta, tb, ta, p, st, "gemm2_tc");

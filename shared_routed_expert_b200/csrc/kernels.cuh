@@ -64,6 +64,7 @@ struct FfnArgs {
     // chosen so the chunk's largest |v| maps into [2^14, 2^15)
     int8_t* yexp;
     int unit_rows;                // tensor-core work unit: 0 auto, 128 or 256 rows
+    int cta_pair;                 // tensor-core: 256-row units split over a CTA pair (cta_group::2)
     int direct_e;                 // expert whose rows are tokens 0..T-1 in order (A read from
                                   // xt directly, not gathered), or -1
     int max_mtiles;               // upper bound of sum_e ceil(count_e / kTileM)

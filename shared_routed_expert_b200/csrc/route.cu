@@ -11,129 +11,162 @@
 // computes one segment's chains per block (T x E x H/256 independent chains:
 // enough parallelism to fill the GPU at any T), and the top-K kernel adds the
 // segment partials in order.
+#include <mutex>
+
 #include "kernels.cuh"
 
 namespace sre {
 
 namespace {
 
-constexpr int RT_BT = 128;    // tokens per block
-constexpr int RT_BE = 32;     // experts per block
-constexpr int RT_KC = 32;     // h per shared-memory chunk
-constexpr int RT_SEG = 256;   // segment length of the fixed order
-constexpr int RT_XP = RT_BT + 4;   // row pitch (floats) of the transposed x tile
-constexpr int RT_WP = RT_BE + 4;   // row pitch (floats) of the transposed w tile
+constexpr int RT_BT = 64;      // tokens per block
+constexpr int RT_EL = 16;      // expert lanes per block
+constexpr int RT_EJ = 10;      // experts per thread (strided by RT_EL)
+constexpr int RT_BE = RT_EL * RT_EJ;   // experts per block (160)
+constexpr int RT_KC = 32;      // h per shared-memory chunk
+constexpr int RT_SEG = 256;    // segment length of the fixed order
+constexpr int RT_XP = RT_BT + 4;       // row pitch (floats) of the transposed x tile xs[k][t]
+constexpr int RT_WP = RT_KC + 4;       // row pitch (floats) of the w tile ws[e][k]: 144 B rows
+constexpr int RT_THREADS = 256;
 
-// x chunk: 128 tokens x 32 h -> xs[h][t]; thread i loads tokens i and i + 64
-template <bool kBf16>
-__device__ __forceinline__ void load_x_chunk(const void* x, int T, int H, int t0, int h0,
-                                             float (*xs)[RT_XP]) {
+struct RouterSmem {
+    float xs[2][RT_KC][RT_XP];
+    float ws[2][RT_BE][RT_WP];
+};
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+                 "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// w chunk: rows e0.. (up to 160 experts) x 32 h, copied as is into ws[e][k]
+// (16-byte pieces; rows past E are left unwritten: their results are never stored)
+__device__ __forceinline__ void issue_w_chunk(const float* wr, int E, int H, int e0, int h0,
+                                              float (*ws)[RT_WP]) {
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-        const int tl = threadIdx.x + half * 64;
-        const int t = t0 + tl;
-        float v[32];
-        if (t < T) {
-            if constexpr (kBf16) {
-                const uint4* p = reinterpret_cast<const uint4*>(
-                    static_cast<const uint16_t*>(x) + static_cast<size_t>(t) * H + h0);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint4 a = p[q];
-                    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        v[8 * q + 2 * j] = __uint_as_float(w[j] << 16);
-                        v[8 * q + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-                    }
-                }
-            } else {
-                const float4* p = reinterpret_cast<const float4*>(
-                    static_cast<const float*>(x) + static_cast<size_t>(t) * H + h0);
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const float4 a = p[q];
-                    v[4 * q] = a.x; v[4 * q + 1] = a.y; v[4 * q + 2] = a.z; v[4 * q + 3] = a.w;
-                }
-            }
-        } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = 0.0f;
-        }
-#pragma unroll
-        for (int j = 0; j < 32; ++j) xs[j][tl] = v[j];
+    for (int i = 0; i < (RT_BE * RT_KC / 4) / RT_THREADS; ++i) {
+        const int piece = threadIdx.x + i * RT_THREADS;
+        const int e = piece >> 3, c = piece & 7;
+        if (e0 + e < E) cp_async16(&ws[e][c * 4], wr + static_cast<size_t>(e0 + e) * H + h0 + c * 4);
     }
+    cp_async_commit();
 }
 
-// w chunk: 32 experts x 32 h -> ws[h][e]; thread i loads expert i/2, h-half i%2
-__device__ __forceinline__ void load_w_chunk(const float* wr, int E, int H, int e0, int h0,
-                                             float (*ws)[RT_WP]) {
-    const int i = threadIdx.x;
-    const int e = e0 + (i >> 1);
-    const int hb = (i & 1) * 16;
-    float v[16];
-    if (e < E) {
-        const float4* p = reinterpret_cast<const float4*>(wr + static_cast<size_t>(e) * H + h0 + hb);
+// x chunk: 64 tokens x 32 h; thread i holds token t0 + i % 64, h h0 + 8 (i / 64) .. +7
+template <bool kBf16>
+__device__ __forceinline__ void load_x_chunk(const void* x, int T, int H, int t0, int h0, float (&v)[8]) {
+    const int t = t0 + (threadIdx.x & (RT_BT - 1));
+    const int q = (threadIdx.x >> 6) * 8;
+    if (t < T) {
+        if constexpr (kBf16) {
+            const uint4 a = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) +
+                                                            static_cast<size_t>(t) * H + h0 + q);
+            const uint32_t w[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float4 q = p[j];
-            v[4 * j] = q.x; v[4 * j + 1] = q.y; v[4 * j + 2] = q.z; v[4 * j + 3] = q.w;
+            for (int j = 0; j < 4; ++j) {
+                v[2 * j] = __uint_as_float(w[j] << 16);
+                v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+            }
+        } else {
+            const float* p = static_cast<const float*>(x) + static_cast<size_t>(t) * H + h0 + q;
+            const float4 a = *reinterpret_cast<const float4*>(p);
+            const float4 b = *reinterpret_cast<const float4*>(p + 4);
+            v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+            v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
         }
     } else {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] = 0.0f;
+        for (int j = 0; j < 8; ++j) v[j] = 0.0f;
     }
-#pragma unroll
-    for (int j = 0; j < 16; ++j) ws[hb + j][i >> 1] = v[j];
 }
 
-// grid (ceil(T/128), ceil(E/32), H/256); 64 threads, 8 tokens x 8 experts each.
-// P[s][t][e] = fma chain over the 256 h of segment s (blockIdx.z), from +0.
+__device__ __forceinline__ void store_x_chunk(const float (&v)[8], float (*xs)[RT_XP]) {
+    const int tl = threadIdx.x & (RT_BT - 1);
+    const int q = (threadIdx.x >> 6) * 8;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) xs[q + j][tl] = v[j];
+}
+
+// grid (ceil(T/64), ceil(E/160), H/256); 256 threads: thread (ty, tx) =
+// (threadIdx / 16, threadIdx % 16) owns tokens t0 + 4 ty .. +3 and experts
+// e0 + tx + 16 j (j < 10). P[s][t][e] = fma chain over the 256 h of segment s
+// (blockIdx.z), from +0, h ascending. The next chunk's copies are in flight
+// while this one is multiplied.
 template <bool kBf16>
-__global__ void __launch_bounds__(64) router_segment_kernel(const void* __restrict__ x,
-                                                            const float* __restrict__ wr,
-                                                            float* __restrict__ P, int T, int H,
-                                                            int E) {
-    __shared__ __align__(16) float xs[RT_KC][RT_XP];
-    __shared__ __align__(16) float ws[RT_KC][RT_WP];
+__global__ void __launch_bounds__(RT_THREADS, 2) router_segment_kernel(const void* __restrict__ x,
+                                                                       const float* __restrict__ wr,
+                                                                       float* __restrict__ P, int T, int H,
+                                                                       int E) {
+    extern __shared__ __align__(16) uint8_t rt_smem[];
+    RouterSmem& sm = *reinterpret_cast<RouterSmem*>(rt_smem);
     const int t0 = blockIdx.x * RT_BT, e0 = blockIdx.y * RT_BE, s = blockIdx.z;
-    const int ty = threadIdx.x >> 2, tx = threadIdx.x & 3;   // tokens ty*8.., experts tx*8..
+    const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
 
-    float acc[8][8];
+    float acc[4][RT_EJ];
 #pragma unroll
-    for (int a = 0; a < 8; ++a)
+    for (int a = 0; a < 4; ++a)
 #pragma unroll
-        for (int b = 0; b < 8; ++b) acc[a][b] = 0.0f;
+        for (int j = 0; j < RT_EJ; ++j) acc[a][j] = 0.0f;
 
-    for (int kc = 0; kc < RT_SEG; kc += RT_KC) {
-        const int h0 = s * RT_SEG + kc;
-        load_x_chunk<kBf16>(x, T, H, t0, h0, xs);
-        load_w_chunk(wr, E, H, e0, h0, ws);
-        __syncthreads();
-#pragma unroll 4
-        for (int k = 0; k < RT_KC; ++k) {
-            const float4 x0 = *reinterpret_cast<const float4*>(&xs[k][ty * 8]);
-            const float4 x1 = *reinterpret_cast<const float4*>(&xs[k][ty * 8 + 4]);
-            const float4 w0 = *reinterpret_cast<const float4*>(&ws[k][tx * 8]);
-            const float4 w1 = *reinterpret_cast<const float4*>(&ws[k][tx * 8 + 4]);
-            const float xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-            const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+    constexpr int NCHUNK = RT_SEG / RT_KC;
+    float xv_next[8];
+    issue_w_chunk(wr, E, H, e0, s * RT_SEG, sm.ws[0]);
+    load_x_chunk<kBf16>(x, T, H, t0, s * RT_SEG, xv_next);
+    store_x_chunk(xv_next, sm.xs[0]);
+    cp_async_wait_all();
+    __syncthreads();
+
+#pragma unroll 1
+    for (int c = 0; c < NCHUNK; ++c) {
+        const int buf = c & 1;
+        const bool more = c + 1 < NCHUNK;
+        if (more) {
+            const int h1 = s * RT_SEG + (c + 1) * RT_KC;
+            issue_w_chunk(wr, E, H, e0, h1, sm.ws[buf ^ 1]);
+            load_x_chunk<kBf16>(x, T, H, t0, h1, xv_next);
+        }
+        const float (*xs)[RT_XP] = sm.xs[buf];
+        const float (*ws)[RT_WP] = sm.ws[buf];
 #pragma unroll
-            for (int a = 0; a < 8; ++a)
+        for (int k4 = 0; k4 < RT_KC; k4 += 4) {
+            float xv[4][4];   // [token][k]
 #pragma unroll
-                for (int b = 0; b < 8; ++b) acc[a][b] = __fmaf_rn(xv[a], wv[b], acc[a][b]);
+            for (int kk = 0; kk < 4; ++kk) {
+                const float4 v = *reinterpret_cast<const float4*>(&xs[k4 + kk][ty * 4]);
+                xv[0][kk] = v.x; xv[1][kk] = v.y; xv[2][kk] = v.z; xv[3][kk] = v.w;
+            }
+#pragma unroll
+            for (int j = 0; j < RT_EJ; ++j) {
+                const float4 w = *reinterpret_cast<const float4*>(&ws[tx + RT_EL * j][k4]);
+#pragma unroll
+                for (int a = 0; a < 4; ++a) {
+                    float r = acc[a][j];
+                    r = __fmaf_rn(xv[a][0], w.x, r);
+                    r = __fmaf_rn(xv[a][1], w.y, r);
+                    r = __fmaf_rn(xv[a][2], w.z, r);
+                    r = __fmaf_rn(xv[a][3], w.w, r);
+                    acc[a][j] = r;
+                }
+            }
+        }
+        if (more) {
+            store_x_chunk(xv_next, sm.xs[buf ^ 1]);
+            cp_async_wait_all();
         }
         __syncthreads();
     }
     float* out = P + static_cast<size_t>(s) * T * E;
 #pragma unroll
-    for (int a = 0; a < 8; ++a) {
-        const int t = t0 + ty * 8 + a;
+    for (int a = 0; a < 4; ++a) {
+        const int t = t0 + ty * 4 + a;
         if (t >= T) continue;
 #pragma unroll
-        for (int b = 0; b < 8; ++b) {
-            const int e = e0 + tx * 8 + b;
-            if (e < E) out[static_cast<size_t>(t) * E + e] = acc[a][b];
+        for (int j = 0; j < RT_EJ; ++j) {
+            const int e = e0 + tx + RT_EL * j;
+            if (e < E) out[static_cast<size_t>(t) * E + e] = acc[a][j];
         }
     }
 }
@@ -239,11 +272,21 @@ cudaError_t launch_route(const moe_shape& s, const void* x, const float* wr, con
     const int split = router_split_count(T, H);
     dim3 grid(ceil_div(T, RT_BT), ceil_div(E, RT_BE), split);
     {
+        constexpr int smem = static_cast<int>(sizeof(RouterSmem));
+        static std::once_flag once;
+        static cudaError_t attr_err = cudaSuccess;
+        std::call_once(once, [] {
+            attr_err = cudaFuncSetAttribute(router_segment_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            if (attr_err == cudaSuccess)
+                attr_err = cudaFuncSetAttribute(router_segment_kernel<false>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        });
+        if (attr_err != cudaSuccess) return attr_err;
         ProfileScope ps("route_logits", st);
         if (s.act_dtype == MOE_BF16)
-            router_segment_kernel<true><<<grid, 64, 0, st>>>(x, wr, partials, T, H, E);
+            router_segment_kernel<true><<<grid, RT_THREADS, smem, st>>>(x, wr, partials, T, H, E);
         else
-            router_segment_kernel<false><<<grid, 64, 0, st>>>(x, wr, partials, T, H, E);
+            router_segment_kernel<false><<<grid, RT_THREADS, smem, st>>>(x, wr, partials, T, H, E);
         note_launch();
     }
     {

@@ -13,12 +13,14 @@ from tests.parity_util import rel_err, to_f64, tol_of
 pytestmark = pytest.mark.gpu
 
 
-def test_wait_timeout_is_reported_and_the_context_survives():
+@pytest.mark.parametrize("impl", [_lib.MOE_FFN_AUTO, _lib.MOE_FFN_TCGEN05_PAIR, _lib.MOE_FFN_TCGEN05_WIDE],
+                         ids=["auto", "cta_pair", "cta_pair_wide"])
+def test_wait_timeout_is_reported_and_the_context_survives(impl):
     build.build()
     cfg = synth.variant(synth.CONFIGS["prefill_bf16"], T=64, H=512, I=128, n_routed=8, top_k=2)
     inp = synth.make_inputs(cfg)
     d = synth.to_device(inp, "cuda")
-    layer = MoELayer(cfg, d)
+    layer = MoELayer(cfg, d, impl=impl)
     _lib.moe_inject_wait_timeout(1)
     layer.forward(d["x"])
     assert layer.status() == _lib.MOE_ERR_TIMEOUT

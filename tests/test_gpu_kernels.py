@@ -10,7 +10,8 @@ import torch
 import oracle
 from shared_routed_expert_b200 import _lib, build, synth
 from shared_routed_expert_b200._lib import (MOE_FFN_SIMT, MOE_FFN_TCGEN05, MOE_FFN_TCGEN05_M128,
-                                            MOE_FFN_TCGEN05_M256)
+                                            MOE_FFN_TCGEN05_M256, MOE_FFN_TCGEN05_PAIR,
+                                            MOE_FFN_TCGEN05_WIDE)
 from tests.parity_util import oracle_logits, rel_err, to_f64, tol_of
 
 pytestmark = pytest.mark.gpu
@@ -158,8 +159,8 @@ FFN_CASES = {
 }
 
 
-IMPLS = [MOE_FFN_SIMT, MOE_FFN_TCGEN05_M128, MOE_FFN_TCGEN05_M256]
-IMPL_IDS = ["simt", "tcgen05_m128", "tcgen05_m256"]
+IMPLS = [MOE_FFN_SIMT, MOE_FFN_TCGEN05_M128, MOE_FFN_TCGEN05_M256, MOE_FFN_TCGEN05_PAIR, MOE_FFN_TCGEN05_WIDE]
+IMPL_IDS = ["simt", "tcgen05_m128", "tcgen05_m256", "tcgen05_pair", "tcgen05_wide"]
 
 
 @pytest.mark.parametrize("name", list(FFN_CASES))
