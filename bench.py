@@ -190,8 +190,8 @@ def algorithmic(cfg, kernel: str, counts: np.ndarray | None):
     if kernel.startswith("gemm1"):
         return 2.0 * R * 2 * I * H, touched * 2 * I * H * wb + R * H * xb + R * I * ab
     if kernel.startswith("gemm2"):
-        # combine fused in: reads h, writes fp32 partial sums of [T, H] (L2-resident)
-        return 2.0 * R * I * H, touched * H * I * wb + R * I * xb + T * H * 4
+        # reads h, writes the expert rows y as scaled fp16 plus one exponent byte per 32 columns
+        return 2.0 * R * I * H, touched * H * I * wb + R * I * xb + R * H * 2 + R * (H // 32)
     if kernel == "route_logits":
         return None, T * H * ab + Er * H * 4 + (H // 256) * T * Er * 4
     if kernel == "combine":
@@ -207,13 +207,14 @@ def algorithmic(cfg, kernel: str, counts: np.ndarray | None):
 # capture of the same kernel variant on a 1024-token, 32-routed-expert case of
 # the bf16 workload (its per-expert row counts match the full one). Traffic is
 # dominated by the touched experts' weights, so it scales with the launch.
-# Keyed by (kernel, weight dtype, rows per tensor-core unit).
-PROFILED_TRAFFIC_RATIO = {("gemm1_tc", "bf16", 256): 1.09, ("gemm2_tc", "bf16", 256): 0.97}
+# Keyed by (kernel, weight dtype, tensor-core work unit).
+PROFILED_TRAFFIC_RATIO = {("gemm1_tc", "bf16", 256): 1.09,
+                          ("gemm1_tc", "bf16", "pair256x512"): 1.02, ("gemm2_tc", "bf16", "pair256x512"): 0.97}
 
 
 def unit_rows(cfg, ffn: str):
-    """Tensor-core work unit the run uses: 128, 256 (one CTA) or "pair256"
-    (256 rows over a CTA pair)."""
+    """Tensor-core work unit the run uses: 128, 256 (one CTA), "pair256"
+    (256 x 256 tiles over a CTA pair) or "pair256x512" (256 x 512 pair tiles)."""
     if ffn == "tcgen05_m128":
         return 128
     if ffn == "tcgen05_m256":
@@ -222,7 +223,7 @@ def unit_rows(cfg, ffn: str):
         return "pair256"
     if ffn == "tcgen05_wide":
         return "pair256x512"
-    return 256 if (cfg.w_dtype == "bf16" and cfg.rows >= 192 * cfg.n_experts) else 128
+    return "pair256x512" if (cfg.w_dtype == "bf16" and cfg.rows >= 192 * cfg.n_experts) else 128
 
 
 def roofline_of(cfg, kernel: str, ms_per_launch: float, counts, pk, urows=128) -> dict:

@@ -75,9 +75,9 @@ typedef struct moe_shape {
 
 /* Kernel choice for the expert GEMMs. AUTO picks the tcgen05 tensor-core
  * kernels for bf16/E4M3 weights and the CUDA-core kernels for fp32. TCGEN05
- * picks the tensor-core work unit itself: 256 rows (two 128-row tiles of one
- * expert sharing each weight tile) for bf16 weights when groups average >= 192
- * rows, else 128;
+ * picks the tensor-core work unit itself: for bf16 weights whose groups average
+ * >= 192 rows, 256 x 512 tiles on CTA pairs (as TCGEN05_WIDE), else 128-row
+ * units on single CTAs (as TCGEN05_M128);
  * TCGEN05_M128 / TCGEN05_M256 force one of them; TCGEN05_PAIR forces 256-row
  * units split over a pair of CTAs on the two SMs of a TPC (tcgen05 cta_group::2,
  * each SM staging half of every weight tile); TCGEN05_WIDE the same with

@@ -914,10 +914,16 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
     }
 
     // CTA pairs (cta_pair > 0); 256 x 512 pair tiles (cta_pair == 2) where the
-    // output width divides into them (GEMM1: I % 256, GEMM2: H % 512)
-    const bool two_sm = a.cta_pair > 0;
-    const bool wide1 = a.cta_pair == 2 && half == 128 && a.I % 256 == 0;
-    const bool wide2 = a.cta_pair == 2 && a.H % 512 == 0;
+    // output width divides into them (GEMM1: I % 256, GEMM2: H % 512). Chosen by
+    // default for bf16 layers whose groups average >= 192 rows: measured on B200,
+    // prefill_bf16 GEMM1 + GEMM2 1.86 ms with pair tiles vs 1.91 ms with
+    // single-CTA 256-row units; E4M3 layers and small groups are faster on
+    // single-CTA 128-row units (prefill_fp8 4.95 vs 6.29 ms per layer).
+    const bool big_bf16 = a.w_dtype == MOE_BF16 && a.R >= 192 * a.E;
+    const int cta_pair = a.cta_pair >= 0 ? a.cta_pair : ((a.unit_rows == 0 && big_bf16) ? 2 : 0);
+    const bool two_sm = cta_pair > 0;
+    const bool wide1 = cta_pair == 2 && half == 128 && a.I % 256 == 0;
+    const bool wide2 = cta_pair == 2 && a.H % 512 == 0;
     const int bn1 = wide1 ? 2 * half : half;     // h columns per unit
 
     // GEMM1: A = Xp [R, H] (rows gathered by the gather kernel); B = W13 viewed as
@@ -957,12 +963,10 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
     p.status = a.status;
     p.wait_limit = inject ? (20ll << 20) : (4ll << 30);
     p.inject_stall = inject;
-    // M = 256 units (two m-tiles sharing each weight stage) for bf16 layers whose
-    // groups average >= 192 rows; 128-row units otherwise. Measured on B200:
-    // prefill_bf16 2.38 vs 2.43 ms per layer (256 vs 128), but E4M3 layers are
-    // faster with 128-row units (prefill_fp8 4.95 vs 6.04 ms, skewed_fp8 0.84 vs 0.99 ms).
-    const bool pair = a.unit_rows == 256 ||
-                      (a.unit_rows == 0 && a.w_dtype == MOE_BF16 && a.R >= 192 * a.E);
+    // single-CTA units: M = 256 (two m-tiles sharing each weight stage) when
+    // forced, 128 rows otherwise (measured on B200: E4M3 layers are faster with
+    // 128-row units, prefill_fp8 4.95 vs 6.04 ms, skewed_fp8 0.84 vs 0.99 ms)
+    const bool pair = a.unit_rows == 256;
     cudaError_t err;
     if (two_sm)
         err = fp8 ? launch_gemm1_pair<true>(ta, tb, ta2, p, half, wide1, st)

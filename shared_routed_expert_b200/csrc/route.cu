@@ -19,7 +19,14 @@ namespace sre {
 
 namespace {
 
-constexpr int RT_BT = 64;      // tokens per block
+#ifndef SRE_RT_TPT
+#define SRE_RT_TPT 4           // tokens per thread: 4 or 8
+#endif
+#ifndef SRE_RT_MINB
+#define SRE_RT_MINB 2          // resident blocks per SM the register budget aims for
+#endif
+constexpr int RT_TPT = SRE_RT_TPT;
+constexpr int RT_BT = 16 * RT_TPT;     // tokens per block (16 token groups)
 constexpr int RT_EL = 16;      // expert lanes per block
 constexpr int RT_EJ = 10;      // experts per thread (strided by RT_EL)
 constexpr int RT_BE = RT_EL * RT_EJ;   // experts per block (160)
@@ -55,48 +62,74 @@ __device__ __forceinline__ void issue_w_chunk(const float* wr, int E, int H, int
     cp_async_commit();
 }
 
-// x chunk: 64 tokens x 32 h; thread i holds token t0 + i % 64, h h0 + 8 (i / 64) .. +7
+// x chunk: RT_BT tokens x 32 h in pieces of 8 h; piece p = thread + 256 g holds
+// token t0 + p % RT_BT, h h0 + 8 (p / RT_BT) .. +7
+constexpr int RT_XG = RT_BT * RT_KC / 8 / RT_THREADS;   // pieces per thread
+
+// The next chunk's x is held raw (bf16 pairs or fp32 bits) in registers while
+// the current chunk is multiplied, and converted when stored.
 template <bool kBf16>
-__device__ __forceinline__ void load_x_chunk(const void* x, int T, int H, int t0, int h0, float (&v)[8]) {
-    const int t = t0 + (threadIdx.x & (RT_BT - 1));
-    const int q = (threadIdx.x >> 6) * 8;
-    if (t < T) {
+struct XStage {
+    static constexpr int N = RT_XG * (kBf16 ? 4 : 8);   // 32-bit words per thread
+    uint32_t w[N];
+};
+
+template <bool kBf16>
+__device__ __forceinline__ void load_x_chunk(const void* x, int T, int H, int t0, int h0, XStage<kBf16>& st) {
+#pragma unroll
+    for (int g = 0; g < RT_XG; ++g) {
+        const int piece = threadIdx.x + g * RT_THREADS;
+        const int t = t0 + (piece & (RT_BT - 1));
+        const int q = (piece / RT_BT) * 8;
         if constexpr (kBf16) {
-            const uint4 a = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) +
-                                                            static_cast<size_t>(t) * H + h0 + q);
-            const uint32_t w[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                v[2 * j] = __uint_as_float(w[j] << 16);
-                v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-            }
+            uint4 a = make_uint4(0u, 0u, 0u, 0u);
+            if (t < T)
+                a = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + static_cast<size_t>(t) * H + h0 + q);
+            st.w[4 * g] = a.x; st.w[4 * g + 1] = a.y; st.w[4 * g + 2] = a.z; st.w[4 * g + 3] = a.w;
         } else {
-            const float* p = static_cast<const float*>(x) + static_cast<size_t>(t) * H + h0 + q;
-            const float4 a = *reinterpret_cast<const float4*>(p);
-            const float4 b = *reinterpret_cast<const float4*>(p + 4);
-            v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-            v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+            float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+            if (t < T) {
+                const float* p = static_cast<const float*>(x) + static_cast<size_t>(t) * H + h0 + q;
+                a = *reinterpret_cast<const float4*>(p);
+                b = *reinterpret_cast<const float4*>(p + 4);
+            }
+            st.w[8 * g] = __float_as_uint(a.x); st.w[8 * g + 1] = __float_as_uint(a.y);
+            st.w[8 * g + 2] = __float_as_uint(a.z); st.w[8 * g + 3] = __float_as_uint(a.w);
+            st.w[8 * g + 4] = __float_as_uint(b.x); st.w[8 * g + 5] = __float_as_uint(b.y);
+            st.w[8 * g + 6] = __float_as_uint(b.z); st.w[8 * g + 7] = __float_as_uint(b.w);
         }
-    } else {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = 0.0f;
     }
 }
 
-__device__ __forceinline__ void store_x_chunk(const float (&v)[8], float (*xs)[RT_XP]) {
-    const int tl = threadIdx.x & (RT_BT - 1);
-    const int q = (threadIdx.x >> 6) * 8;
+// transposed into xs[k][t] as fp32 (bf16 -> fp32 is exact)
+template <bool kBf16>
+__device__ __forceinline__ void store_x_chunk(const XStage<kBf16>& st, float (*xs)[RT_XP]) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) xs[q + j][tl] = v[j];
+    for (int g = 0; g < RT_XG; ++g) {
+        const int piece = threadIdx.x + g * RT_THREADS;
+        const int tl = piece & (RT_BT - 1);
+        const int q = (piece / RT_BT) * 8;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            float v;
+            if constexpr (kBf16) {
+                const uint32_t pr = st.w[4 * g + (j >> 1)];
+                v = __uint_as_float((j & 1) ? (pr & 0xFFFF0000u) : (pr << 16));
+            } else {
+                v = __uint_as_float(st.w[8 * g + j]);
+            }
+            xs[q + j][tl] = v;
+        }
+    }
 }
 
-// grid (ceil(T/64), ceil(E/160), H/256); 256 threads: thread (ty, tx) =
-// (threadIdx / 16, threadIdx % 16) owns tokens t0 + 4 ty .. +3 and experts
-// e0 + tx + 16 j (j < 10). P[s][t][e] = fma chain over the 256 h of segment s
+// grid (ceil(T/RT_BT), ceil(E/160), H/256); 256 threads: thread (ty, tx) =
+// (threadIdx / 16, threadIdx % 16) owns tokens t0 + RT_TPT ty .. +RT_TPT-1 and
+// experts e0 + tx + 16 j (j < 10). P[s][t][e] = fma chain over the 256 h of segment s
 // (blockIdx.z), from +0, h ascending. The next chunk's copies are in flight
 // while this one is multiplied.
 template <bool kBf16>
-__global__ void __launch_bounds__(RT_THREADS, 2) router_segment_kernel(const void* __restrict__ x,
+__global__ void __launch_bounds__(RT_THREADS, SRE_RT_MINB) router_segment_kernel(const void* __restrict__ x,
                                                                        const float* __restrict__ wr,
                                                                        float* __restrict__ P, int T, int H,
                                                                        int E) {
@@ -105,17 +138,17 @@ __global__ void __launch_bounds__(RT_THREADS, 2) router_segment_kernel(const voi
     const int t0 = blockIdx.x * RT_BT, e0 = blockIdx.y * RT_BE, s = blockIdx.z;
     const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
 
-    float acc[4][RT_EJ];
+    float acc[RT_TPT][RT_EJ];
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
+    for (int a = 0; a < RT_TPT; ++a)
 #pragma unroll
         for (int j = 0; j < RT_EJ; ++j) acc[a][j] = 0.0f;
 
     constexpr int NCHUNK = RT_SEG / RT_KC;
-    float xv_next[8];
+    XStage<kBf16> xnext;
     issue_w_chunk(wr, E, H, e0, s * RT_SEG, sm.ws[0]);
-    load_x_chunk<kBf16>(x, T, H, t0, s * RT_SEG, xv_next);
-    store_x_chunk(xv_next, sm.xs[0]);
+    load_x_chunk<kBf16>(x, T, H, t0, s * RT_SEG, xnext);
+    store_x_chunk<kBf16>(xnext, sm.xs[0]);
     cp_async_wait_all();
     __syncthreads();
 
@@ -126,23 +159,26 @@ __global__ void __launch_bounds__(RT_THREADS, 2) router_segment_kernel(const voi
         if (more) {
             const int h1 = s * RT_SEG + (c + 1) * RT_KC;
             issue_w_chunk(wr, E, H, e0, h1, sm.ws[buf ^ 1]);
-            load_x_chunk<kBf16>(x, T, H, t0, h1, xv_next);
+            load_x_chunk<kBf16>(x, T, H, t0, h1, xnext);
         }
         const float (*xs)[RT_XP] = sm.xs[buf];
         const float (*ws)[RT_WP] = sm.ws[buf];
 #pragma unroll
         for (int k4 = 0; k4 < RT_KC; k4 += 4) {
-            float xv[4][4];   // [token][k]
+            float xv[RT_TPT][4];   // [token][k]
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-                const float4 v = *reinterpret_cast<const float4*>(&xs[k4 + kk][ty * 4]);
-                xv[0][kk] = v.x; xv[1][kk] = v.y; xv[2][kk] = v.z; xv[3][kk] = v.w;
+#pragma unroll
+                for (int a4 = 0; a4 < RT_TPT; a4 += 4) {
+                    const float4 v = *reinterpret_cast<const float4*>(&xs[k4 + kk][ty * RT_TPT + a4]);
+                    xv[a4][kk] = v.x; xv[a4 + 1][kk] = v.y; xv[a4 + 2][kk] = v.z; xv[a4 + 3][kk] = v.w;
+                }
             }
 #pragma unroll
             for (int j = 0; j < RT_EJ; ++j) {
                 const float4 w = *reinterpret_cast<const float4*>(&ws[tx + RT_EL * j][k4]);
 #pragma unroll
-                for (int a = 0; a < 4; ++a) {
+                for (int a = 0; a < RT_TPT; ++a) {
                     float r = acc[a][j];
                     r = __fmaf_rn(xv[a][0], w.x, r);
                     r = __fmaf_rn(xv[a][1], w.y, r);
@@ -153,15 +189,15 @@ __global__ void __launch_bounds__(RT_THREADS, 2) router_segment_kernel(const voi
             }
         }
         if (more) {
-            store_x_chunk(xv_next, sm.xs[buf ^ 1]);
+            store_x_chunk<kBf16>(xnext, sm.xs[buf ^ 1]);
             cp_async_wait_all();
         }
         __syncthreads();
     }
     float* out = P + static_cast<size_t>(s) * T * E;
 #pragma unroll
-    for (int a = 0; a < 4; ++a) {
-        const int t = t0 + ty * 4 + a;
+    for (int a = 0; a < RT_TPT; ++a) {
+        const int t = t0 + ty * RT_TPT + a;
         if (t >= T) continue;
 #pragma unroll
         for (int j = 0; j < RT_EJ; ++j) {
