@@ -19,6 +19,7 @@ import statistics
 import subprocess
 import sys
 import tempfile
+import threading
 import time
 
 import numpy as np
@@ -89,17 +90,51 @@ class Dist:
 # ------------------------------------------------------------------ clocks
 
 class Clocks:
-    """nvidia-smi sampling every 200 ms while the timed region runs."""
+    """SM clock and clock-event reasons sampled while the timed region runs:
+    through NVML every 5 ms (the library nvidia-smi reads), else nvidia-smi
+    every 200 ms."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, gpu_index: str):
         self.idx = gpu_index
         self.proc = None
         self.path = None
+        self.thread = None
+        self.nvml = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        if self.idx.startswith(("GPU-", "MIG-")):
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID(self.idx)
+        return pynvml, pynvml.nvmlDeviceGetHandleByIndex(int(self.idx))
 
     def start(self):
+        try:
+            nv, h = self._nvml_handle()
+        except Exception:       # no NVML: fall back to nvidia-smi
+            nv = None
+        if nv is not None:
+            bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                    "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                    "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                    "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+            self.nvml = {"sm": [], "reasons": set(), "stop": threading.Event(),
+                         "max": nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)}
+
+            def run():
+                st = self.nvml
+                while not st["stop"].is_set():
+                    st["sm"].append(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    st["reasons"].update(n for n, b in bits.items() if r & b)
+                    st["stop"].wait(0.005)
+            self.thread = threading.Thread(target=run, daemon=True)
+            self.thread.start()
+            return
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
         try:
@@ -110,13 +145,19 @@ class Clocks:
             self.proc = None
 
     def stop(self) -> dict:
+        if self.thread is not None:
+            st = self.nvml
+            st["stop"].set()
+            self.thread.join(timeout=5)
+            sm = st["sm"]
+            return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": st["max"],
+                    "reasons": sorted(st["reasons"]), "samples": len(sm), "source": "nvml, 5 ms"}
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         time.sleep(0.25)
         self.proc.terminate()
         self.proc.wait(timeout=10)
         sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in open(self.path):
             f = [c.strip() for c in line.split(",")]
             if len(f) < 9:
@@ -126,12 +167,12 @@ class Clocks:
                 smax = float(f[2])
             except ValueError:
                 continue
-            for n, v in zip(names, f[5:9]):
+            for n, v in zip(self.NAMES, f[5:9]):
                 if v.lower() in ("active", "1"):
                     reasons.add(n)
         os.unlink(self.path)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "source": "nvidia-smi, 200 ms"}
 
 
 # ------------------------------------------------------------------ timing
@@ -328,7 +369,7 @@ def describe(cfg) -> str:
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="prefill_bf16", choices=list(synth.CONFIGS))
@@ -380,7 +421,6 @@ def main():
     # timed region: device-resident inputs, per-kernel events on the launching stream
     vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
     clocks = Clocks(vis.split(",")[dist.local] if vis else str(dist.local))
-    clocks.start()
     _lib.moe_profile_reset()
     n0 = _lib.moe_launch_count()
     _lib.moe_profile_enable(True)
@@ -389,10 +429,11 @@ def main():
     torch.cuda.synchronize()
     _lib.moe_profile_reset()
     n0 = _lib.moe_launch_count()
+    clocks.start()
     ms = time_steps(step, args.steps, 0, dist, stream)
+    clk = clocks.stop()
     launches = _lib.moe_launch_count() - n0
     _lib.moe_profile_enable(False)
-    clk = clocks.stop()
     tab = kernel_table(args.steps)
     st = fused.status()
     if st != _lib.MOE_OK:
