@@ -18,6 +18,7 @@ namespace sre {
 namespace {
 
 constexpr int CB_THREADS = 128;
+constexpr int CB_BATCH = 5;      // slot rows loaded together (S = 9: two groups)
 
 // bf16 rows: each thread owns 8-element vectors of the token's row.
 __global__ void __launch_bounds__(CB_THREADS) combine_bf16_kernel(int T, int S, int H,
@@ -123,16 +124,31 @@ __global__ void __launch_bounds__(CB_THREADS) combine_f16s_kernel(int T, int S, 
         float acc[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
-        for (int k = 0; k < S; ++k) {
-            const size_t r = static_cast<size_t>(s_row[k]);
-            const uint4 q = y[r * nv + i];
-            const float wk = s_w[k] * exp2_int(yexp[r * ne + (i >> 2)]);
-            const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+        // slots in groups of CB_BATCH: the group's row loads are all in flight
+        // before the first of them is accumulated (accumulation stays in slot order)
+        for (int k0 = 0; k0 < S; k0 += CB_BATCH) {
+            uint4 q[CB_BATCH];
+            int8_t ex[CB_BATCH];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float2 f = unpack_f16x2(u[j]);
-                acc[2 * j] = __fmaf_rn(wk, f.x, acc[2 * j]);
-                acc[2 * j + 1] = __fmaf_rn(wk, f.y, acc[2 * j + 1]);
+            for (int g = 0; g < CB_BATCH; ++g) {
+                if (k0 + g < S) {
+                    const size_t r = static_cast<size_t>(s_row[k0 + g]);
+                    q[g] = y[r * nv + i];
+                    ex[g] = yexp[r * ne + (i >> 2)];
+                }
+            }
+#pragma unroll
+            for (int g = 0; g < CB_BATCH; ++g) {
+                if (k0 + g < S) {
+                    const float wk = s_w[k0 + g] * exp2_int(ex[g]);
+                    const uint32_t u[4] = {q[g].x, q[g].y, q[g].z, q[g].w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float2 f = unpack_f16x2(u[j]);
+                        acc[2 * j] = __fmaf_rn(wk, f.x, acc[2 * j]);
+                        acc[2 * j + 1] = __fmaf_rn(wk, f.y, acc[2 * j + 1]);
+                    }
+                }
             }
         }
         if (add != nullptr) {
