@@ -10,8 +10,8 @@
 // Three kernels, no atomics on the order-defining path:
 //   hist:    per 512-slot chunk, per-expert counts (shared-memory histogram)
 //   scan:    one block; warp-parallel scans over chunks (per expert) and over
-//            experts give each chunk's first row per expert, the counts, the
-//            offsets and the GEMM tile prefix
+//            experts give each chunk's first row inside each expert's group,
+//            the counts, the offsets and the GEMM tile prefix
 //   scatter: one warp per chunk walks its slots in order, 32 at a time;
 //            __match_any_sync ranks equal experts inside a group.
 #include "kernels.cuh"
@@ -51,24 +51,51 @@ __device__ __forceinline__ int warp_inclusive_scan(int v, int lane) {
     return v;
 }
 
-// One block of 1024 threads. Warp w owns experts w, w+32, ...:
-//   counts[e] = sum over chunks; offsets = exclusive scan over experts;
-//   chunk_hist[e][c] <- offsets[e] + sum_{c' < c} chunk_hist[e][c'] (each chunk's first row)
-// Also the GEMM tile prefix tile_off[e] = sum_{e' < e} ceil(counts[e'] / kTileM).
+// One block of 1024 threads. Warp w owns experts w, w+32, ...: the expert's
+// row of chunk counts is read 32 consecutive chunks per instruction, every
+// load of the row in flight before the scans (rows of up to 32 * kScanVals
+// chunks; longer rows go 32 chunks per round trip). Writes
+// chunk_hist[e][c] <- sum_{c' < c} chunk_hist[e][c'] (the chunk's first row
+// inside expert e's group) and counts[e]; warp 0 then scans the counts into
+// offsets and the GEMM tile prefix tile_off[e] = sum_{e' < e} ceil(counts[e'] /
+// kTileM). The scatter adds offsets[e].
+constexpr int kScanVals = 12;    // 32-chunk groups per row held in registers (n_chunks <= 384)
 __global__ void __launch_bounds__(1024) perm_scan_kernel(int n_chunks, int E, int32_t* __restrict__ chunk_hist,
                                                          int32_t* __restrict__ counts,
                                                          int32_t* __restrict__ offsets,
                                                          int32_t* __restrict__ tile_off) {
     __shared__ int32_t s_cnt[1024];
-    __shared__ int32_t s_off[1025];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int groups = ceil_div(n_chunks, 32);
     for (int e = warp; e < E; e += 32) {
-        const int32_t* row = chunk_hist + static_cast<size_t>(e) * n_chunks;
-        int sum = 0;
-        for (int c = lane; c < n_chunks; c += 32) sum += row[c];
+        int32_t* row = chunk_hist + static_cast<size_t>(e) * n_chunks;
+        int carry = 0;
+        if (groups <= kScanVals) {
+            int v[kScanVals];
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, off);
-        if (lane == 0) s_cnt[e] = sum;
+            for (int g = 0; g < kScanVals; ++g) {
+                const int c = g * 32 + lane;
+                v[g] = (g < groups && c < n_chunks) ? row[c] : 0;
+            }
+#pragma unroll
+            for (int g = 0; g < kScanVals; ++g) {
+                if (g < groups) {
+                    const int c = g * 32 + lane;
+                    const int inc = warp_inclusive_scan(v[g], lane);
+                    if (c < n_chunks) row[c] = carry + inc - v[g];
+                    carry += __shfl_sync(0xFFFFFFFFu, inc, 31);
+                }
+            }
+        } else {
+            for (int cb = 0; cb < n_chunks; cb += 32) {
+                const int c = cb + lane;
+                const int v = (c < n_chunks) ? row[c] : 0;
+                const int inc = warp_inclusive_scan(v, lane);
+                if (c < n_chunks) row[c] = carry + inc - v;
+                carry += __shfl_sync(0xFFFFFFFFu, inc, 31);
+            }
+        }
+        if (lane == 0) s_cnt[e] = carry;
     }
     __syncthreads();
     if (warp == 0) {
@@ -80,7 +107,6 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(int n_chunks, int E, in
             const int inc = warp_inclusive_scan(c, lane);
             const int tinc = warp_inclusive_scan(tc, lane);
             if (e < E) {
-                s_off[e] = carry + inc - c;
                 counts[e] = c;
                 offsets[e] = carry + inc - c;
                 tile_off[e] = tcarry + tinc - tc;
@@ -89,21 +115,8 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(int n_chunks, int E, in
             tcarry += __shfl_sync(0xFFFFFFFFu, tinc, 31);
         }
         if (lane == 0) {
-            s_off[E] = carry;
             offsets[E] = carry;
             tile_off[E] = tcarry;
-        }
-    }
-    __syncthreads();
-    for (int e = warp; e < E; e += 32) {
-        int32_t* row = chunk_hist + static_cast<size_t>(e) * n_chunks;
-        int carry = s_off[e];
-        for (int c0 = 0; c0 < n_chunks; c0 += 32) {
-            const int c = c0 + lane;
-            const int v = (c < n_chunks) ? row[c] : 0;
-            const int inc = warp_inclusive_scan(v, lane);
-            if (c < n_chunks) row[c] = carry + inc - v;
-            carry += __shfl_sync(0xFFFFFFFFu, inc, 31);
         }
     }
 }
@@ -115,11 +128,13 @@ constexpr int kPermPerLane = kPermChunk / 32;
 __global__ void __launch_bounds__(32) perm_scatter_kernel(const int32_t* __restrict__ ids, int R, int E,
                                                           int n_chunks,
                                                           const int32_t* __restrict__ chunk_base,
+                                                          const int32_t* __restrict__ offsets,
                                                           int32_t* __restrict__ perm,
                                                           int32_t* __restrict__ inv) {
     extern __shared__ int32_t next[];
     const int lane = threadIdx.x;
-    for (int e = lane; e < E; e += 32) next[e] = chunk_base[static_cast<size_t>(e) * n_chunks + blockIdx.x];
+    for (int e = lane; e < E; e += 32)
+        next[e] = offsets[e] + chunk_base[static_cast<size_t>(e) * n_chunks + blockIdx.x];
     const int base = blockIdx.x * kPermChunk;
     int my[kPermPerLane];
 #pragma unroll
@@ -230,7 +245,7 @@ cudaError_t launch_permute(int R, int E, const int32_t* ids, int32_t* counts, in
     }
     if (n_chunks > 0) {
         ProfileScope ps("permute_scatter", stream);
-        perm_scatter_kernel<<<n_chunks, 32, hsm, stream>>>(ids, R, E, n_chunks, scratch, perm, inv);
+        perm_scatter_kernel<<<n_chunks, 32, hsm, stream>>>(ids, R, E, n_chunks, scratch, offsets, perm, inv);
         note_launch();
     }
     return cudaGetLastError();

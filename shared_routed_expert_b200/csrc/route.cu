@@ -225,18 +225,37 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ P, 
     if (warp >= T) return;
     const int t = warp;
     const int S = K + (shared_id >= 0 ? 1 : 0);
+    // segment partials summed in segment order; TK_PB segments' loads are in
+    // flight before the first of them is added
+    constexpr int TK_PB = 4;
+    float tot[TK_MAXPL];
+#pragma unroll
+    for (int j = 0; j < TK_MAXPL; ++j) tot[j] = 0.0f;
+    for (int p0 = 0; p0 < n_part; p0 += TK_PB) {
+        float v[TK_PB][TK_MAXPL];
+#pragma unroll
+        for (int q = 0; q < TK_PB; ++q)
+#pragma unroll
+            for (int j = 0; j < TK_MAXPL; ++j) {
+                const int e = lane + 32 * j;
+                v[q][j] = (p0 + q < n_part && e < E) ? P[(static_cast<size_t>(p0 + q) * T + t) * E + e] : 0.0f;
+            }
+#pragma unroll
+        for (int q = 0; q < TK_PB; ++q)
+            if (p0 + q < n_part)
+#pragma unroll
+                for (int j = 0; j < TK_MAXPL; ++j) tot[j] = __fadd_rn(tot[j], v[q][j]);
+    }
     float key[TK_MAXPL];
 #pragma unroll
     for (int j = 0; j < TK_MAXPL; ++j) {
         const int e = lane + 32 * j;
         float v = -INFINITY;
         if (e < E) {
-            float tot = 0.0f;
-            for (int p = 0; p < n_part; ++p)
-                tot = __fadd_rn(tot, P[(static_cast<size_t>(p) * T + t) * E + e]);
-            if (bias != nullptr) tot = __fadd_rn(tot, bias[e]);
-            if (logits_out != nullptr) logits_out[static_cast<size_t>(t) * E + e] = tot;
-            v = isnan(tot) ? -INFINITY : tot;
+            float tj = tot[j];
+            if (bias != nullptr) tj = __fadd_rn(tj, bias[e]);
+            if (logits_out != nullptr) logits_out[static_cast<size_t>(t) * E + e] = tj;
+            v = isnan(tj) ? -INFINITY : tj;
         }
         key[j] = v;
     }
