@@ -201,7 +201,7 @@ def time_steps(fn, steps: int, warmup: int, dist: Dist, stream) -> float:
     return dist.max(e0.elapsed_time(e1))
 
 
-KERNELS = ["route_logits", "route_topk", "permute_hist", "permute_scan", "permute_scatter",
+KERNELS = ["route_logits", "route_topk", "permute_small", "permute_hist", "permute_scan", "permute_scatter",
            "quant_rows", "gather", "gemm1_tc", "gemm2_tc", "gemm1_simt", "gemm2_simt", "combine",
            "round_out"]
 

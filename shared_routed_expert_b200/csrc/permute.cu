@@ -161,6 +161,83 @@ __global__ void __launch_bounds__(32) perm_scatter_kernel(const int32_t* __restr
     }
 }
 
+// Small batches (R <= kSmallR slots, E <= kSmallE experts): the whole
+// permutation in one block of 1024 threads, same result as the three kernels
+// above. Counts by shared-memory histogram; offsets and tile prefix by a warp
+// scan; then rounds of 1024 slots in slot order: warp w ranks its 32 slots
+// with __match_any_sync, per-expert counts of the warps are scanned across
+// warps, and each slot's row is run[e] + (slots of e in lower warps) + rank.
+constexpr int kSmallR = 8192;
+constexpr int kSmallE = 256;
+__global__ void __launch_bounds__(1024) perm_small_kernel(const int32_t* __restrict__ ids, int R, int E,
+                                                          int32_t* __restrict__ counts,
+                                                          int32_t* __restrict__ offsets,
+                                                          int32_t* __restrict__ tile_off,
+                                                          int32_t* __restrict__ perm,
+                                                          int32_t* __restrict__ inv, DevStatus* status) {
+    __shared__ int32_t s_cnt[kSmallE];
+    __shared__ int32_t s_run[kSmallE];
+    __shared__ int32_t s_w[32][kSmallE];      // per round: slots of expert e in warp w, then its first row
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int e = tid; e < E; e += 1024) s_cnt[e] = 0;
+    __syncthreads();
+    for (int f = tid; f < R; f += 1024) {
+        const int e = ids[f];
+        if (e < 0 || e >= E) report(status, MOE_ERR_DEVICE, static_cast<unsigned>(f));
+        else atomicAdd(&s_cnt[e], 1);
+    }
+    __syncthreads();
+    if (warp == 0) {
+        int carry = 0, tcarry = 0;
+        for (int e0 = 0; e0 < E; e0 += 32) {
+            const int e = e0 + lane;
+            const int c = (e < E) ? s_cnt[e] : 0;
+            const int tc = ceil_div(c, kTileM);
+            const int inc = warp_inclusive_scan(c, lane);
+            const int tinc = warp_inclusive_scan(tc, lane);
+            if (e < E) {
+                counts[e] = c;
+                offsets[e] = carry + inc - c;
+                tile_off[e] = tcarry + tinc - tc;
+                s_run[e] = carry + inc - c;
+            }
+            carry += __shfl_sync(0xFFFFFFFFu, inc, 31);
+            tcarry += __shfl_sync(0xFFFFFFFFu, tinc, 31);
+        }
+        if (lane == 0) {
+            offsets[E] = carry;
+            tile_off[E] = tcarry;
+        }
+    }
+    const unsigned lt = (1u << lane) - 1u;
+    for (int base = 0; base < R; base += 1024) {
+        for (int i = tid; i < 32 * E; i += 1024) s_w[i / E][i % E] = 0;
+        __syncthreads();
+        const int f = base + tid;
+        int e = (f < R) ? ids[f] : -1;
+        if (e >= E) e = -1;
+        const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
+        if (e >= 0 && (peers & lt) == 0) s_w[warp][e] = __popc(peers);
+        __syncthreads();
+        for (int x = tid; x < E; x += 1024) {       // exclusive scan over warps, in warp order
+            int run = s_run[x];
+            for (int w = 0; w < 32; ++w) {
+                const int c = s_w[w][x];
+                s_w[w][x] = run;
+                run += c;
+            }
+            s_run[x] = run;
+        }
+        __syncthreads();
+        if (e >= 0) {
+            const int row = s_w[warp][e] + __popc(peers & lt);
+            perm[row] = f;
+            inv[f] = row;
+        }
+        __syncthreads();
+    }
+}
+
 // Xp[r] = x[perm[r] / S]: one warp per row, 16-byte vectors.
 __global__ void __launch_bounds__(256) gather_rows_kernel(int R, int S, int row_vecs,
                                                           const uint4* __restrict__ x,
@@ -231,6 +308,12 @@ size_t permute_scratch_ints(int R, int E) {
 cudaError_t launch_permute(int R, int E, const int32_t* ids, int32_t* counts, int32_t* offsets,
                            int32_t* perm, int32_t* inv, int32_t* tile_off, int32_t* scratch,
                            DevStatus* st, cudaStream_t stream) {
+    if (R <= kSmallR && E <= kSmallE) {
+        ProfileScope ps("permute_small", stream);
+        perm_small_kernel<<<1, 1024, 0, stream>>>(ids, R, E, counts, offsets, tile_off, perm, inv, st);
+        note_launch();
+        return cudaGetLastError();
+    }
     const int n_chunks = ceil_div(R, kPermChunk);
     const size_t hsm = static_cast<size_t>(E) * sizeof(int32_t);
     if (n_chunks > 0) {

@@ -27,18 +27,18 @@ namespace {
 #endif
 constexpr int RT_TPT = SRE_RT_TPT;
 constexpr int RT_BT = 16 * RT_TPT;     // tokens per block (16 token groups)
-constexpr int RT_EL = 16;      // expert lanes per block
-constexpr int RT_EJ = 10;      // experts per thread (strided by RT_EL)
-constexpr int RT_BE = RT_EL * RT_EJ;   // experts per block (160)
+constexpr int RT_EL = 16;      // expert lanes per block; a thread owns kEJ experts strided by RT_EL
 constexpr int RT_KC = 32;      // h per shared-memory chunk
 constexpr int RT_SEG = 256;    // segment length of the fixed order
 constexpr int RT_XP = RT_BT + 4;       // row pitch (floats) of the transposed x tile xs[k][t]
 constexpr int RT_WP = RT_KC + 4;       // row pitch (floats) of the w tile ws[e][k]: 144 B rows
 constexpr int RT_THREADS = 256;
 
+template <int kEJ>
 struct RouterSmem {
+    static constexpr int BE = RT_EL * kEJ;     // experts per block
     float xs[2][RT_KC][RT_XP];
-    float ws[2][RT_BE][RT_WP];
+    float ws[2][BE][RT_WP];
 };
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
@@ -49,12 +49,14 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
-// w chunk: rows e0.. (up to 160 experts) x 32 h, copied as is into ws[e][k]
+// w chunk: rows e0.. (kBE experts) x 32 h, copied as is into ws[e][k]
 // (16-byte pieces; rows past E are left unwritten: their results are never stored)
+template <int kBE>
 __device__ __forceinline__ void issue_w_chunk(const float* wr, int E, int H, int e0, int h0,
                                               float (*ws)[RT_WP]) {
+    static_assert((kBE * RT_KC / 4) % RT_THREADS == 0, "whole pieces per thread");
 #pragma unroll
-    for (int i = 0; i < (RT_BE * RT_KC / 4) / RT_THREADS; ++i) {
+    for (int i = 0; i < (kBE * RT_KC / 4) / RT_THREADS; ++i) {
         const int piece = threadIdx.x + i * RT_THREADS;
         const int e = piece >> 3, c = piece & 7;
         if (e0 + e < E) cp_async16(&ws[e][c * 4], wr + static_cast<size_t>(e0 + e) * H + h0 + c * 4);
@@ -128,25 +130,26 @@ __device__ __forceinline__ void store_x_chunk(const XStage<kBf16>& st, float (*x
 // experts e0 + tx + 16 j (j < 10). P[s][t][e] = fma chain over the 256 h of segment s
 // (blockIdx.z), from +0, h ascending. The next chunk's copies are in flight
 // while this one is multiplied.
-template <bool kBf16>
+template <bool kBf16, int kEJ>
 __global__ void __launch_bounds__(RT_THREADS, SRE_RT_MINB) router_segment_kernel(const void* __restrict__ x,
                                                                        const float* __restrict__ wr,
                                                                        float* __restrict__ P, int T, int H,
                                                                        int E) {
     extern __shared__ __align__(16) uint8_t rt_smem[];
-    RouterSmem& sm = *reinterpret_cast<RouterSmem*>(rt_smem);
-    const int t0 = blockIdx.x * RT_BT, e0 = blockIdx.y * RT_BE, s = blockIdx.z;
+    using Smem = RouterSmem<kEJ>;
+    Smem& sm = *reinterpret_cast<Smem*>(rt_smem);
+    const int t0 = blockIdx.x * RT_BT, e0 = blockIdx.y * Smem::BE, s = blockIdx.z;
     const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
 
-    float acc[RT_TPT][RT_EJ];
+    float acc[RT_TPT][kEJ];
 #pragma unroll
     for (int a = 0; a < RT_TPT; ++a)
 #pragma unroll
-        for (int j = 0; j < RT_EJ; ++j) acc[a][j] = 0.0f;
+        for (int j = 0; j < kEJ; ++j) acc[a][j] = 0.0f;
 
     constexpr int NCHUNK = RT_SEG / RT_KC;
     XStage<kBf16> xnext;
-    issue_w_chunk(wr, E, H, e0, s * RT_SEG, sm.ws[0]);
+    issue_w_chunk<Smem::BE>(wr, E, H, e0, s * RT_SEG, sm.ws[0]);
     load_x_chunk<kBf16>(x, T, H, t0, s * RT_SEG, xnext);
     store_x_chunk<kBf16>(xnext, sm.xs[0]);
     cp_async_wait_all();
@@ -158,7 +161,7 @@ __global__ void __launch_bounds__(RT_THREADS, SRE_RT_MINB) router_segment_kernel
         const bool more = c + 1 < NCHUNK;
         if (more) {
             const int h1 = s * RT_SEG + (c + 1) * RT_KC;
-            issue_w_chunk(wr, E, H, e0, h1, sm.ws[buf ^ 1]);
+            issue_w_chunk<Smem::BE>(wr, E, H, e0, h1, sm.ws[buf ^ 1]);
             load_x_chunk<kBf16>(x, T, H, t0, h1, xnext);
         }
         const float (*xs)[RT_XP] = sm.xs[buf];
@@ -175,7 +178,7 @@ __global__ void __launch_bounds__(RT_THREADS, SRE_RT_MINB) router_segment_kernel
                 }
             }
 #pragma unroll
-            for (int j = 0; j < RT_EJ; ++j) {
+            for (int j = 0; j < kEJ; ++j) {
                 const float4 w = *reinterpret_cast<const float4*>(&ws[tx + RT_EL * j][k4]);
 #pragma unroll
                 for (int a = 0; a < RT_TPT; ++a) {
@@ -200,7 +203,7 @@ __global__ void __launch_bounds__(RT_THREADS, SRE_RT_MINB) router_segment_kernel
         const int t = t0 + ty * RT_TPT + a;
         if (t >= T) continue;
 #pragma unroll
-        for (int j = 0; j < RT_EJ; ++j) {
+        for (int j = 0; j < kEJ; ++j) {
             const int e = e0 + tx + RT_EL * j;
             if (e < E) out[static_cast<size_t>(t) * E + e] = acc[a][j];
         }
@@ -309,6 +312,30 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ P, 
     }
 }
 
+template <int kEJ>
+cudaError_t launch_router_segments(const moe_shape& s, const void* x, const float* wr, float* partials, int T,
+                                   int H, int E, int split, cudaStream_t st) {
+    constexpr int smem = static_cast<int>(sizeof(RouterSmem<kEJ>));
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(router_segment_kernel<true, kEJ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        smem);
+        if (attr_err == cudaSuccess)
+            attr_err = cudaFuncSetAttribute(router_segment_kernel<false, kEJ>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    dim3 grid(ceil_div(T, RT_BT), ceil_div(E, RouterSmem<kEJ>::BE), split);
+    ProfileScope ps("route_logits", st);
+    if (s.act_dtype == MOE_BF16)
+        router_segment_kernel<true, kEJ><<<grid, RT_THREADS, smem, st>>>(x, wr, partials, T, H, E);
+    else
+        router_segment_kernel<false, kEJ><<<grid, RT_THREADS, smem, st>>>(x, wr, partials, T, H, E);
+    note_launch();
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 int router_split_count(int T, int H) {
@@ -325,25 +352,11 @@ cudaError_t launch_route(const moe_shape& s, const void* x, const float* wr, con
                          cudaStream_t st) {
     const int T = s.T, H = s.H, E = s.n_routed;
     const int split = router_split_count(T, H);
-    dim3 grid(ceil_div(T, RT_BT), ceil_div(E, RT_BE), split);
-    {
-        constexpr int smem = static_cast<int>(sizeof(RouterSmem));
-        static std::once_flag once;
-        static cudaError_t attr_err = cudaSuccess;
-        std::call_once(once, [] {
-            attr_err = cudaFuncSetAttribute(router_segment_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-            if (attr_err == cudaSuccess)
-                attr_err = cudaFuncSetAttribute(router_segment_kernel<false>,
-                                                cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        });
-        if (attr_err != cudaSuccess) return attr_err;
-        ProfileScope ps("route_logits", st);
-        if (s.act_dtype == MOE_BF16)
-            router_segment_kernel<true><<<grid, RT_THREADS, smem, st>>>(x, wr, partials, T, H, E);
-        else
-            router_segment_kernel<false><<<grid, RT_THREADS, smem, st>>>(x, wr, partials, T, H, E);
-        note_launch();
-    }
+    // small batches: 32 experts per block (5x the blocks at 160 routed experts)
+    const bool narrow = T <= 4 * RT_BT;
+    cudaError_t err = narrow ? launch_router_segments<2>(s, x, wr, partials, T, H, E, split, st)
+                             : launch_router_segments<10>(s, x, wr, partials, T, H, E, split, st);
+    if (err != cudaSuccess) return err;
     {
         ProfileScope ps("route_topk", st);
         topk_kernel<<<ceil_div(T * 32, 256), 256, 0, st>>>(partials, split, bias, T, E, s.top_k,

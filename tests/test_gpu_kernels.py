@@ -83,8 +83,11 @@ def _permute(cfg, ids_np):
     return [t.cpu().numpy() for t in (counts, offsets, perm, inv)], st
 
 
+# small batches (R <= 8192 slots, <= 256 experts) take the one-block path, the
+# rest the three-kernel path; the cases straddle both limits
 @pytest.mark.parametrize("T,E_r,K", [(1, 8, 2), (333, 40, 6), (4096, 160, 8), (16384, 160, 8),
-                                     (70, 4, 4)])
+                                     (70, 4, 4), (1024, 64, 7), (1171, 64, 6), (500, 255, 4),
+                                     (500, 256, 4)])
 def test_permute_bit_exact(T, E_r, K):
     cfg = synth.variant(synth.CONFIGS["prefill_bf16"], T=T, H=256, I=64, n_routed=E_r, top_k=K)
     rng = np.random.default_rng(T)
