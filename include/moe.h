@@ -64,6 +64,13 @@ typedef enum moe_dtype { MOE_F32 = 0, MOE_BF16 = 1, MOE_E4M3 = 2 } moe_dtype;
  *   act_dtype    dtype of x, out and of the expert rows y: MOE_F32 or MOE_BF16
  *   w_dtype      expert weight dtype: MOE_F32 (with act F32), MOE_BF16 or
  *                MOE_E4M3 (both with act BF16)
+ *   routed_scale routed scaling factor s (> 0, finite; 1.0 = none): the routed
+ *                slots' weights are s * softmax; the shared slot keeps
+ *                shared_weight (engines that scale the whole fused sum by s
+ *                give the shared slot 1/s instead: the same output)
+ *   bias_select_only  0: router_bias is added to the logits used for both
+ *                ranking and weights; 1: the bias only ranks (ids), the
+ *                weights use the logits without it
  * Derived: S = top_k + (shared_id >= 0) slots per token in the fused layout,
  * E = n_routed + (shared_id >= 0) experts, R = T*S expert rows. */
 typedef struct moe_shape {
@@ -71,6 +78,8 @@ typedef struct moe_shape {
     float shared_weight;
     int32_t renormalize;
     int32_t act_dtype, w_dtype;
+    float routed_scale;
+    int32_t bias_select_only;
 } moe_shape;
 
 /* Kernel choice for the expert GEMMs. AUTO picks the tcgen05 tensor-core

@@ -52,7 +52,7 @@ def lib():
         L.orc_router_logits_f64.restype = None
         L.orc_router_logits_f64.argtypes = [i, i, i, p, p, p, p]
         L.orc_topk.restype = None
-        L.orc_topk.argtypes = [i, i, i, p, i, i, f, p, p]
+        L.orc_topk.argtypes = [i, i, i, p, p, i, f, i, f, p, p]
         L.orc_permute.restype = i
         L.orc_permute.argtypes = [i, i, p, p, p, p, p]
         L.orc_expert_ffn.restype = None
@@ -142,13 +142,17 @@ def router_logits_f64(x, wr, bias=None) -> np.ndarray:
 
 
 def topk(L: np.ndarray, K: int, renormalize: bool = True, shared_id: int = -1,
-         shared_weight: float = 1.0):
+         shared_weight: float = 1.0, weight_logits: np.ndarray | None = None, routed_scale: float = 1.0):
+    """Top-K by the ranking keys L; weights from weight_logits (default: L),
+    routed slots scaled by routed_scale."""
     L = np.ascontiguousarray(L, dtype=np.float32)
     T, E = L.shape
+    Lw = None if weight_logits is None else np.ascontiguousarray(weight_logits, dtype=np.float32)
     S = K + (1 if shared_id >= 0 else 0)
     ids = np.empty((T, S), dtype=np.int32)
     w = np.empty((T, S), dtype=np.float64)
-    lib().orc_topk(T, E, K, _ptr(L), int(renormalize), shared_id, shared_weight, _ptr(ids), _ptr(w))
+    lib().orc_topk(T, E, K, _ptr(L), _ptr(Lw), int(renormalize), routed_scale, shared_id, shared_weight,
+                   _ptr(ids), _ptr(w))
     return ids, w
 
 
@@ -182,7 +186,7 @@ class _Layer(C.Structure):
     _fields_ = [("T", C.c_int), ("H", C.c_int), ("I", C.c_int), ("E_r", C.c_int),
                 ("K", C.c_int), ("shared_id", C.c_int), ("shared_weight", C.c_float),
                 ("renormalize", C.c_int), ("act_dtype", C.c_int), ("w_dtype", C.c_int),
-                ("x", C.c_void_p), ("router_w", C.c_void_p), ("router_bias", C.c_void_p),
+                ("routed_scale", C.c_float), ("bias_select_only", C.c_int), ("x", C.c_void_p), ("router_w", C.c_void_p), ("router_bias", C.c_void_p),
                 ("w13", C.c_void_p), ("s13", C.c_void_p), ("w2", C.c_void_p),
                 ("s2", C.c_void_p)]
 
@@ -196,7 +200,8 @@ class Layer:
         k = self._keep
         self.s = _Layer(cfg.T, cfg.H, cfg.I, cfg.n_routed, cfg.top_k, cfg.shared_id,
                         cfg.shared_weight, int(cfg.renormalize), _DT[cfg.act_dtype],
-                        _DT[cfg.w_dtype], _ptr(k["x"]), _ptr(k["router_w"]),
+                        _DT[cfg.w_dtype], float(getattr(cfg, "routed_scale", 1.0)),
+                        int(getattr(cfg, "bias_select_only", False)), _ptr(k["x"]), _ptr(k["router_w"]),
                         _ptr(k["router_bias"]), _ptr(k["w13"]), _ptr(k["s13"]),
                         _ptr(k["w2"]), _ptr(k["s2"]))
 

@@ -7,8 +7,8 @@
  *
  * What it computes (the plain definition; slow and obviously correct):
  *
- *   "Optimizing GLM4-MoE for production" (Novita AI; the zh rewrite, section 2.1
- *   "Shared Experts Fusion", the pseudocode block): the unfused layer is
+ *   "GLM4-MoE生产环境优化：SGLang降低65%首Token延迟" (intelliparadigm.com), section
+ *   2.1 "Shared Experts Fusion", the pseudocode block: the unfused layer is
  *       out = shared_expert(x) + sum(route(x, top_k = 8))
  *   Same page, numbered list under the pseudocode, and the de/en pages,
  *   section 1 "Shared Experts Fusion": the shared expert becomes routed expert
@@ -41,6 +41,12 @@
  *      has been rounded to bf16. Everything else is fp64.
  *   R8 E4M3 is the OCP "E4M3FN" format: bias 7, no infinities, 0x7F/0xFF NaN,
  *      largest finite 448, smallest subnormal 2^-9.
+ *   R15 routed scaling factor s (the de/en pages, section 1, mention that the
+ *      shared expert's weight needs special handling): the routed slots weigh
+ *      s * softmax and the shared slot keeps shared_weight, the same sum as an
+ *      engine that scales the whole fused sum by s with the shared slot at 1/s.
+ *   R16 bias for selection only: the bias enters the ranking key (R3, R4) but
+ *      the softmax uses the logits without it.
  */
 #include <math.h>
 #include <pthread.h>
@@ -170,15 +176,18 @@ void orc_router_logits_f64(int T, int H, int E_r, const float* x, const float* w
 
 static double rank_key(float v) { return isnan(v) ? -INFINITY : (double)v; }
 
-/* Top-K selection and weights for T tokens (R1-R3). Slots 0..K-1 hold the
- * routed experts in rank order; if shared_id >= 0, slot K holds
- * (shared_id, shared_weight). S = K + (shared_id >= 0). */
-void orc_topk(int T, int E_r, int K, const float* L, int renormalize, int shared_id,
-              float shared_weight, int32_t* ids, double* w) {
+/* Top-K selection and weights for T tokens (R1-R3, R15, R16). L holds the
+ * ranking keys; Lw the logits the weights use (NULL: the keys). Slots 0..K-1
+ * hold the routed experts in rank order with weight routed_scale * softmax; if
+ * shared_id >= 0, slot K holds (shared_id, shared_weight).
+ * S = K + (shared_id >= 0). */
+void orc_topk(int T, int E_r, int K, const float* L, const float* Lw, int renormalize, float routed_scale,
+              int shared_id, float shared_weight, int32_t* ids, double* w) {
     int S = K + (shared_id >= 0 ? 1 : 0);
     char* taken = (char*)malloc((size_t)E_r);
     for (int t = 0; t < T; ++t) {
         const float* l = L + (size_t)t * E_r;
+        const float* lw = (Lw ? Lw : L) + (size_t)t * E_r;
         int32_t* id = ids + (size_t)t * S;
         double* wt = w + (size_t)t * S;
         memset(taken, 0, (size_t)E_r);
@@ -191,16 +200,17 @@ void orc_topk(int T, int E_r, int K, const float* L, int renormalize, int shared
             taken[best] = 1;
             id[k] = best;
         }
-        double m, den = 0.0;
+        /* softmax over the selected (renormalize) or all weight logits, taken
+         * relative to their largest value */
+        double m = -INFINITY, den = 0.0;
         if (renormalize) {
-            m = rank_key(l[id[0]]);
-            for (int k = 0; k < K; ++k) den += exp(rank_key(l[id[k]]) - m);
+            for (int k = 0; k < K; ++k) if (rank_key(lw[id[k]]) > m) m = rank_key(lw[id[k]]);
+            for (int k = 0; k < K; ++k) den += exp(rank_key(lw[id[k]]) - m);
         } else {
-            m = -INFINITY;
-            for (int e = 0; e < E_r; ++e) if (rank_key(l[e]) > m) m = rank_key(l[e]);
-            for (int e = 0; e < E_r; ++e) den += exp(rank_key(l[e]) - m);
+            for (int e = 0; e < E_r; ++e) if (rank_key(lw[e]) > m) m = rank_key(lw[e]);
+            for (int e = 0; e < E_r; ++e) den += exp(rank_key(lw[e]) - m);
         }
-        for (int k = 0; k < K; ++k) wt[k] = exp(rank_key(l[id[k]]) - m) / den;
+        for (int k = 0; k < K; ++k) wt[k] = (double)routed_scale * (exp(rank_key(lw[id[k]]) - m) / den);
         if (shared_id >= 0) {
             id[K] = shared_id;
             wt[K] = (double)shared_weight;
@@ -216,6 +226,7 @@ void orc_topk(int T, int E_r, int K, const float* L, int renormalize, int shared
  * Returns -1 if an id is out of [0, E). */
 int orc_permute(int R, int E, const int32_t* ids, int32_t* counts, int32_t* offsets,
                 int32_t* perm, int32_t* inv) {
+    if (E <= 0 || R < 0) return -1;
     for (int e = 0; e < E; ++e) counts[e] = 0;
     for (int f = 0; f < R; ++f) {
         if (ids[f] < 0 || ids[f] >= E) return -1;
@@ -242,6 +253,8 @@ typedef struct {
     int renormalize;
     int act_dtype;          /* ORC_F32 | ORC_BF16 */
     int w_dtype;            /* ORC_F32 | ORC_BF16 | ORC_E4M3 */
+    float routed_scale;     /* R15 */
+    int bias_select_only;   /* R16 */
     const void* x;          /* [T, H] fp32 or bf16 bits */
     const float* router_w;  /* [E_r, H] */
     const float* router_bias;  /* [E_r] or NULL */
@@ -349,22 +362,26 @@ static void forward_token(const orc_layer* Ly, int t, int fuse_shared, double* o
                           double* out_rnd, int32_t* ids, double* w, void* scratch) {
     const int H = Ly->H, E_r = Ly->E_r, K = Ly->K;
     float* v = (float*)malloc((size_t)H * sizeof(float));
-    float* L = (float*)malloc((size_t)E_r * sizeof(float));
+    float* L = (float*)malloc((size_t)E_r * sizeof(float));      /* ranking keys */
+    float* Lw = (float*)malloc((size_t)E_r * sizeof(float));     /* logits without the bias */
     double* y = (double*)malloc((size_t)H * sizeof(double));
     for (int h = 0; h < H; ++h) v[h] = (float)xval(Ly, t, h);
-    orc_router_logits(1, H, E_r, v, Ly->router_w, Ly->router_bias, L);
+    orc_router_logits(1, H, E_r, v, Ly->router_w, NULL, Lw);
+    for (int e = 0; e < E_r; ++e) L[e] = Ly->router_bias ? Lw[e] + Ly->router_bias[e] : Lw[e];
+    const float* Lweights = Ly->bias_select_only ? Lw : NULL;
     for (int j = 0; j < H; ++j) out[j] = 0.0;
     if (fuse_shared) {
         /* Fused: one pass over the S = K + 1 slots, shared expert in slot K. */
         int S = K + (Ly->shared_id >= 0 ? 1 : 0);
-        orc_topk(1, E_r, K, L, Ly->renormalize, Ly->shared_id, Ly->shared_weight, ids, w);
+        orc_topk(1, E_r, K, L, Lweights, Ly->renormalize, Ly->routed_scale, Ly->shared_id, Ly->shared_weight,
+                 ids, w);
         for (int k = 0; k < S; ++k) {
             expert_ffn(Ly, ids[k], v, y, scratch);
             for (int j = 0; j < H; ++j) out[j] += w[k] * y[j];
         }
     } else {
         /* Unfused: routed top-K sum, then the shared expert added on its own. */
-        orc_topk(1, E_r, K, L, Ly->renormalize, -1, 0.0f, ids, w);
+        orc_topk(1, E_r, K, L, Lweights, Ly->renormalize, Ly->routed_scale, -1, 0.0f, ids, w);
         for (int k = 0; k < K; ++k) {
             expert_ffn(Ly, ids[k], v, y, scratch);
             for (int j = 0; j < H; ++j) out[j] += w[k] * y[j];
@@ -377,6 +394,7 @@ static void forward_token(const orc_layer* Ly, int t, int fuse_shared, double* o
     for (int j = 0; j < H; ++j) out_rnd[j] = round_out(Ly, out[j]);
     free(v);
     free(L);
+    free(Lw);
     free(y);
 }
 

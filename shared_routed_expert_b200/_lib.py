@@ -34,7 +34,8 @@ class MoeError(RuntimeError):
 class moe_shape(C.Structure):
     _fields_ = [("T", C.c_int32), ("H", C.c_int32), ("I", C.c_int32), ("n_routed", C.c_int32),
                 ("top_k", C.c_int32), ("shared_id", C.c_int32), ("shared_weight", C.c_float),
-                ("renormalize", C.c_int32), ("act_dtype", C.c_int32), ("w_dtype", C.c_int32)]
+                ("renormalize", C.c_int32), ("act_dtype", C.c_int32), ("w_dtype", C.c_int32),
+                ("routed_scale", C.c_float), ("bias_select_only", C.c_int32)]
 
 
 _lib = None
@@ -113,7 +114,8 @@ def make_shape(cfg, T: int | None = None) -> moe_shape:
     """moe_shape of a LayerConfig-like object (T overrides cfg.T)."""
     return moe_shape(cfg.T if T is None else T, cfg.H, cfg.I, cfg.n_routed, cfg.top_k,
                      cfg.shared_id, cfg.shared_weight, int(cfg.renormalize),
-                     DTYPES[cfg.act_dtype], DTYPES[cfg.w_dtype])
+                     DTYPES[cfg.act_dtype], DTYPES[cfg.w_dtype],
+                     float(getattr(cfg, "routed_scale", 1.0)), int(getattr(cfg, "bias_select_only", False)))
 
 
 def moe_workspace_size(shape: moe_shape, fuse_shared: bool = True) -> int:

@@ -143,6 +143,8 @@ moe_status check_shape(const moe_shape* s) {
     if (s->top_k > s->n_routed) return MOE_ERR_INVALID_ARG;
     if (s->shared_id != -1 && s->shared_id != s->n_routed) return MOE_ERR_INVALID_ARG;
     if (s->renormalize != 0 && s->renormalize != 1) return MOE_ERR_INVALID_ARG;
+    if (!(s->routed_scale > 0.0f) || !isfinite(s->routed_scale)) return MOE_ERR_INVALID_ARG;
+    if (s->bias_select_only != 0 && s->bias_select_only != 1) return MOE_ERR_INVALID_ARG;
     if (s->H % 256 != 0 || s->I % 64 != 0) return MOE_ERR_UNSUPPORTED;
     if (s->n_routed > 256 || s->top_k > 32) return MOE_ERR_UNSUPPORTED;
     const bool ok_dt = (s->act_dtype == MOE_F32 && s->w_dtype == MOE_F32) ||

@@ -217,10 +217,14 @@ __device__ __forceinline__ bool better(float v1, int i1, float v2, int i2) {
 constexpr int TK_MAXPL = 8;   // logits per lane: n_routed <= 256
 
 // One warp per token. P holds n_part ordered partials [n_part][T][E].
+// key = ranking score (logit + bias, fp32, bias added last); the weights use
+// the key, or the logit without the bias when bias_select_only; routed slots
+// weigh routed_scale * softmax.
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ P, int n_part,
                                                    const float* __restrict__ bias, int T, int E,
                                                    int K, int renormalize, int shared_id,
-                                                   float shared_weight, int32_t* __restrict__ ids,
+                                                   float shared_weight, float routed_scale,
+                                                   int bias_select_only, int32_t* __restrict__ ids,
                                                    float* __restrict__ wts,
                                                    float* __restrict__ logits_out) {
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -249,23 +253,26 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ P, 
 #pragma unroll
                 for (int j = 0; j < TK_MAXPL; ++j) tot[j] = __fadd_rn(tot[j], v[q][j]);
     }
-    float key[TK_MAXPL];
+    float key[TK_MAXPL], wlog[TK_MAXPL];
 #pragma unroll
     for (int j = 0; j < TK_MAXPL; ++j) {
         const int e = lane + 32 * j;
-        float v = -INFINITY;
+        float v = -INFINITY, u = -INFINITY;
         if (e < E) {
             float tj = tot[j];
+            const float raw = isnan(tj) ? -INFINITY : tj;
             if (bias != nullptr) tj = __fadd_rn(tj, bias[e]);
             if (logits_out != nullptr) logits_out[static_cast<size_t>(t) * E + e] = tj;
             v = isnan(tj) ? -INFINITY : tj;
+            u = (bias_select_only && bias != nullptr) ? raw : v;
         }
         key[j] = v;
+        wlog[j] = u;
     }
     unsigned taken = 0;    // bit j: element lane + 32j taken
-    float sel_v[32];
+    float sel_w[32];       // weight logits of the selected experts, in rank order
     int my_id = -1;
-    float my_v = 0.0f;
+    float my_w = 0.0f;
     for (int k = 0; k < K; ++k) {
         float bv = -INFINITY;
         int bi = 0x7FFFFFFF;
@@ -281,30 +288,34 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ P, 
             if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
         }
         if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-        sel_v[k] = bv;
-        if (lane == k) { my_id = bi; my_v = bv; }
-    }
-    float m, den = 0.0f;
-    if (renormalize) {
-        m = sel_v[0];
-        for (int k = 0; k < K; ++k) den += expf(sel_v[k] - m);
-    } else {
-        m = -INFINITY;
+        float wv = 0.0f;     // the owner lane's weight logit of expert bi
 #pragma unroll
-        for (int j = 0; j < TK_MAXPL; ++j) m = fmaxf(m, key[j]);
+        for (int j = 0; j < TK_MAXPL; ++j)
+            if (j == (bi >> 5)) wv = wlog[j];
+        wv = __shfl_sync(0xFFFFFFFFu, wv, bi & 31);
+        sel_w[k] = wv;
+        if (lane == k) { my_id = bi; my_w = wv; }
+    }
+    float m = -INFINITY, den = 0.0f;
+    if (renormalize) {
+        for (int k = 0; k < K; ++k) m = fmaxf(m, sel_w[k]);
+        for (int k = 0; k < K; ++k) den += expf(sel_w[k] - m);
+    } else {
+#pragma unroll
+        for (int j = 0; j < TK_MAXPL; ++j) m = fmaxf(m, wlog[j]);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
         float part = 0.0f;
 #pragma unroll
         for (int j = 0; j < TK_MAXPL; ++j)
-            if (lane + 32 * j < E) part += expf(key[j] - m);
+            if (lane + 32 * j < E) part += expf(wlog[j] - m);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xFFFFFFFFu, part, off);
         den = part;
     }
     if (lane < K) {
         ids[static_cast<size_t>(t) * S + lane] = my_id;
-        wts[static_cast<size_t>(t) * S + lane] = expf(my_v - m) / den;
+        wts[static_cast<size_t>(t) * S + lane] = routed_scale * (expf(my_w - m) / den);
     }
     if (shared_id >= 0 && lane == 0) {
         ids[static_cast<size_t>(t) * S + K] = shared_id;
@@ -360,8 +371,9 @@ cudaError_t launch_route(const moe_shape& s, const void* x, const float* wr, con
     {
         ProfileScope ps("route_topk", st);
         topk_kernel<<<ceil_div(T * 32, 256), 256, 0, st>>>(partials, split, bias, T, E, s.top_k,
-                                                          s.renormalize, shared_id,
-                                                          s.shared_weight, ids, wts, logits);
+                                                          s.renormalize, shared_id, s.shared_weight,
+                                                          s.routed_scale, s.bias_select_only, ids, wts,
+                                                          logits);
         note_launch();
     }
     return cudaGetLastError();

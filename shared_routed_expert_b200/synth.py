@@ -50,6 +50,8 @@ class LayerConfig:
     shared: bool = True
     shared_weight: float = 1.0
     renormalize: bool = True
+    routed_scale: float = 1.0        # routed slots weigh routed_scale * softmax
+    bias_select_only: bool = False   # router bias ranks the experts but does not weigh them
 
     @property
     def n_experts(self) -> int:

@@ -29,6 +29,11 @@ ROUTE_CASES = {
                                top_k=5, renormalize=False),
     "no_shared": synth.variant(synth.CONFIGS["prefill_bf16"], T=64, H=256, I=64, n_routed=256,
                                top_k=32, shared=False),
+    "routed_scale": synth.variant(synth.CONFIGS["prefill_bf16"], T=300, H=512, I=64, n_routed=40,
+                                  top_k=6, routed_scale=2.5),
+    "bias_select_only": synth.variant(synth.CONFIGS["skewed_fp8"], T=257, I=64, bias_select_only=True),
+    "bias_select_full_softmax": synth.variant(synth.CONFIGS["skewed_fp8"], T=100, I=64, bias_select_only=True,
+                                              renormalize=False, routed_scale=0.5),
 }
 
 
@@ -55,7 +60,9 @@ def test_route_topk_bit_exact(name):
     ids, w, L = _route(cfg, inp)
     Lr = oracle_logits(inp["x"], inp["router_w"], inp["router_bias"])
     assert np.array_equal(L.view(np.uint32), Lr.view(np.uint32)), "logits differ in some bit"
-    rid, rw = oracle.topk(Lr, cfg.top_k, cfg.renormalize, cfg.shared_id, cfg.shared_weight)
+    Lw = oracle_logits(inp["x"], inp["router_w"], None) if cfg.bias_select_only else None
+    rid, rw = oracle.topk(Lr, cfg.top_k, cfg.renormalize, cfg.shared_id, cfg.shared_weight,
+                          weight_logits=Lw, routed_scale=cfg.routed_scale)
     assert np.array_equal(ids, rid)
     assert np.allclose(w, rw, rtol=2e-6, atol=1e-7)
 

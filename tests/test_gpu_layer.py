@@ -27,6 +27,10 @@ SMALL = {
                                    top_k=2, shared_weight=0.5),
     "no_renorm": synth.variant(synth.CONFIGS["prefill_bf16"], T=50, H=256, I=64, n_routed=8,
                                top_k=2, renormalize=False),
+    "routed_scale": synth.variant(synth.CONFIGS["prefill_bf16"], T=150, H=512, I=128, n_routed=16,
+                                  top_k=4, routed_scale=2.5),
+    "bias_select_only_fp8": synth.variant(synth.CONFIGS["skewed_fp8"], T=200, H=512, I=192, n_routed=24,
+                                          top_k=4, bias_select_only=True, routed_scale=1.5),
 }
 
 

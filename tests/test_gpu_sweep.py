@@ -1,10 +1,10 @@
 """A seeded random sweep of layer shapes through moe_forward against the CPU
 oracle: token counts with ragged tails, hidden and intermediate sizes the
 tensor-core tiles divide differently, expert counts from 1 to 48, top-k from 1
-to 8, bf16 and E4M3 weights, fused and unfused, and every GEMM variant (the
-CUDA-core one, single-CTA 128- and 256-row units, CTA pairs with 256 x 256 and
-256 x 512 tiles). Each case compares every output and the routing of every
-token."""
+to 8, bf16 and E4M3 weights, routed scaling factors and selection-only bias,
+fused and unfused, and every GEMM variant (the CUDA-core one, single-CTA 128-
+and 256-row units, CTA pairs with 256 x 256 and 256 x 512 tiles). Each case
+compares every output and the routing of every token."""
 import numpy as np
 import pytest
 import torch
@@ -31,6 +31,8 @@ def _case(seed: int):
                         seed=seed, renormalize=bool(rng.integers(0, 4) > 0),
                         shared_weight=float(rng.choice([1.0, 1.0, 0.5])),
                         zipf_s=(1.1 if rng.integers(0, 3) == 0 else None))
+    cfg = synth.variant(cfg, routed_scale=float(rng.choice([1.0, 1.0, 2.5])),
+                        bias_select_only=bool(cfg.zipf_s is not None and rng.integers(0, 2)))
     impl = IMPLS[int(rng.integers(0, len(IMPLS)))]
     fuse = bool(rng.integers(0, 4) > 0)
     return cfg, impl, fuse

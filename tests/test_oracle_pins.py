@@ -353,6 +353,65 @@ def test_identical_experts_give_twice_one_expert():
         assert np.allclose(res["out"][t], 2.0 * y, rtol=1e-12, atol=1e-15)
 
 
+@pytest.mark.parametrize("s", [2.5, 0.25])
+def test_identical_experts_with_routed_scale(s):
+    """Identical experts and a routed scaling factor s: the routed weights sum
+    to s and the shared slot keeps weight 1, so out = (s + 1) * FFN(x)."""
+    cfg = synth.variant(synth.CONFIGS["tiny_fp32"], routed_scale=s)
+    inp = synth.make_inputs(cfg)
+    inp["w13"][:] = inp["w13"][0].clone()
+    inp["w2"][:] = inp["w2"][0].clone()
+    Ly = oracle.Layer(cfg, inp)
+    res = Ly.forward(n_threads=2)
+    for t in range(cfg.T):
+        y = Ly.expert_ffn(0, inp["x"][t].numpy())
+        assert np.allclose(res["out"][t], (s + 1.0) * y, rtol=1e-12, atol=1e-15)
+
+
+def test_routed_scale_equals_scaling_the_fused_sum_with_shared_weight_one_over_s():
+    """An engine that scales the whole fused sum by s must give the shared slot
+    1/s; scaling the routed slots by s instead yields the same output (s = 4:
+    1/s is exact in fp32, so the two differ only by fp64 rounding)."""
+    s = 4.0
+    base = synth.variant(synth.CONFIGS["prefill_bf16"], T=12, H=256, I=64, n_routed=8, top_k=3)
+    inp = synth.make_inputs(base)
+    a = oracle.Layer(synth.variant(base, routed_scale=s), inp).forward(n_threads=2)
+    b = oracle.Layer(synth.variant(base, shared_weight=1.0 / s), inp).forward(n_threads=2)
+    assert np.array_equal(a["ids"], b["ids"])
+    assert np.allclose(a["out"], s * b["out"], rtol=1e-12, atol=1e-12)
+
+
+def test_bias_for_selection_only_weighs_with_the_unbiased_logits():
+    """A bias that forces experts 3 and 5 into a top-2: they are selected in
+    either mode, but with bias_select_only the weights are the softmax of their
+    unbiased logits (numpy, fp64), otherwise of the biased ones."""
+    base = synth.variant(synth.CONFIGS["prefill_bf16"], T=10, H=256, I=64, n_routed=8, top_k=2)
+    inp = synth.make_inputs(base)
+    bias = torch.zeros(8)
+    bias[3], bias[5] = 40.0, 39.0
+    inp["router_bias"] = bias
+    x = inp["x"].float().numpy()
+    raw = oracle.router_logits_f64(x, inp["router_w"].numpy())[:, [3, 5]]
+    for sel_only in (True, False):
+        cfg = synth.variant(base, bias_select_only=sel_only)
+        r = oracle.Layer(cfg, inp).forward(n_threads=2)
+        assert np.array_equal(r["ids"][:, :2], np.tile([3, 5], (10, 1)))
+        z = raw if sel_only else raw + np.array([40.0, 39.0])
+        ref = np.exp(z - z.max(1, keepdims=True))
+        ref /= ref.sum(1, keepdims=True)
+        assert np.allclose(r["w"][:, :2], ref, rtol=0, atol=1e-6)
+        assert np.all(r["w"][:, 2] == 1.0)
+
+
+def test_bias_for_selection_only_without_bias_changes_nothing():
+    base = synth.variant(synth.CONFIGS["skewed_fp8"], T=16, H=256, I=64, n_routed=12, top_k=3)
+    inp = synth.make_inputs(base)
+    inp["router_bias"] = torch.zeros(12)
+    a = oracle.Layer(base, inp).forward(n_threads=2)
+    b = oracle.Layer(synth.variant(base, bias_select_only=True), inp).forward(n_threads=2)
+    assert np.array_equal(a["ids"], b["ids"]) and np.array_equal(a["out"], b["out"])
+
+
 def test_single_routed_expert_is_two_dense_mlps():
     cfg = synth.variant(synth.CONFIGS["tiny_fp32"], n_routed=1, top_k=1)
     inp = synth.make_inputs(cfg)
