@@ -59,6 +59,8 @@ def lib():
         L.orc_expert_ffn.argtypes = [p, i, p, p]
         L.orc_forward.restype = i
         L.orc_forward.argtypes = [p, i, p, i, p, p, p, p, i]
+        L.orc_qk_norm_rope.restype = None
+        L.orc_qk_norm_rope.argtypes = [i, i, i, i, i, f, p, p, p, p, p, p]
         L.orc_combine.restype = None
         L.orc_combine.argtypes = [i, i, i, p, p, p, i, p]
         _lib = L
@@ -177,6 +179,27 @@ def combine(Y: np.ndarray, inv: np.ndarray, w: np.ndarray, act_dtype: str) -> np
     inv = np.ascontiguousarray(inv, dtype=np.int32)
     out = np.empty((T, H), dtype=np.float64)
     lib().orc_combine(T, S, H, _ptr(Y), _ptr(inv), _ptr(w), _DT[act_dtype], _ptr(out))
+    return out
+
+
+# ------------------------------------------------------------------ QK-norm + partial RoPE
+
+def qk_norm_rope(qkv_bits: np.ndarray, pos: np.ndarray, qw_bits: np.ndarray, kw_bits: np.ndarray,
+                 cos_sin: np.ndarray, n_q: int, n_kv: int, d: int, rot: int, eps: float) -> np.ndarray:
+    """qkv_bits [T, (n_q + 2 n_kv) d] bf16 bits, pos [T], norm weights [d] bf16
+    bits, cos_sin [max_pos, rot] fp32 -> normalised and rotated q and k heads,
+    [T, n_q + n_kv, d] fp64 (unrounded)."""
+    qkv_bits = np.ascontiguousarray(qkv_bits, dtype=np.uint16)
+    T = qkv_bits.shape[0]
+    assert qkv_bits.shape[1] == (n_q + 2 * n_kv) * d and rot % 2 == 0 and rot <= d
+    pos = np.ascontiguousarray(pos, dtype=np.int32)
+    assert pos.shape == (T,) and (T == 0 or (pos.min() >= 0 and pos.max() < cos_sin.shape[0]))
+    cos_sin = np.ascontiguousarray(cos_sin, dtype=np.float32)
+    qw_bits = np.ascontiguousarray(qw_bits, dtype=np.uint16)
+    kw_bits = np.ascontiguousarray(kw_bits, dtype=np.uint16)
+    out = np.empty((T, n_q + n_kv, d), dtype=np.float64)
+    lib().orc_qk_norm_rope(T, n_q, n_kv, d, rot, eps, _ptr(qkv_bits), _ptr(pos), _ptr(qw_bits),
+                           _ptr(kw_bits), _ptr(cos_sin), _ptr(out))
     return out
 
 

@@ -219,6 +219,51 @@ void orc_topk(int T, int E_r, int K, const float* L, const float* Lw, int renorm
     free(taken);
 }
 
+/* ---------------------------------------------------------------- QK-norm + partial RoPE */
+
+/* "GLM4-MoE生产环境优化：SGLang降低65%首Token延迟", section 2.2 QK-Norm-RoPE
+ * fusion, and the de/en pages, section 2 "Qknorm Fusion": the attention's q
+ * and k heads are normalised head by head and rotated, and in GLM4-MoE only
+ * half of each head's dimensions rotate. Readings (the pages give no formula):
+ *   R17 the norm is RMSNorm over head_dim with a per-dimension weight (one for
+ *       q heads, one for k heads): u = v / sqrt(mean(v^2) + eps) * w;
+ *   R18 RoPE on the first rot dimensions, pairs (i, i + rot/2) for i < rot/2:
+ *       (a, b) -> (a cos - b sin, b cos + a sin) with cos/sin of the token's
+ *       position from the caller's table [max_pos][rot] (cos in [0, rot/2),
+ *       sin in [rot/2, rot)); dimensions >= rot pass through;
+ *   R19 the fused qkv row of a token is [q heads | k heads | v heads]; v is
+ *       left alone. Everything here is fp64 (the output is not rounded).
+ * out: [T][n_q + n_kv][d]. */
+void orc_qk_norm_rope(int T, int n_q, int n_kv, int d, int rot, float eps, const uint16_t* qkv,
+                      const int32_t* pos, const uint16_t* qw, const uint16_t* kw, const float* cos_sin,
+                      double* out) {
+    const int row = (n_q + 2 * n_kv) * d;
+    const int half = rot / 2;
+    double* u = (double*)malloc((size_t)d * sizeof(double));
+    for (int t = 0; t < T; ++t) {
+        const float* cs = cos_sin + (size_t)pos[t] * rot;
+        for (int h = 0; h < n_q + n_kv; ++h) {
+            const uint16_t* v = qkv + (size_t)t * row + (size_t)h * d;
+            const uint16_t* w = h < n_q ? qw : kw;
+            double ss = 0.0;
+            for (int i = 0; i < d; ++i) {
+                const double a = orc_bf16_to_double(v[i]);
+                ss += a * a;
+            }
+            const double r = 1.0 / sqrt(ss / d + (double)eps);
+            for (int i = 0; i < d; ++i) u[i] = orc_bf16_to_double(v[i]) * r * orc_bf16_to_double(w[i]);
+            double* o = out + ((size_t)t * (n_q + n_kv) + h) * d;
+            for (int i = 0; i < d; ++i) o[i] = u[i];
+            for (int i = 0; i < half; ++i) {
+                const double c = cs[i], s = cs[half + i];
+                o[i] = u[i] * c - u[i + half] * s;
+                o[i + half] = u[i + half] * c + u[i] * s;
+            }
+        }
+    }
+    free(u);
+}
+
 /* ---------------------------------------------------------------- permute */
 
 /* Counting sort of the R = T*S slots by expert, stable by flat index (R5).

@@ -177,3 +177,66 @@ def to_host(inputs: dict) -> dict:
 
 def to_device(inputs: dict, device) -> dict:
     return {k: (v.to(device) if isinstance(v, torch.Tensor) else v) for k, v in inputs.items()}
+
+
+# ------------------------------------------------------------------ attention pre-processing
+# Inputs of the fused QK-norm + partial RoPE step (the attention's q and k heads
+# normalised per head, then the first rot dimensions of each head rotated).
+
+@dataclass(frozen=True)
+class AttnConfig:
+    name: str
+    T: int              # tokens
+    n_q: int            # query heads
+    n_kv: int           # key / value heads
+    d: int              # head dimension
+    rot: int            # rotated dimensions per head (half of d in GLM4-MoE)
+    max_pos: int        # rows of the cos/sin table
+    seed: int
+    theta: float = 1.0e6
+    eps: float = 1.0e-5
+    sequential: bool = True   # positions 0..T-1 (prefill); else random (decode)
+
+    @property
+    def row(self) -> int:
+        return (self.n_q + 2 * self.n_kv) * self.d
+
+    def moved_bytes(self) -> int:
+        """q and k heads read and written once, bf16, plus positions."""
+        return 2 * self.T * (self.n_q + self.n_kv) * self.d * 2 + self.T * 4
+
+
+ATTN_CONFIGS = {
+    "qknorm_tiny": AttnConfig("qknorm_tiny", T=5, n_q=4, n_kv=2, d=64, rot=32, max_pos=64, seed=10),
+    # GLM4-MoE attention heads: 96 query and 8 key/value heads of 128, half rotated
+    "qknorm_prefill": AttnConfig("qknorm_prefill", T=4096, n_q=96, n_kv=8, d=128, rot=64, max_pos=4096,
+                                 seed=11),
+    "qknorm_decode": AttnConfig("qknorm_decode", T=64, n_q=96, n_kv=8, d=128, rot=64, max_pos=32768,
+                                seed=12, sequential=False),
+}
+
+
+def make_attn_inputs(cfg: AttnConfig, device: str | torch.device = "cpu") -> dict:
+    """qkv [T, (n_q + 2 n_kv) d] bf16 with per-head scales spread over 10^-1..10^1,
+    positions [T] int32, q/k norm weights [d] bf16 around 1, and the cos/sin
+    table [max_pos, rot] fp32 (angle pos * theta^(-2j/rot), cos then sin)."""
+    device = torch.device(device)
+    g = torch.Generator(device="cpu")
+    g.manual_seed(cfg.seed)
+    heads = cfg.n_q + 2 * cfg.n_kv
+    qkv = torch.empty(cfg.T, heads, cfg.d).normal_(0.0, 1.0, generator=g)
+    scale = torch.pow(10.0, torch.empty(cfg.T, heads, 1).uniform_(-1.0, 1.0, generator=g))
+    qkv = (qkv * scale).reshape(cfg.T, cfg.row).to(torch.bfloat16)
+    if cfg.sequential:
+        pos = torch.arange(cfg.T, dtype=torch.int32) % cfg.max_pos
+    else:
+        pos = torch.randint(0, cfg.max_pos, (cfg.T,), generator=g, dtype=torch.int64).to(torch.int32)
+    qw = (1.0 + 0.1 * torch.empty(cfg.d).normal_(0.0, 1.0, generator=g)).to(torch.bfloat16)
+    kw = (1.0 + 0.1 * torch.empty(cfg.d).normal_(0.0, 1.0, generator=g)).to(torch.bfloat16)
+    half = cfg.rot // 2
+    inv = torch.pow(torch.tensor(cfg.theta, dtype=torch.float64),
+                    -2.0 * torch.arange(half, dtype=torch.float64) / cfg.rot)
+    ang = torch.arange(cfg.max_pos, dtype=torch.float64)[:, None] * inv[None, :]
+    cos_sin = torch.cat([torch.cos(ang), torch.sin(ang)], 1).float()
+    out = {"qkv": qkv, "pos": pos, "q_w": qw, "k_w": kw, "cos_sin": cos_sin.contiguous()}
+    return {k: v.to(device) for k, v in out.items()}

@@ -462,3 +462,71 @@ def test_weights_sum_to_one_and_ids_distinct_on_a_glm_shape():
     # the Zipf prior pulls routing toward low expert ids
     counts = np.bincount(ids[:, :cfg.top_k].ravel(), minlength=cfg.n_routed)
     assert counts[:16].sum() > counts[-16:].sum()
+
+
+# ------------------------------------------------------------------ QK-norm + partial RoPE
+
+def _attn(cfg):
+    inp = synth.make_attn_inputs(cfg)
+    bits = lambda t: t.view(torch.int16).numpy().view(np.uint16)     # noqa: E731
+    out = oracle.qk_norm_rope(bits(inp["qkv"]), inp["pos"].numpy(), bits(inp["q_w"]), bits(inp["k_w"]),
+                              inp["cos_sin"].numpy(), cfg.n_q, cfg.n_kv, cfg.d, cfg.rot, cfg.eps)
+    return inp, out
+
+
+def test_qk_norm_matches_torch_rms_norm_and_rope_matches_complex_rotation():
+    """Norm: torch's rms_norm (fp64, eps as the fp32 value the call takes).
+    Rotation: the pair (u_i, u_{i+rot/2}) as the complex number u_i + i u_{i+rot/2}
+    times exp(i angle), angle read back from the table with atan2; dimensions
+    past rot unchanged."""
+    cfg = synth.ATTN_CONFIGS["qknorm_tiny"]
+    inp, out = _attn(cfg)
+    half = cfg.rot // 2
+    heads = inp["qkv"].double().reshape(cfg.T, cfg.n_q + 2 * cfg.n_kv, cfg.d)
+    for t in range(cfg.T):
+        cs = inp["cos_sin"][inp["pos"][t]].double().numpy()
+        ang = np.arctan2(cs[half:], cs[:half])
+        rad = np.hypot(cs[half:], cs[:half])          # 1 up to fp32 rounding of the table
+        for h in range(cfg.n_q + cfg.n_kv):
+            w = (inp["q_w"] if h < cfg.n_q else inp["k_w"]).double()
+            u = torch.nn.functional.rms_norm(heads[t, h], (cfg.d,), w, float(np.float32(cfg.eps))).numpy()
+            z = (u[:half] + 1j * u[half:cfg.rot]) * rad * np.exp(1j * ang)
+            ref = np.concatenate([z.real, z.imag, u[cfg.rot:]])
+            assert np.allclose(out[t, h], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_rope_dot_products_depend_only_on_the_position_difference():
+    """The defining property of rotary embeddings: over the rotated dimensions
+    <q at m, k at n> = <q at m + s, k at n + s> (unit norm weights, fp32 table)."""
+    base = synth.ATTN_CONFIGS["qknorm_tiny"]
+    cfg = synth.replace(base, T=2, max_pos=64)
+    inp = synth.make_attn_inputs(cfg)
+    inp["q_w"][:] = 1.0
+    inp["k_w"][:] = 1.0
+    qkv = inp["qkv"].clone()
+    qkv[1] = qkv[0]                     # the same token content at two positions
+    bits = lambda t: t.view(torch.int16).numpy().view(np.uint16)     # noqa: E731
+    dots = []
+    for m, n in [(3, 10), (20, 27), (50, 57)]:
+        pos = np.array([m, n], np.int32)
+        o = oracle.qk_norm_rope(bits(qkv), pos, bits(inp["q_w"]), bits(inp["k_w"]),
+                                inp["cos_sin"].numpy(), cfg.n_q, cfg.n_kv, cfg.d, cfg.rot, cfg.eps)
+        q, k = o[0, 0, :cfg.rot], o[1, cfg.n_q, :cfg.rot]
+        dots.append(float(q @ k))
+    assert np.allclose(dots, dots[0], rtol=1e-5, atol=1e-6)
+
+
+def test_qk_norm_is_scale_invariant_and_position_zero_is_the_identity_rotation():
+    cfg = synth.ATTN_CONFIGS["qknorm_tiny"]
+    inp = synth.make_attn_inputs(cfg)
+    bits = lambda t: t.view(torch.int16).numpy().view(np.uint16)     # noqa: E731
+    args = (bits(inp["q_w"]), bits(inp["k_w"]), inp["cos_sin"].numpy(), cfg.n_q, cfg.n_kv, cfg.d, cfg.rot, 0.0)
+    pos0 = np.zeros(cfg.T, np.int32)
+    a = oracle.qk_norm_rope(bits(inp["qkv"]), pos0, *args)
+    b = oracle.qk_norm_rope(bits((inp["qkv"].float() * 4.0).to(torch.bfloat16)), pos0, *args)
+    assert np.allclose(a, b, rtol=1e-13, atol=1e-13)       # x4 is exact in bf16; eps = 0
+    # position 0: cos 1, sin 0, so every output is the normalised value
+    heads = inp["qkv"].double().reshape(cfg.T, -1, cfg.d)[:, :cfg.n_q + cfg.n_kv]
+    rms = torch.sqrt((heads ** 2).mean(-1, keepdim=True))
+    w = torch.cat([inp["q_w"].double().expand(cfg.n_q, -1), inp["k_w"].double().expand(cfg.n_kv, -1)])
+    assert np.allclose(a, (heads / rms * w).numpy(), rtol=1e-12, atol=1e-12)
