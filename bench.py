@@ -367,6 +367,73 @@ def describe(cfg) -> str:
 
 # ------------------------------------------------------------------ main
 
+def bench_qk_norm_rope(args, dist):
+    """The fused QK-norm + partial RoPE kernel on its own: tokens/s from the
+    kernel's CUDA events (L2 flushed between launches by an untimed 256 MB
+    read, which leaves no dirty lines to write back during the kernel), rated
+    against the measured HBM copy peak; e2e uploads qkv and downloads it every
+    step."""
+    cfg = synth.ATTN_CONFIGS[args.attn_workload]
+    inp = synth.make_attn_inputs(cfg, dist.device)
+    stream = torch.cuda.current_stream()
+    flush = torch.ones(64 << 20, dtype=torch.float32, device=dist.device)
+
+    def launch(qkv):
+        _lib.moe_qk_norm_rope(cfg, qkv, inp["pos"], inp["q_w"], inp["k_w"], inp["cos_sin"])
+
+    def step():
+        flush.amax()
+        launch(inp["qkv"])
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    clocks = Clocks(vis.split(",")[dist.local] if vis else str(dist.local))
+    n0 = _lib.moe_launch_count()
+    _lib.moe_profile_reset()
+    _lib.moe_profile_enable(True)
+    clocks.start()
+    time_steps(step, args.steps, 0, dist, stream)
+    clk = clocks.stop()
+    _lib.moe_profile_enable(False)
+    launches = _lib.moe_launch_count() - n0
+    n, tot = _lib.moe_profile_read("qk_norm_rope")
+    ms_launch = dist.max(tot / max(n, 1))
+    # end to end: pinned host qkv up, kernel, qkv down, every step
+    host_in = inp["qkv"].cpu().pin_memory()
+    host_out = torch.empty_like(host_in).pin_memory()
+    dev = torch.empty_like(inp["qkv"])
+
+    def e2e_step():
+        dev.copy_(host_in, non_blocking=True)
+        launch(dev)
+        host_out.copy_(dev, non_blocking=True)
+    ms_e2e = time_steps(e2e_step, args.steps, args.warmup, dist, stream)
+    pk = peaks()
+    nbytes = cfg.moved_bytes()
+    ach = nbytes / (ms_launch / 1e3) / 1e9
+    N = dist.world
+    line = {
+        "metric": "fused QK-norm + partial RoPE tokens/s vs B200 HBM roofline", "op": "qk_norm_rope",
+        "value": N * cfg.T / (ms_launch / 1e3), "unit": "tokens/s", "n_gpus": N, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_launch, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{cfg.name}: T={cfg.T} q heads {cfg.n_q}, kv heads {cfg.n_kv}, head_dim {cfg.d}, "
+                               f"rotated {cfg.rot}, positions {'0..T-1' if cfg.sequential else 'random'}",
+                   "l2": "flushed between launches (256 MB read, not timed)"},
+        "e2e": {"value": N * cfg.T * args.steps / (ms_e2e / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": host_in.numel() * 2, "d2h_bytes_per_step": host_out.numel() * 2},
+        "gpu_launches": int(launches),
+        "roofline": {"kernel": "qk_norm_rope", "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"],
+                     "unit": "GB/s", "frac": ach / pk["hbm_gbs"], "traffic": None, "peak_source": pk["source"],
+                     "algorithmic_bytes": nbytes},
+        "clocks": clk,
+    }
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -384,6 +451,9 @@ def main():
     ap.add_argument("--tokens", type=int, default=None, help="override T (smaller profiling case)")
     ap.add_argument("--routed", type=int, default=None, help="override the routed expert count")
     ap.add_argument("--inter", type=int, default=None, help="override I (smaller profiling case)")
+    ap.add_argument("--op", default="moe", choices=["moe", "qk_norm_rope"],
+                    help="moe: the expert layer (default); qk_norm_rope: the attention pre-processing kernel")
+    ap.add_argument("--attn-workload", default="qknorm_prefill", choices=list(synth.ATTN_CONFIGS))
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -395,6 +465,10 @@ def main():
         return
 
     build.build()
+    if args.op == "qk_norm_rope":
+        bench_qk_norm_rope(args, dist)
+        dist.close()
+        return
     cfg = synth.CONFIGS[args.workload]
     if args.tokens is not None or args.routed is not None or args.inter is not None:
         cfg = synth.variant(cfg, T=args.tokens or cfg.T, n_routed=args.routed or cfg.n_routed,

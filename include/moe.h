@@ -234,6 +234,34 @@ moe_status moe_permute_noalloc(const moe_shape* shape, const int32_t* ids, int32
  * word (the outputs of those calls are garbage). No GPU fault is involved. */
 void moe_inject_wait_timeout(int n_calls);
 
+/* Fused QK-norm + partial RoPE on the attention's q and k heads, in place.
+ * "GLM4-MoE生产环境优化：SGLang降低65%首Token延迟", section 2.2 QK-Norm-RoPE
+ * fusion, and the de/en pages, section 2 "Qknorm Fusion": both steps are
+ * head-wise and run as one kernel; in GLM4-MoE only half of each head's
+ * dimensions rotate. For token t and each q and k head:
+ *   u = v / sqrt(mean(v^2) + eps) * w     (RMSNorm over head_dim; w = q_norm_w
+ *                                          for q heads, k_norm_w for k heads)
+ *   (u_i, u_{i+rot_dim/2}) -> (u_i c_i - u_{i+rot_dim/2} s_i,
+ *                              u_{i+rot_dim/2} c_i + u_i s_i),  i < rot_dim/2
+ * with c_i = cos_sin[positions[t]][i], s_i = cos_sin[positions[t]][rot_dim/2 + i];
+ * dimensions from rot_dim on pass through. fp32 arithmetic, one rounding.
+ *   qkv        [T][(n_q + 2*n_kv) * head_dim] bf16, caller-owned; each row is
+ *              q heads | k heads | v heads; q and k are overwritten, v is not
+ *              touched
+ *   positions  [T] int32, each in [0, max_pos)
+ *   q_norm_w, k_norm_w  [head_dim] bf16
+ *   cos_sin    [max_pos][rot_dim] fp32 (may be NULL when rot_dim == 0)
+ *   eps        >= 0
+ *   bad_positions  device int32 counter or NULL: a token whose position is out
+ *              of range leaves its heads unchanged and adds one per head
+ * head_dim 64, 128 or 256; rot_dim even, <= head_dim, rot_dim/2 a multiple of
+ * head_dim/32 (GLM4-MoE: 128 and 64). Asynchronous on `stream`. Returns
+ * MOE_ERR_INVALID_ARG for null or misaligned pointers (16 bytes) or bad sizes,
+ * MOE_ERR_UNSUPPORTED for other head shapes, MOE_ERR_CUDA on launch failure. */
+moe_status moe_qk_norm_rope(int32_t T, int32_t n_q, int32_t n_kv, int32_t head_dim, int32_t rot_dim, float eps,
+                            void* qkv, const int32_t* positions, int32_t max_pos, const void* q_norm_w,
+                            const void* k_norm_w, const float* cos_sin, int32_t* bad_positions, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

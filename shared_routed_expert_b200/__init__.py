@@ -17,12 +17,12 @@ import torch
 from ._lib import (MOE_BF16, MOE_E4M3, MOE_F32, MOE_FFN_AUTO, MOE_FFN_SIMT, MOE_FFN_TCGEN05,
                    MoeError, alloc_workspace, make_shape, moe_clear_status, moe_combine,
                    moe_forward, moe_get_status, moe_grouped_ffn, moe_launch_count, moe_permute,
-                   moe_profile_enable, moe_profile_read, moe_profile_reset, moe_quant_rows_e4m3,
-                   moe_route_topk, moe_shape, moe_workspace_size)
+                   moe_profile_enable, moe_profile_read, moe_profile_reset, moe_qk_norm_rope,
+                   moe_quant_rows_e4m3, moe_route_topk, moe_shape, moe_workspace_size)
 
 __all__ = ["MoELayer", "moe_shape", "make_shape", "alloc_workspace", "moe_workspace_size",
            "moe_route_topk", "moe_permute", "moe_grouped_ffn", "moe_combine", "moe_forward",
-           "moe_quant_rows_e4m3", "moe_get_status", "moe_clear_status", "moe_launch_count",
+           "moe_quant_rows_e4m3", "moe_qk_norm_rope", "moe_get_status", "moe_clear_status", "moe_launch_count",
            "moe_profile_enable", "moe_profile_reset", "moe_profile_read", "MoeError",
            "MOE_F32", "MOE_BF16", "MOE_E4M3", "MOE_FFN_AUTO", "MOE_FFN_SIMT", "MOE_FFN_TCGEN05"]
 

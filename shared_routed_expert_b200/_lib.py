@@ -22,7 +22,7 @@ EXPORTS = ("moe_workspace_size", "moe_route_topk", "moe_permute", "moe_grouped_f
            "moe_combine", "moe_forward", "moe_quant_rows_e4m3", "moe_get_status",
            "moe_clear_status", "moe_status_string", "moe_launch_count", "moe_profile_enable",
            "moe_profile_reset", "moe_profile_read", "moe_inject_wait_timeout",
-           "moe_permute_noalloc")
+           "moe_permute_noalloc", "moe_qk_norm_rope")
 
 
 class MoeError(RuntimeError):
@@ -81,6 +81,8 @@ def lib() -> C.CDLL:
         L.moe_permute_noalloc.argtypes = [S, p, p, p, p, p, p]
         L.moe_inject_wait_timeout.restype = None
         L.moe_inject_wait_timeout.argtypes = [i]
+        L.moe_qk_norm_rope.restype = i
+        L.moe_qk_norm_rope.argtypes = [i, i, i, i, i, f, p, p, i, p, p, p, p, p]
         _lib = L
     return _lib
 
@@ -168,6 +170,14 @@ def moe_permute_noalloc(shape, ids, counts, offsets, perm, inv, stream=None):
     device scratch replaces the workspace (see include/moe.h)."""
     _check("moe_permute_noalloc", lib().moe_permute_noalloc(
         C.byref(shape), _p(ids), _p(counts), _p(offsets), _p(perm), _p(inv), _stream(stream)))
+
+
+def moe_qk_norm_rope(cfg, qkv, positions, q_norm_w, k_norm_w, cos_sin, bad_positions=None, stream=None):
+    """In place on the q and k heads of qkv [T, (n_q + 2 n_kv) d] bf16; cfg
+    carries T, n_q, n_kv, d, rot, eps and max_pos = cos_sin rows."""
+    _check("moe_qk_norm_rope", lib().moe_qk_norm_rope(
+        qkv.shape[0], cfg.n_q, cfg.n_kv, cfg.d, cfg.rot, cfg.eps, _p(qkv), _p(positions), cos_sin.shape[0],
+        _p(q_norm_w), _p(k_norm_w), _p(cos_sin if cfg.rot > 0 else None), _p(bad_positions), _stream(stream)))
 
 
 def moe_quant_rows_e4m3(rows, cols, inp, codes, scales, stream=None):

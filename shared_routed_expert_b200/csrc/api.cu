@@ -436,6 +436,21 @@ moe_status moe_quant_rows_e4m3(int32_t rows, int32_t cols, const void* in, uint8
                                          static_cast<cudaStream_t>(stream)));
 }
 
+moe_status moe_qk_norm_rope(int32_t T, int32_t n_q, int32_t n_kv, int32_t head_dim, int32_t rot_dim, float eps,
+                            void* qkv, const int32_t* positions, int32_t max_pos, const void* q_norm_w,
+                            const void* k_norm_w, const float* cos_sin, int32_t* bad_positions, void* stream) {
+    if (T < 0 || n_q < 0 || n_kv < 0 || max_pos <= 0 || !(eps >= 0.0f) || !isfinite(eps))
+        return MOE_ERR_INVALID_ARG;
+    if (!qkv || !positions || !q_norm_w || !k_norm_w) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(qkv) || !aligned16(q_norm_w) || !aligned16(k_norm_w)) return MOE_ERR_INVALID_ARG;
+    if (rot_dim > 0 && (!cos_sin || !aligned16(cos_sin))) return MOE_ERR_INVALID_ARG;   // unused when rot_dim == 0
+    if (!qk_norm_rope_supported(head_dim, rot_dim)) return MOE_ERR_UNSUPPORTED;
+    return cuda_status(launch_qk_norm_rope(T, n_q, n_kv, head_dim, rot_dim, eps, static_cast<uint16_t*>(qkv),
+                                           positions, max_pos, static_cast<const uint16_t*>(q_norm_w),
+                                           static_cast<const uint16_t*>(k_norm_w), cos_sin, bad_positions,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
 moe_status moe_get_status(void* ws, void* stream) {
     if (!ws) return MOE_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);

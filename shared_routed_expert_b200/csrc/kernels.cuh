@@ -72,6 +72,12 @@ struct FfnArgs {
 };
 cudaError_t launch_ffn_simt(const FfnArgs& a, cudaStream_t stream);
 
+// ---- fused QK-norm + partial RoPE (qknorm.cu)
+bool qk_norm_rope_supported(int head_dim, int rot);
+cudaError_t launch_qk_norm_rope(int T, int n_q, int n_kv, int head_dim, int rot, float eps, uint16_t* qkv,
+                                const int32_t* pos, int max_pos, const uint16_t* q_w, const uint16_t* k_w,
+                                const float* cos_sin, int32_t* bad, cudaStream_t st);
+
 // ---- expert FFN, tcgen05 tensor-core path (ffn_tc.cu)
 bool ffn_tc_supported(const FfnArgs& a);
 cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t stream);
