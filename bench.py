@@ -367,6 +367,32 @@ def describe(cfg) -> str:
 
 # ------------------------------------------------------------------ main
 
+def bench_tp(args, dist):
+    """Tensor-parallel layer: each of the N ranks holds 1/N of every expert's
+    intermediate dimension and the ranks sum their fp32 shares with one NCCL
+    all-reduce of [T, H] (strong scaling: the layer is fixed, N GPUs share it)."""
+    from shared_routed_expert_b200 import tp
+    N = dist.world
+    cfg = synth.CONFIGS[args.workload]
+    if cfg.I % N or (cfg.I // N) % 64:
+        raise SystemExit(f"I = {cfg.I} does not split into {N} slices of a multiple of 64")
+    full = synth.make_inputs(cfg, "cpu")
+    shard = synth.to_device(tp.shard_weights(full, cfg.I, dist.rank, N), dist.device)
+    x = full["x"].to(dist.device)
+    del full
+    layer = tp.TPMoELayer(cfg, shard, N)          # the default process group: the N ranks
+    stream = torch.cuda.current_stream()
+    ms = time_steps(lambda: layer.forward(x), args.steps, args.warmup, dist, stream)
+    line = {"metric": "tensor-parallel MoE layer tokens/s", "value": cfg.T * args.steps / (ms / 1e3),
+            "unit": "tokens/s", "n_gpus": N, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+            "dtype": cfg.w_dtype, "data": "synthetic",
+            "config": {"workload": describe(cfg), "parallelism": f"tp{N} (intermediate slices of {cfg.I // N}, "
+                                                               "one fp32 all-reduce of [T, H] per layer)"}}
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def bench_qk_norm_rope(args, dist):
     """The fused QK-norm + partial RoPE kernel on its own: tokens/s from the
     kernel's CUDA events (L2 flushed between launches by an untimed 256 MB
@@ -454,6 +480,8 @@ def main():
     ap.add_argument("--op", default="moe", choices=["moe", "qk_norm_rope"],
                     help="moe: the expert layer (default); qk_norm_rope: the attention pre-processing kernel")
     ap.add_argument("--attn-workload", default="qknorm_prefill", choices=list(synth.ATTN_CONFIGS))
+    ap.add_argument("--tp", action="store_true",
+                    help="tensor parallelism over the launched ranks instead of replicas")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -467,6 +495,10 @@ def main():
     build.build()
     if args.op == "qk_norm_rope":
         bench_qk_norm_rope(args, dist)
+        dist.close()
+        return
+    if args.tp:
+        bench_tp(args, dist)
         dist.close()
         return
     cfg = synth.CONFIGS[args.workload]

@@ -71,6 +71,9 @@ typedef enum moe_dtype { MOE_F32 = 0, MOE_BF16 = 1, MOE_E4M3 = 2 } moe_dtype;
  *   bias_select_only  0: router_bias is added to the logits used for both
  *                ranking and weights; 1: the bias only ranks (ids), the
  *                weights use the logits without it
+ *   out_f32      0: moe_forward writes out in act_dtype; 1: out is fp32, the
+ *                unrounded sum (a tensor-parallel rank's partial output, to
+ *                be summed across ranks and rounded once, moe_cast_f32_bf16)
  * Derived: S = top_k + (shared_id >= 0) slots per token in the fused layout,
  * E = n_routed + (shared_id >= 0) experts, R = T*S expert rows. */
 typedef struct moe_shape {
@@ -80,6 +83,7 @@ typedef struct moe_shape {
     int32_t act_dtype, w_dtype;
     float routed_scale;
     int32_t bias_select_only;
+    int32_t out_f32;
 } moe_shape;
 
 /* Kernel choice for the expert GEMMs. AUTO picks the tcgen05 tensor-core
@@ -167,14 +171,25 @@ moe_status moe_combine(const moe_shape* shape, const void* y, const int32_t* inv
  * shared_id >= 0).
  * The expert rows are kept as fp16 scaled by a power of two per 32 columns
  * (11 significant bits) and aggregated in fp32 in slot order, rounded once to
- * act_dtype; the result is deterministic.
+ * act_dtype (or left in fp32 when shape->out_f32); the result is deterministic.
  *   x [T, H], router_w [n_routed, H], router_bias [n_routed] or NULL,
- *   w13 [E, 2I, H], s13, w2 [E, H, I], s2 as in moe_grouped_ffn, out [T, H].
+ *   w13 [E, 2I, H], s13, w2 [E, H, I], s2 as in moe_grouped_ffn, out [T, H]
+ *   (act_dtype, or fp32 when out_f32).
+ * Tensor parallelism: a rank that holds every expert's slice of the
+ * intermediate dimension (w13 rows gate[j0, j1) and up[j0, j1), w2 columns
+ * [j0, j1), I = j1 - j0, with their E4M3 scales) and calls this with out_f32 = 1
+ * computes its exact share of the layer: the SwiGLU is per intermediate column,
+ * so the ranks' outputs sum to the layer's (E4M3 layers quantise h per row of
+ * the slice). Sum the shares across ranks, then moe_cast_f32_bf16.
  * Needs moe_workspace_size(shape, fuse_shared) bytes of ws. */
 moe_status moe_forward(const moe_shape* shape, const void* x, const float* router_w,
                        const float* router_bias, const void* w13, const float* s13,
                        const void* w2, const float* s2, int fuse_shared, void* out,
                        void* ws, size_t ws_bytes, int ffn_impl, void* stream);
+
+/* out[i] = bf16(in[i]), round to nearest even; n a multiple of 4, in 16-byte
+ * and out 8-byte aligned. */
+moe_status moe_cast_f32_bf16(size_t n, const float* in, void* out, void* stream);
 
 /* Per-row E4M3 quantisation used before each E4M3 GEMM: scale = amax/448 in
  * fp32 (amax = 0 -> 1), codes = E4M3_rn_satfinite(v / scale) (fp32 divide).

@@ -22,7 +22,7 @@ EXPORTS = ("moe_workspace_size", "moe_route_topk", "moe_permute", "moe_grouped_f
            "moe_combine", "moe_forward", "moe_quant_rows_e4m3", "moe_get_status",
            "moe_clear_status", "moe_status_string", "moe_launch_count", "moe_profile_enable",
            "moe_profile_reset", "moe_profile_read", "moe_inject_wait_timeout",
-           "moe_permute_noalloc", "moe_qk_norm_rope")
+           "moe_permute_noalloc", "moe_qk_norm_rope", "moe_cast_f32_bf16")
 
 
 class MoeError(RuntimeError):
@@ -35,7 +35,7 @@ class moe_shape(C.Structure):
     _fields_ = [("T", C.c_int32), ("H", C.c_int32), ("I", C.c_int32), ("n_routed", C.c_int32),
                 ("top_k", C.c_int32), ("shared_id", C.c_int32), ("shared_weight", C.c_float),
                 ("renormalize", C.c_int32), ("act_dtype", C.c_int32), ("w_dtype", C.c_int32),
-                ("routed_scale", C.c_float), ("bias_select_only", C.c_int32)]
+                ("routed_scale", C.c_float), ("bias_select_only", C.c_int32), ("out_f32", C.c_int32)]
 
 
 _lib = None
@@ -81,6 +81,8 @@ def lib() -> C.CDLL:
         L.moe_permute_noalloc.argtypes = [S, p, p, p, p, p, p]
         L.moe_inject_wait_timeout.restype = None
         L.moe_inject_wait_timeout.argtypes = [i]
+        L.moe_cast_f32_bf16.restype = i
+        L.moe_cast_f32_bf16.argtypes = [sz, p, p, p]
         L.moe_qk_norm_rope.restype = i
         L.moe_qk_norm_rope.argtypes = [i, i, i, i, i, f, p, p, i, p, p, p, p, p]
         _lib = L
@@ -117,7 +119,8 @@ def make_shape(cfg, T: int | None = None) -> moe_shape:
     return moe_shape(cfg.T if T is None else T, cfg.H, cfg.I, cfg.n_routed, cfg.top_k,
                      cfg.shared_id, cfg.shared_weight, int(cfg.renormalize),
                      DTYPES[cfg.act_dtype], DTYPES[cfg.w_dtype],
-                     float(getattr(cfg, "routed_scale", 1.0)), int(getattr(cfg, "bias_select_only", False)))
+                     float(getattr(cfg, "routed_scale", 1.0)), int(getattr(cfg, "bias_select_only", False)),
+                     int(getattr(cfg, "out_f32", False)))
 
 
 def moe_workspace_size(shape: moe_shape, fuse_shared: bool = True) -> int:
@@ -178,6 +181,11 @@ def moe_qk_norm_rope(cfg, qkv, positions, q_norm_w, k_norm_w, cos_sin, bad_posit
     _check("moe_qk_norm_rope", lib().moe_qk_norm_rope(
         qkv.shape[0], cfg.n_q, cfg.n_kv, cfg.d, cfg.rot, cfg.eps, _p(qkv), _p(positions), cos_sin.shape[0],
         _p(q_norm_w), _p(k_norm_w), _p(cos_sin if cfg.rot > 0 else None), _p(bad_positions), _stream(stream)))
+
+
+def moe_cast_f32_bf16(inp, out, stream=None):
+    """out (bf16) = inp (fp32) rounded to nearest even, same element count."""
+    _check("moe_cast_f32_bf16", lib().moe_cast_f32_bf16(inp.numel(), _p(inp), _p(out), _stream(stream)))
 
 
 def moe_quant_rows_e4m3(rows, cols, inp, codes, scales, stream=None):

@@ -145,6 +145,7 @@ moe_status check_shape(const moe_shape* s) {
     if (s->renormalize != 0 && s->renormalize != 1) return MOE_ERR_INVALID_ARG;
     if (!(s->routed_scale > 0.0f) || !isfinite(s->routed_scale)) return MOE_ERR_INVALID_ARG;
     if (s->bias_select_only != 0 && s->bias_select_only != 1) return MOE_ERR_INVALID_ARG;
+    if (s->out_f32 != 0 && s->out_f32 != 1) return MOE_ERR_INVALID_ARG;
     if (s->H % 256 != 0 || s->I % 64 != 0) return MOE_ERR_UNSUPPORTED;
     if (s->n_routed > 256 || s->top_k > 32) return MOE_ERR_UNSUPPORTED;
     const bool ok_dt = (s->act_dtype == MOE_F32 && s->w_dtype == MOE_F32) ||
@@ -332,6 +333,12 @@ moe_status moe_combine(const moe_shape* shape, const void* y, const int32_t* inv
                                       0.0f, out, st));
 }
 
+moe_status moe_cast_f32_bf16(size_t n, const float* in, void* out, void* stream) {
+    if (n % 4 != 0 || (n > 0 && (!in || !out))) return MOE_ERR_INVALID_ARG;
+    if (n > 0 && (!aligned16(in) || (reinterpret_cast<uintptr_t>(out) & 7u))) return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_cast_f32_bf16(n, in, static_cast<uint16_t*>(out), static_cast<cudaStream_t>(stream)));
+}
+
 moe_status moe_forward(const moe_shape* shape, const void* x, const float* router_w,
                        const float* router_bias, const void* w13, const float* s13,
                        const void* w2, const float* s2, int fuse_shared, void* out, void* ws,
@@ -404,7 +411,7 @@ moe_status moe_forward(const moe_shape* shape, const void* x, const float* route
         a.y = at<void>(ws, L.sh_y);
         a.yexp = f32_act ? nullptr : at<int8_t>(ws, L.sh_yexp);
         a.unit_rows = 0;
-    a.cta_pair = 0;
+        a.cta_pair = 0;
         a.direct_e = -1;
         a.max_mtiles = ceil_div(d.T, kTileM);
         a.status = at<DevStatus>(ws, L.status);
@@ -422,7 +429,7 @@ moe_status moe_forward(const moe_shape* shape, const void* x, const float* route
             err = launch_combine_f16s(d.T, d.S, d.H, at<uint16_t>(ws, L.y), at<int8_t>(ws, L.yexp), inv, wts,
                                       fused ? nullptr : at<uint16_t>(ws, L.sh_y),
                                       fused ? nullptr : at<int8_t>(ws, L.sh_yexp), shape->shared_weight,
-                                      static_cast<uint16_t*>(out), st);
+                                      out, shape->out_f32 != 0, st);
     }
     return cuda_status(err);
 }

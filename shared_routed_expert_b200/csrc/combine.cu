@@ -11,6 +11,8 @@
 // so that storing the rows adds ~2^-12 relative error per slot instead of
 // bf16's 2^-9). `add` (weight add_w) is an optional [T, H] term added last:
 // the unfused layer's separately computed shared expert.
+#include <algorithm>
+
 #include "kernels.cuh"
 
 namespace sre {
@@ -102,7 +104,9 @@ __global__ void __launch_bounds__(CB_THREADS) combine_f32_kernel(int T, int S, i
 
 // Scaled-fp16 rows (see the GEMM2 epilogue): value = fp16 * 2^k, one k per 32
 // columns. Each thread owns 8-column vectors of the token's row (4 threads per
-// exponent byte).
+// exponent byte). The sum is written rounded to bf16, or as fp32 (kF32Out: a
+// tensor-parallel rank's partial output).
+template <bool kF32Out>
 __global__ void __launch_bounds__(CB_THREADS) combine_f16s_kernel(int T, int S, int H,
                                                                   const uint4* __restrict__ y,
                                                                   const int8_t* __restrict__ yexp,
@@ -110,7 +114,7 @@ __global__ void __launch_bounds__(CB_THREADS) combine_f16s_kernel(int T, int S, 
                                                                   const float* __restrict__ w,
                                                                   const uint4* __restrict__ add,
                                                                   const int8_t* __restrict__ addexp,
-                                                                  float add_w, uint4* __restrict__ out) {
+                                                                  float add_w, void* __restrict__ out) {
     const int t = blockIdx.x;
     const int nv = H / 8, ne = H / 32;
     __shared__ int32_t s_row[64];
@@ -162,9 +166,24 @@ __global__ void __launch_bounds__(CB_THREADS) combine_f16s_kernel(int T, int S, 
                 acc[2 * j + 1] = __fmaf_rn(wk, f.y, acc[2 * j + 1]);
             }
         }
-        out[static_cast<size_t>(t) * nv + i] =
-            make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
-                       pack_bf16x2(acc[6], acc[7]));
+        if constexpr (kF32Out) {
+            float4* o = static_cast<float4*>(out) + (static_cast<size_t>(t) * nv + i) * 2;
+            o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        } else {
+            static_cast<uint4*>(out)[static_cast<size_t>(t) * nv + i] =
+                make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
+                           pack_bf16x2(acc[6], acc[7]));
+        }
+    }
+}
+
+__global__ void __launch_bounds__(256) cast_f32_bf16_kernel(size_t n4, const float4* __restrict__ in,
+                                                            uint2* __restrict__ out) {
+    for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+         i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+        const float4 v = in[i];
+        out[i] = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
     }
 }
 
@@ -172,12 +191,28 @@ __global__ void __launch_bounds__(CB_THREADS) combine_f16s_kernel(int T, int S, 
 
 cudaError_t launch_combine_f16s(int T, int S, int H, const uint16_t* y16, const int8_t* yexp,
                                 const int32_t* inv, const float* w, const uint16_t* add16,
-                                const int8_t* addexp, float add_w, uint16_t* out, cudaStream_t stream) {
+                                const int8_t* addexp, float add_w, void* out, bool out_f32, cudaStream_t stream) {
     if (T == 0) return cudaSuccess;
     ProfileScope ps("combine", stream);
-    combine_f16s_kernel<<<T, CB_THREADS, 0, stream>>>(T, S, H, reinterpret_cast<const uint4*>(y16), yexp, inv,
-                                                      w, reinterpret_cast<const uint4*>(add16), addexp, add_w,
-                                                      reinterpret_cast<uint4*>(out));
+    if (out_f32)
+        combine_f16s_kernel<true><<<T, CB_THREADS, 0, stream>>>(T, S, H, reinterpret_cast<const uint4*>(y16), yexp,
+                                                                inv, w, reinterpret_cast<const uint4*>(add16),
+                                                                addexp, add_w, out);
+    else
+        combine_f16s_kernel<false><<<T, CB_THREADS, 0, stream>>>(T, S, H, reinterpret_cast<const uint4*>(y16),
+                                                                 yexp, inv, w, reinterpret_cast<const uint4*>(add16),
+                                                                 addexp, add_w, out);
+    note_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_cast_f32_bf16(size_t n, const float* in, uint16_t* out, cudaStream_t stream) {
+    if (n == 0) return cudaSuccess;
+    ProfileScope ps("cast_bf16", stream);
+    const size_t n4 = n / 4;
+    const unsigned blocks = static_cast<unsigned>(std::min<size_t>((n4 + 255) / 256, 148 * 16));
+    cast_f32_bf16_kernel<<<blocks, 256, 0, stream>>>(n4, reinterpret_cast<const float4*>(in),
+                                                     reinterpret_cast<uint2*>(out));
     note_launch();
     return cudaGetLastError();
 }

@@ -93,6 +93,8 @@ cudaError_t launch_combine(int T, int S, int H, int act_dtype, const void* y, co
 // same over scaled-fp16 rows (y16/yexp, add16/addexp as produced by the GEMM2 epilogue), bf16 out
 cudaError_t launch_combine_f16s(int T, int S, int H, const uint16_t* y16, const int8_t* yexp,
                                 const int32_t* inv, const float* w, const uint16_t* add16,
-                                const int8_t* addexp, float add_w, uint16_t* out, cudaStream_t stream);
+                                const int8_t* addexp, float add_w, void* out, bool out_f32, cudaStream_t stream);
+// fp32 -> bf16, round to nearest even (the last step of a tensor-parallel layer)
+cudaError_t launch_cast_f32_bf16(size_t n, const float* in, uint16_t* out, cudaStream_t stream);
 
 }  // namespace sre

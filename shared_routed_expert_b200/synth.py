@@ -52,6 +52,7 @@ class LayerConfig:
     renormalize: bool = True
     routed_scale: float = 1.0        # routed slots weigh routed_scale * softmax
     bias_select_only: bool = False   # router bias ranks the experts but does not weigh them
+    out_f32: bool = False            # the layer writes its unrounded fp32 sum (tensor-parallel partials)
 
     @property
     def n_experts(self) -> int:

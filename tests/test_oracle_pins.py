@@ -530,3 +530,19 @@ def test_qk_norm_is_scale_invariant_and_position_zero_is_the_identity_rotation()
     rms = torch.sqrt((heads ** 2).mean(-1, keepdim=True))
     w = torch.cat([inp["q_w"].double().expand(cfg.n_q, -1), inp["k_w"].double().expand(cfg.n_kv, -1)])
     assert np.allclose(a, (heads / rms * w).numpy(), rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------------------------ tensor-parallel slices
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_intermediate_slices_sum_to_the_layer(world):
+    """The SwiGLU is per intermediate column, so the layers of the N slices of
+    every expert's intermediate dimension (router replicated) sum to the full
+    layer (bf16: h is rounded per element either way; fp64 sums)."""
+    from shared_routed_expert_b200 import tp
+    cfg = synth.variant(synth.CONFIGS["prefill_bf16"], T=10, H=256, I=256, n_routed=8, top_k=3)
+    inp = synth.make_inputs(cfg)
+    full = oracle.Layer(cfg, inp).forward(n_threads=2)["out"]
+    parts = [oracle.Layer(tp.local_config(cfg, world), tp.shard_weights(inp, cfg.I, r, world))
+             .forward(n_threads=2)["out"] for r in range(world)]
+    assert np.allclose(sum(parts), full, rtol=1e-12, atol=1e-14)
