@@ -59,6 +59,31 @@ class MoELayer:
                     impl=self.impl, stream=stream)
         return out
 
+    def capture(self, x: torch.Tensor, out: torch.Tensor) -> torch.cuda.CUDAGraph:
+        """Record one forward from the device buffer x into out as a CUDA graph:
+        replay() reruns every kernel of the layer with one launch from the host
+        (new inputs go into x in place). The kernels take no host decisions and
+        allocate nothing, so the recorded launches are the eager ones."""
+        was = self.profiling_off()
+        try:
+            self.forward(x, out)                 # one eager pass sets up every kernel
+            torch.cuda.synchronize(self.device)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self.forward(x, out)
+        finally:
+            moe_profile_enable(was)
+        return g
+
+    @staticmethod
+    def profiling_off() -> bool:
+        """Turns per-kernel event timing off (it does not belong inside a graph)
+        and returns whether it was on."""
+        from ._lib import profile_enabled
+        was = profile_enabled()
+        moe_profile_enable(False)
+        return was
+
     def forward_host(self, x_host: torch.Tensor, out_host: torch.Tensor, x_dev: torch.Tensor,
                      out_dev: torch.Tensor, stream=None) -> torch.Tensor:
         """Host buffers in and out: copy x to the device, run the layer, copy

@@ -205,8 +205,18 @@ def moe_launch_count() -> int:
     return int(lib().moe_launch_count())
 
 
+_prof_on = False
+
+
 def moe_profile_enable(on: bool):
+    global _prof_on
     lib().moe_profile_enable(int(on))
+    _prof_on = bool(on)
+
+
+def profile_enabled() -> bool:
+    """Whether per-kernel event timing was last switched on through this module."""
+    return _prof_on
 
 
 def moe_profile_reset():

@@ -166,3 +166,25 @@ def test_pipelined_host_submission_matches_forward():
     for x, o in zip(xs, outs):
         ref = layer.forward(x.to(DEV)).cpu()
         assert torch.equal(o.view(torch.int16), ref.view(torch.int16))
+
+
+@pytest.mark.parametrize("name", ["bf16_small", "fp8_i192_zipf"])
+def test_cuda_graph_replay_equals_eager(name):
+    """The layer recorded as one CUDA graph gives the eager pass's bits, also
+    after new inputs are written into the captured input buffer."""
+    cfg = SMALL[name]
+    d = synth.to_device(synth.make_inputs(cfg), DEV)
+    layer = MoELayer(cfg, d)
+    x = d["x"].clone()
+    out = torch.empty_like(x)
+    g = layer.capture(x, out)
+    ref = layer.forward(x).clone()
+    g.replay()
+    torch.cuda.synchronize()
+    assert layer.status() == _lib.MOE_OK
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+    x.copy_(torch.flip(d["x"], [0]))               # new batch, same buffer
+    g.replay()
+    ref2 = layer.forward(x).clone()
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), ref2.view(torch.int16))
