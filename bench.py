@@ -250,12 +250,14 @@ def algorithmic(cfg, kernel: str, counts: np.ndarray | None):
 # dominated by the touched experts' weights, so it scales with the launch.
 # Keyed by (kernel, weight dtype, tensor-core work unit).
 PROFILED_TRAFFIC_RATIO = {("gemm1_tc", "bf16", 256): 1.09,
-                          ("gemm1_tc", "bf16", "pair256x512"): 1.02, ("gemm2_tc", "bf16", "pair256x512"): 0.97}
+                          ("gemm1_tc", "bf16", "pair256x512"): 1.02, ("gemm2_tc", "bf16", "pair256x512"): 0.97,
+                          ("gemm1_tc", "bf16", "swap"): 1.013}
 
 
-def unit_rows(cfg, ffn: str):
-    """Tensor-core work unit the run uses: 128, 256 (one CTA), "pair256"
-    (256 x 256 tiles over a CTA pair) or "pair256x512" (256 x 512 pair tiles)."""
+def unit_rows(cfg, ffn: str, kernel: str = "gemm1_tc"):
+    """Tensor-core work unit `kernel` uses in the run: 128, 256 (one CTA),
+    "pair256" (256 x 256 tiles over a CTA pair), "pair256x512" (256 x 512 pair
+    tiles) or "swap" (CTA pairs, 256 weight rows x up to 256 tokens)."""
     if ffn == "tcgen05_m128":
         return 128
     if ffn == "tcgen05_m256":
@@ -264,12 +266,16 @@ def unit_rows(cfg, ffn: str):
         return "pair256"
     if ffn == "tcgen05_wide":
         return "pair256x512"
-    return "pair256x512" if (cfg.w_dtype == "bf16" and cfg.rows >= 192 * cfg.n_experts) else 128
+    if ffn == "tcgen05_swap":
+        return "swap"
+    if cfg.w_dtype == "bf16" and cfg.rows >= 192 * cfg.n_experts:
+        return "swap" if (kernel == "gemm1_tc" and cfg.I % 256 == 0) else "pair256x512"
+    return 128
 
 
-def roofline_of(cfg, kernel: str, ms_per_launch: float, counts, pk, urows=128) -> dict:
+def roofline_of(cfg, kernel: str, ms_per_launch: float, counts, pk, ffn: str = "auto") -> dict:
     flops, nbytes = algorithmic(cfg, kernel, counts)
-    ratio = PROFILED_TRAFFIC_RATIO.get((kernel, cfg.w_dtype, urows))
+    ratio = PROFILED_TRAFFIC_RATIO.get((kernel, cfg.w_dtype, unit_rows(cfg, ffn, kernel)))
     traffic = int(ratio * nbytes) if (ratio and nbytes) else None
     t = ms_per_launch / 1000.0
     tpk = pk["bf16_tflops"] * (2.0 if cfg.w_dtype == "e4m3" else 1.0)
@@ -469,7 +475,7 @@ def main():
     ap.add_argument("--workload", default="prefill_bf16", choices=list(synth.CONFIGS))
     ap.add_argument("--ffn", default="auto",
                     choices=["auto", "simt", "tcgen05", "tcgen05_m128", "tcgen05_m256", "tcgen05_pair",
-                             "tcgen05_wide"])
+                             "tcgen05_wide", "tcgen05_swap"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--quick", action="store_true",
@@ -509,7 +515,8 @@ def main():
                                  f"I={args.inter or cfg.I}]")
     impl = {"auto": _lib.MOE_FFN_AUTO, "simt": _lib.MOE_FFN_SIMT, "tcgen05": _lib.MOE_FFN_TCGEN05,
             "tcgen05_m128": _lib.MOE_FFN_TCGEN05_M128, "tcgen05_m256": _lib.MOE_FFN_TCGEN05_M256,
-            "tcgen05_pair": _lib.MOE_FFN_TCGEN05_PAIR, "tcgen05_wide": _lib.MOE_FFN_TCGEN05_WIDE}[args.ffn]
+            "tcgen05_pair": _lib.MOE_FFN_TCGEN05_PAIR, "tcgen05_wide": _lib.MOE_FFN_TCGEN05_WIDE,
+            "tcgen05_swap": _lib.MOE_FFN_TCGEN05_SWAP}[args.ffn]
     d = synth.make_inputs(cfg, dist.device)
     stream = torch.cuda.current_stream(dist.device)
     fused = MoELayer(cfg, d, fuse_shared=True, impl=impl)
@@ -599,11 +606,10 @@ def main():
 
     roof = None
     if tab:
-        ur = unit_rows(cfg, args.ffn)
         top = max(tab, key=lambda k: tab[k]["total_ms"])
-        roof = roofline_of(cfg, top, tab[top]["ms_per_launch"], counts, pk, ur)
+        roof = roofline_of(cfg, top, tab[top]["ms_per_launch"], counts, pk, args.ffn)
         for k in tab:
-            tab[k]["roofline"] = roofline_of(cfg, k, tab[k]["ms_per_launch"], counts, pk, ur)
+            tab[k]["roofline"] = roofline_of(cfg, k, tab[k]["ms_per_launch"], counts, pk, args.ffn)
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": N, "steps": args.steps,

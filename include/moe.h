@@ -89,18 +89,22 @@ typedef struct moe_shape {
 /* Kernel choice for the expert GEMMs. AUTO picks the tcgen05 tensor-core
  * kernels for bf16/E4M3 weights and the CUDA-core kernels for fp32. TCGEN05
  * picks the tensor-core work unit itself: for bf16 weights whose groups average
- * >= 192 rows, 256 x 512 tiles on CTA pairs (as TCGEN05_WIDE), else 128-row
- * units on single CTAs (as TCGEN05_M128);
+ * >= 192 rows, CTA pairs with GEMM1 as TCGEN05_SWAP and GEMM2 as TCGEN05_WIDE,
+ * else 128-row units on single CTAs (as TCGEN05_M128);
  * TCGEN05_M128 / TCGEN05_M256 force one of them; TCGEN05_PAIR forces 256-row
  * units split over a pair of CTAs on the two SMs of a TPC (tcgen05 cta_group::2,
  * each SM staging half of every weight tile); TCGEN05_WIDE the same with
  * 256 x 512 tiles per pair (two N = 256 MMAs sharing each activation stage)
  * where the output width allows (GEMM1: I % 256 == 0, GEMM2: H % 512 == 0;
- * 256 x 256 pair tiles otherwise). */
+ * 256 x 256 pair tiles otherwise); TCGEN05_SWAP runs CTA pairs with the
+ * operands exchanged: 256 weight rows are the MMA's M and up to 256 rows of one
+ * expert's group its N, in steps of 16, so a group pads to a multiple of 16
+ * rows instead of a multiple of 128 (GEMM1 where I % 256 == 0, GEMM2 where
+ * H % 512 == 0; as TCGEN05_WIDE otherwise). */
 typedef enum moe_ffn_impl {
     MOE_FFN_AUTO = 0, MOE_FFN_SIMT = 1, MOE_FFN_TCGEN05 = 2,
     MOE_FFN_TCGEN05_M128 = 3, MOE_FFN_TCGEN05_M256 = 4, MOE_FFN_TCGEN05_PAIR = 5,
-    MOE_FFN_TCGEN05_WIDE = 6
+    MOE_FFN_TCGEN05_WIDE = 6, MOE_FFN_TCGEN05_SWAP = 7
 } moe_ffn_impl;
 
 /* Bytes of workspace moe_forward needs for this shape (fused or not). The

@@ -15,7 +15,7 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE = 0, 1, 2, 3
 MOE_ERR_CUDA, MOE_ERR_TIMEOUT, MOE_ERR_DEVICE = 4, 5, 6
 MOE_F32, MOE_BF16, MOE_E4M3 = 0, 1, 2
 (MOE_FFN_AUTO, MOE_FFN_SIMT, MOE_FFN_TCGEN05, MOE_FFN_TCGEN05_M128, MOE_FFN_TCGEN05_M256,
- MOE_FFN_TCGEN05_PAIR, MOE_FFN_TCGEN05_WIDE) = 0, 1, 2, 3, 4, 5, 6
+ MOE_FFN_TCGEN05_PAIR, MOE_FFN_TCGEN05_WIDE, MOE_FFN_TCGEN05_SWAP) = 0, 1, 2, 3, 4, 5, 6, 7
 DTYPES = {"f32": MOE_F32, "bf16": MOE_BF16, "e4m3": MOE_E4M3}
 
 EXPORTS = ("moe_workspace_size", "moe_route_topk", "moe_permute", "moe_grouped_ffn",

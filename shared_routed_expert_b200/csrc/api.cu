@@ -179,12 +179,13 @@ cudaError_t run_ffn(const FfnArgs& in, int impl, cudaStream_t st) {
     const bool tc_ok = ffn_tc_supported(in);
     const bool tc_forced = impl == MOE_FFN_TCGEN05 || impl == MOE_FFN_TCGEN05_M128 ||
                            impl == MOE_FFN_TCGEN05_M256 || impl == MOE_FFN_TCGEN05_PAIR ||
-                           impl == MOE_FFN_TCGEN05_WIDE;
+                           impl == MOE_FFN_TCGEN05_WIDE || impl == MOE_FFN_TCGEN05_SWAP;
     if (tc_forced || (impl == MOE_FFN_AUTO && in.w_dtype != MOE_F32 && tc_ok)) {
         if (!tc_ok) return cudaErrorNotSupported;
         FfnArgs a = in;
         a.unit_rows = impl == MOE_FFN_TCGEN05_M128 ? 128 : (impl == MOE_FFN_TCGEN05_M256 ? 256 : 0);
         a.cta_pair = impl == MOE_FFN_TCGEN05_PAIR ? 1 : impl == MOE_FFN_TCGEN05_WIDE ? 2
+                   : impl == MOE_FFN_TCGEN05_SWAP ? 3
                    : (impl == MOE_FFN_AUTO || impl == MOE_FFN_TCGEN05) ? -1 : 0;
         return launch_ffn_tc(a, st);
     }
@@ -192,7 +193,7 @@ cudaError_t run_ffn(const FfnArgs& in, int impl, cudaStream_t st) {
 }
 
 moe_status check_impl(int impl, const moe_shape& s) {
-    if (impl < MOE_FFN_AUTO || impl > MOE_FFN_TCGEN05_WIDE) return MOE_ERR_INVALID_ARG;
+    if (impl < MOE_FFN_AUTO || impl > MOE_FFN_TCGEN05_SWAP) return MOE_ERR_INVALID_ARG;
     if (impl >= MOE_FFN_TCGEN05 && s.w_dtype == MOE_F32) return MOE_ERR_UNSUPPORTED;
     return MOE_OK;
 }

@@ -63,6 +63,7 @@ struct TcParams {
     int out_ld;
     const float* row_scale; // E4M3: per-row activation scale [R]
     int direct_e;           // GEMM1: expert whose A rows are read from the token matrix (tmA2), or -1
+    int first_e;            // tokens-as-N kernel: expert whose units run first (the largest group), or -1
     const float* direct_scale;  // E4M3: per-token scale of that expert's rows
     const float* col_scale; // E4M3: per-output-channel weight scale (s13 [E, 2I] or s2 [E, H])
     // GEMM2 with yexp != null: rows stored as fp16(v * 2^-k), k per 32 columns in yexp
@@ -758,6 +759,372 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
     }
 }
 
+// ------------------------------------------------------------------ tokens as the N dimension
+// grouped_gemm_swap_kernel computes the transposed products, D^T = W . X^T: a
+// unit is 256 weight rows (M, 128 per CTA of the pair) times up to 256 token
+// rows of one expert (N, a multiple of 16, half staged by each CTA). A group
+// of c rows is cut into ceil(c / 256) units of equal size rounded up to 16
+// rows, so a routed group of ~205 rows costs 208 rows of MMA work instead of a
+// 256-row M tile. TMEM lane = output feature, column = token.
+//   GEMM1: sub-tile 0 = gate rows n0 + 128 r .. +127 of W13[e] (CTA rank r),
+//          sub-tile 1 = the up rows of the same h columns; accumulators in
+//          TMEM columns 0 and 256; every epilogue warp reads both and applies
+//          SwiGLU, the two warps of a lane group taking alternate 32-token chunks.
+//   GEMM2: sub-tile j = output columns n0 + 256 j + 128 r .. +127; warps 2-5
+//          drain sub-tile 0 and warps 6-9 sub-tile 1. A scaled-fp16 chunk (32
+//          output columns of one row) is one warp's 32 lanes: its exponent comes
+//          from a warp max-reduction per token.
+// Both sub-tiles of a stage share the token tile. TMEM is full, so the next
+// unit's MMAs wait for the epilogue of this one. The pair protocol (rank 0
+// arms and issues, commits multicast to both CTAs, epilogues arrive on rank
+// 0's barrier, bounded waits and abort) is that of grouped_gemm_pair_kernel.
+
+struct SwapUnit {
+    int e, row0, rows, n0;
+};
+
+__device__ __forceinline__ SwapUnit decode_swap(int id, const int* s_unit, const int* s_off, int E, int NT,
+                                                int bn_out) {
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_unit[mid] * NT <= id) lo = mid; else hi = mid - 1;
+    }
+    const int e = lo;
+    const int nu = s_unit[e + 1] - s_unit[e];
+    const int local = id - s_unit[e] * NT;
+    const int nt = local / nu;
+    const int mu = local - nt * nu;
+    const int count = s_off[e + 1] - s_off[e];
+    const int rpu = ((count + nu - 1) / nu + 15) & ~15;      // <= 256 since nu = ceil(count / 256)
+    SwapUnit t;
+    t.e = e;
+    t.row0 = s_off[e] + mu * rpu;
+    t.rows = min(rpu, count - mu * rpu);                      // >= 1
+    t.n0 = nt * bn_out;
+    return t;
+}
+
+// One warp's 32 x 32 block of 16-bit results with lane = output column col0 +
+// lane and v[i] = output row row0 + i: written column-wise into the warp's 2 KB
+// slice (rows of 64 bytes, 16-byte chunks XOR-swizzled by (row >> 1) & 3: each
+// instruction writes one row, conflict-free), then stored row-wise as
+// stage_store does; rows at or past row_end are not stored.
+__device__ __forceinline__ void stage_store_t(uint8_t* slice, const uint16_t (&v)[32], int lane, uint16_t* out,
+                                              int ld, int row0, int row_end, int col0) {
+    const int chunk = lane >> 3, within = (lane & 7) * 2;
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+        *reinterpret_cast<uint16_t*>(slice + i * 64 + ((chunk ^ ((i >> 1) & 3)) * 16) + within) = v[i];
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int r = j * 8 + (lane >> 2);
+        const int c = lane & 3;
+        const uint4 w = *reinterpret_cast<const uint4*>(slice + r * 64 + ((c ^ ((r >> 1) & 3)) * 16));
+        const int grow = row0 + r;
+        if (grow < row_end)
+            *reinterpret_cast<uint4*>(out + static_cast<size_t>(grow) * ld + col0 + c * 8) = w;
+    }
+    __syncwarp();
+}
+
+__device__ __forceinline__ uint16_t bf16_bits(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
+__device__ __forceinline__ uint16_t f16_bits(float x) { return __half_as_ushort(__float2half_rn(x)); }
+
+template <int kRowB>
+struct RingS {
+    static constexpr int A_SUB = TC_BM * kRowB;         // 128 weight rows of one sub-tile
+    static constexpr int A_TILE = 2 * A_SUB;
+    static constexpr int B_TILE = 128 * kRowB;          // this CTA's token rows (N / 2 <= 128)
+    static constexpr int STAGE = A_TILE + B_TILE;
+    static constexpr int N = (TC_RING_BYTES / STAGE) > 8 ? 8 : (TC_RING_BYTES / STAGE);
+    static constexpr int SMEM = N * STAGE + 8 * 2048 + 1024;
+};
+
+template <bool kFp8, bool kGemm1, int kRowB>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
+    grouped_gemm_swap_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                             const __grid_constant__ CUtensorMap tmX2, const TcParams p) {
+    using RG = RingS<kRowB>;
+    constexpr int NSTAGE = RG::N;
+    constexpr int KEL = kFp8 ? kRowB : kRowB / 2;
+    constexpr int KSTEPS = kRowB / 32;
+    constexpr int EPI_WARPS = 8;
+
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint64_t full_bar[NSTAGE], empty_bar[NSTAGE], tfull_bar, tempty_bar, drain_bar;
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_abort;
+    __shared__ int s_off[TC_MAXE], s_unit[TC_MAXE];
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = ptx::cluster_ctarank();
+    const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+    const uint32_t raw = ptx::smem_u32(smem_raw);
+    uint8_t* base = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+    uint8_t* sA = base;
+    uint8_t* sB = base + NSTAGE * RG::A_TILE;
+    uint8_t* sStage = sB + NSTAGE * RG::B_TILE;
+    volatile int* abort_flag = &s_abort;
+    const uint32_t peer_abort = ptx::mapa(&s_abort, rank ^ 1u);
+
+    for (int i = threadIdx.x; i <= p.E; i += blockDim.x) s_off[i] = p.offsets[i];
+    if (warp == 0) {
+        // prefix of units per expert: ceil(count / 256) = pairs of 128-row tiles
+        int carry = 0;
+        for (int e0 = 0; e0 <= p.E; e0 += 32) {
+            const int e = e0 + lane;
+            const int units = (e < p.E) ? (p.tile_off[e + 1] - p.tile_off[e] + 1) >> 1 : 0;
+            int inc = units;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int o = __shfl_up_sync(0xFFFFFFFFu, inc, off);
+                if (lane >= off) inc += o;
+            }
+            if (e <= p.E) s_unit[e] = carry + inc - units;
+            carry += __shfl_sync(0xFFFFFFFFu, inc, 31);
+        }
+    }
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NSTAGE; ++s) {
+            ptx::mbar_init(&full_bar[s], 1);
+            ptx::mbar_init(&empty_bar[s], 1);
+        }
+        ptx::mbar_init(&tfull_bar, 1);
+        ptx::mbar_init(&tempty_bar, 2 * EPI_WARPS * 32);     // every epilogue thread of both CTAs
+        ptx::mbar_init(&drain_bar, 1);
+        s_abort = 0;
+        ptx::fence_mbar_init();
+        ptx::prefetch_tmap(&tmW);
+        ptx::prefetch_tmap(&tmX);
+        if (p.direct_e >= 0) ptx::prefetch_tmap(&tmX2);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc_pair(&s_tmem, TC_TMEM_COLS);
+        ptx::tmem_relinquish_pair();
+    }
+    ptx::tc_fence_before();
+    ptx::cluster_sync();
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = s_tmem;
+    const int total = s_unit[p.E] * p.n_tiles_n;
+    // the largest group's units (all 256 rows) go first, so that the last wave
+    // holds the smaller routed units; every role walks the same rotated order
+    const int rot = p.first_e >= 0 ? s_unit[p.first_e] * p.n_tiles_n : 0;
+    auto unit = [&](int u) {
+        const int v = u + rot;
+        return decode_swap(v < total ? v : v - total, s_unit, s_off, p.E, p.n_tiles_n, p.bn_out);
+    };
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- producers (both CTAs)
+        if (!p.inject_stall) {
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int u = cluster; u < total; u += nclusters) {
+                const SwapUnit t = unit(u);
+                int ok = 1;
+                if (lane == 0) {
+                    const bool direct = t.e == p.direct_e;
+                    const CUtensorMap* xm = direct ? &tmX2 : &tmX;
+                    const int n_half = ((t.rows + 15) & ~15) >> 1;
+                    const int xr = (direct ? t.row0 - s_off[t.e] : t.row0) + static_cast<int>(rank) * n_half;
+                    constexpr uint32_t tx = 2u * (RG::A_TILE + RG::B_TILE);
+                    for (int kb = 0; kb < p.k_blocks; ++kb) {
+                        if (!ptx::mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, p.wait_limit, p.status, 1u)) {
+                            ok = 0;
+                            break;
+                        }
+                        const uint32_t fb = ptx::mapa(&full_bar[stage], 0);
+                        if (rank == 0) ptx::mbar_arrive_expect_tx(&full_bar[stage], tx);
+                        const int kx = kb * KEL;
+                        uint8_t* a_dst = sA + stage * RG::A_TILE;
+                        if constexpr (kGemm1) {
+                            const int wr = t.n0 + static_cast<int>(rank) * TC_BM;
+                            ptx::tma_load_3d_pair(a_dst, &tmW, fb, kx, wr, 2 * t.e);
+                            ptx::tma_load_3d_pair(a_dst + RG::A_SUB, &tmW, fb, kx, wr, 2 * t.e + 1);
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 2; ++j)
+                                ptx::tma_load_2d_pair(a_dst + j * RG::A_SUB, &tmW, fb, kx,
+                                                      t.e * p.H + t.n0 + j * 256 + static_cast<int>(rank) * TC_BM);
+                        }
+                        ptx::tma_load_2d_pair(sB + stage * RG::B_TILE, xm, fb, kx, xr);
+                        if (++stage == NSTAGE) { stage = 0; phase ^= 1u; }
+                    }
+                }
+                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+                __syncwarp();
+                if (!ok) break;
+            }
+            if (lane == 0 && *abort_flag) {
+                ptx::st_remote_u32(peer_abort, 1u);
+                if (rank == 0) {
+                    for (int s = 0; s < NSTAGE; ++s) {
+                        const uint32_t par = (s < stage) ? phase : (phase ^ 1u);
+                        const long long t0 = clock64();
+                        while (!ptx::mbar_try_wait(&full_bar[s], par) && clock64() - t0 < p.wait_limit) {
+                        }
+                    }
+                } else {
+                    const long long t0 = clock64();
+                    while (clock64() - t0 < (1ll << 21)) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer (rank 0)
+        if (lane == 0 && rank == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t acc_phase = 0;
+            for (int u = cluster; u < total; u += nclusters) {
+                const SwapUnit t = unit(u);
+                const uint32_t idesc = ptx::instr_desc(2 * TC_BM, (t.rows + 15) & ~15, kFp8 ? 0u : 1u);
+                bool ok = ptx::mbar_wait_cluster(&tempty_bar, acc_phase ^ 1u, abort_flag, p.wait_limit, p.status, 2u);
+                if (!ok) break;
+                ptx::tc_fence_after();
+                for (int kb = 0; kb < p.k_blocks; ++kb) {
+                    if (!ptx::mbar_wait(&full_bar[stage], phase, abort_flag, p.wait_limit, p.status, 3u)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    const uint32_t a_addr = ptx::smem_u32(sA + stage * RG::A_TILE);
+                    const uint32_t b_addr = ptx::smem_u32(sB + stage * RG::B_TILE);
+#pragma unroll
+                    for (int k = 0; k < KSTEPS; ++k) {
+                        const uint64_t bd = ptx::smem_desc_sw<kRowB>(b_addr + k * 32);
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) {
+                            const uint64_t ad = ptx::smem_desc_sw<kRowB>(a_addr + j * RG::A_SUB + k * 32);
+                            const uint32_t dj = tmem_base + static_cast<uint32_t>(j * 256);
+                            if constexpr (kFp8) ptx::mma_f8_pair(dj, ad, bd, idesc, (kb | k) != 0);
+                            else ptx::mma_f16_pair(dj, ad, bd, idesc, (kb | k) != 0);
+                        }
+                    }
+                    ptx::mma_commit_pair(&empty_bar[stage], 0x3);
+                    if (++stage == NSTAGE) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                ptx::mma_commit_pair(&tfull_bar, 0x3);
+                acc_phase ^= 1u;
+            }
+            if (*abort_flag) ptx::st_remote_u32(peer_abort, 1u);
+            ptx::mma_commit_pair(&drain_bar, 0x3);
+        }
+        if (lane == 0) {
+            const long long t0 = clock64();
+            while (!ptx::mbar_try_wait(&drain_bar, 0) && clock64() - t0 < p.wait_limit) {
+            }
+        }
+    } else {
+        // ---------------------------------------------------------------- epilogue (both CTAs)
+        const int sub = warp & 3;
+        const int eg = (warp - 2) >> 2;
+        const uint32_t tempty0 = ptx::mapa(&tempty_bar, 0);
+        uint8_t* stage_w = sStage + (warp - 2) * 2048;
+        uint32_t acc_phase = 0;
+        for (int u = cluster; u < total; u += nclusters) {
+            const SwapUnit t = unit(u);
+            int ok = 0;
+            if (lane == 0) ok = ptx::mbar_wait(&tfull_bar, acc_phase, abort_flag, p.wait_limit, p.status, 4u);
+            ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+            if (!ok) {
+                if (lane == 0) ptx::st_remote_u32(peer_abort, 1u);
+                break;
+            }
+            ptx::tc_fence_after();
+            const int nch = (t.rows + 31) >> 5;
+            const int row_end = t.row0 + t.rows;
+            const uint32_t lanes = static_cast<uint32_t>(sub * 32) << 16;
+            const bool direct = t.e == p.direct_e;
+            if constexpr (kGemm1) {
+                const int col0 = t.n0 + static_cast<int>(rank) * TC_BM + sub * 32;   // h columns of this warp
+                float sg = 1.0f, su = 1.0f;
+                if constexpr (kFp8) {
+                    const float* s = p.col_scale + static_cast<size_t>(t.e) * 2 * p.I + col0 + lane;
+                    sg = s[0];
+                    su = s[p.I];
+                }
+#pragma unroll 1
+                for (int c = eg; c < nch; c += 2) {
+                    uint32_t g[32], v[32];
+                    ptx::tmem_ld_32x32b_x32(tmem_base + lanes + c * 32, g);
+                    ptx::tmem_ld_32x32b_x32(tmem_base + lanes + 256 + c * 32, v);
+                    float my_rs = 1.0f;
+                    if constexpr (kFp8) {
+                        const int r = c * 32 + lane;
+                        if (r < t.rows) my_rs = direct ? p.direct_scale[t.row0 - s_off[t.e] + r] : p.row_scale[t.row0 + r];
+                    }
+                    ptx::tmem_ld_wait(g);
+                    ptx::tmem_ld_wait(v);
+                    uint16_t o[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        float gi = __uint_as_float(g[i]), ui = __uint_as_float(v[i]);
+                        if constexpr (kFp8) {
+                            const float rs = __shfl_sync(0xFFFFFFFFu, my_rs, i);
+                            gi = gi * rs * sg;
+                            ui = ui * rs * su;
+                        }
+                        o[i] = bf16_bits(silu_f32(gi) * ui);
+                    }
+                    stage_store_t(stage_w, o, lane, p.out, p.out_ld, t.row0 + c * 32, row_end, col0);
+                }
+            } else {
+                const int col0 = t.n0 + eg * 256 + static_cast<int>(rank) * TC_BM + sub * 32;   // y columns
+                float sc = 1.0f;
+                if constexpr (kFp8) sc = p.col_scale[static_cast<size_t>(t.e) * p.H + col0 + lane];
+#pragma unroll 1
+                for (int c = 0; c < nch; ++c) {
+                    uint32_t v[32];
+                    ptx::tmem_ld_32x32b_x32(tmem_base + lanes + static_cast<uint32_t>(eg * 256) + c * 32, v);
+                    float my_rs = 1.0f;
+                    if constexpr (kFp8) {
+                        const int r = c * 32 + lane;
+                        if (r < t.rows) my_rs = p.row_scale[t.row0 + r];
+                    }
+                    ptx::tmem_ld_wait(v);
+                    uint16_t o[32];
+                    int my_k = 0;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        float a = __uint_as_float(v[i]);
+                        if constexpr (kFp8) a = a * __shfl_sync(0xFFFFFFFFu, my_rs, i) * sc;
+                        if (p.yexp != nullptr) {
+                            const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(a) & 0x7FFFFFFFu);
+                            const int k = f16_chunk_exp(__uint_as_float(m));
+                            if (lane == i) my_k = k;
+                            o[i] = f16_bits(a * exp2_int(-k));
+                        } else {
+                            o[i] = bf16_bits(a);
+                        }
+                    }
+                    const int r0 = t.row0 + c * 32;
+                    stage_store_t(stage_w, o, lane, p.out, p.out_ld, r0, row_end, col0);
+                    if (p.yexp != nullptr && r0 + lane < row_end)
+                        p.yexp[static_cast<size_t>(r0 + lane) * (p.H / 32) + col0 / 32] =
+                            static_cast<int8_t>(my_k);
+                }
+            }
+            ptx::tc_fence_before();
+            ptx::mbar_arrive_remote(tempty0);
+            acc_phase ^= 1u;
+        }
+    }
+
+    __syncwarp();
+    ptx::tc_fence_before();
+    ptx::cluster_sync();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc_pair(tmem_base, TC_TMEM_COLS);
+    }
+}
+
 // ------------------------------------------------------------------ host side
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -855,6 +1222,35 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtens
     return cudaGetLastError();
 }
 
+// tokens as N on CTA pairs: sized like launch_pair
+template <bool kFp8, bool kGemm1>
+cudaError_t launch_swap(const CUtensorMap& w, const CUtensorMap& x, const CUtensorMap& x2, const TcParams& p,
+                        cudaStream_t st, const char* name) {
+    constexpr int kRowB = SRE_STAGE_ROW_BYTES;
+    constexpr int smem = RingS<kRowB>::SMEM;
+    auto kern = grouped_gemm_swap_kernel<kFp8, kGemm1, kRowB>;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    static int clusters = 0;
+    std::call_once(once, [kern] {
+        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (attr_err != cudaSuccess) return;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(num_sms() & ~1), 1, 1);
+        cfg.blockDim = dim3(320, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        int n = 0;
+        attr_err = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+        clusters = n;
+        if (attr_err == cudaSuccess && n < 1) attr_err = cudaErrorNotSupported;
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    ProfileScope ps(name, st);
+    kern<<<2 * clusters, 320, smem, st>>>(w, x, x2, p);
+    note_launch();
+    return cudaGetLastError();
+}
+
 template <bool kFp8, bool kPair>
 cudaError_t launch_gemm1(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2, const TcParams& p,
                          int half, cudaStream_t st) {
@@ -919,12 +1315,17 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
     // prefill_bf16 GEMM1 + GEMM2 1.86 ms with pair tiles vs 1.91 ms with
     // single-CTA 256-row units; E4M3 layers and small groups are faster on
     // single-CTA 128-row units (prefill_fp8 4.95 vs 6.29 ms per layer).
+    // cta_pair == 3: tokens as the MMA's N dimension (grouped_gemm_swap_kernel)
+    // where the widths divide (GEMM1: I % 256, GEMM2: H % 512), else as 2.
+    // cta_pair == 4 (the default for large bf16 groups): GEMM1 as 3, GEMM2 as 2.
     const bool big_bf16 = a.w_dtype == MOE_BF16 && a.R >= 192 * a.E;
-    const int cta_pair = a.cta_pair >= 0 ? a.cta_pair : ((a.unit_rows == 0 && big_bf16) ? 2 : 0);
+    const int cta_pair = a.cta_pair >= 0 ? a.cta_pair : ((a.unit_rows == 0 && big_bf16) ? 4 : 0);
     const bool two_sm = cta_pair > 0;
-    const bool wide1 = cta_pair == 2 && half == 128 && a.I % 256 == 0;
-    const bool wide2 = cta_pair == 2 && a.H % 512 == 0;
-    const int bn1 = wide1 ? 2 * half : half;     // h columns per unit
+    const bool swap1 = (cta_pair == 3 || cta_pair == 4) && a.I % 256 == 0;
+    const bool swap2 = cta_pair == 3 && a.H % 512 == 0;
+    const bool wide1 = cta_pair >= 2 && half == 128 && a.I % 256 == 0;
+    const bool wide2 = cta_pair >= 2 && a.H % 512 == 0;
+    const int bn1 = wide1 ? 2 * half : half;     // h columns per unit (swap: 256 as well)
 
     // GEMM1: A = Xp [R, H] (rows gathered by the gather kernel); B = W13 viewed as
     // [2E][I][H] (gate/up halves separately clipped at I)
@@ -935,7 +1336,9 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
         const cuuint64_t bd[3] = {static_cast<cuuint64_t>(a.H), static_cast<cuuint64_t>(a.I),
                                   static_cast<cuuint64_t>(2 * a.E)};
         const cuuint64_t bs[2] = {static_cast<cuuint64_t>(a.H) * esz, static_cast<cuuint64_t>(a.I) * a.H * esz};
-        if (!make_map(&ta, xp, fp8, 2, ad, as, TC_BM, kRowBytes) || !make_map(&tb, a.w13, fp8, 3, bd, bs, bn1, kRowBytes))
+        // swap: each CTA stages 128 gate and 128 up rows of the 256 h columns
+        if (!make_map(&ta, xp, fp8, 2, ad, as, TC_BM, kRowBytes) ||
+            !make_map(&tb, a.w13, fp8, 3, bd, bs, swap1 ? TC_BM : bn1, kRowBytes))
             return cudaErrorInvalidValue;
     }
     // the direct group's A: the token matrix [T, H]
@@ -957,6 +1360,7 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
     p.out_ld = a.I;
     p.row_scale = fp8 ? xp_scale : nullptr;
     p.direct_e = direct_e;
+    p.first_e = a.perm != nullptr ? a.direct_e : -1;
     p.direct_scale = fp8 ? a.xt_scale : nullptr;
     p.col_scale = fp8 ? a.s13 : nullptr;
     p.yexp = nullptr;
@@ -968,7 +1372,10 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
     // 128-row units, prefill_fp8 4.95 vs 6.04 ms, skewed_fp8 0.84 vs 0.99 ms)
     const bool pair = a.unit_rows == 256;
     cudaError_t err;
-    if (two_sm)
+    if (swap1)
+        err = fp8 ? launch_swap<true, true>(tb, ta, ta2, p, st, "gemm1_tc")
+                  : launch_swap<false, true>(tb, ta, ta2, p, st, "gemm1_tc");
+    else if (two_sm)
         err = fp8 ? launch_gemm1_pair<true>(ta, tb, ta2, p, half, wide1, st)
                   : launch_gemm1_pair<false>(ta, tb, ta2, p, half, wide1, st);
     else
@@ -1004,6 +1411,9 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
     p.direct_e = -1;
     p.col_scale = fp8 ? a.s2 : nullptr;
     p.yexp = a.yexp;
+    if (swap2)
+        return fp8 ? launch_swap<true, false>(tb, ta, ta, p, st, "gemm2_tc")
+                   : launch_swap<false, false>(tb, ta, ta, p, st, "gemm2_tc");
     if (wide2)
         return fp8 ? launch_pair<true, false, 256, 2>(ta, tb, ta, p, st, "gemm2_tc")
                    : launch_pair<false, false, 256, 2>(ta, tb, ta, p, st, "gemm2_tc");

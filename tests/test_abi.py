@@ -84,7 +84,7 @@ def test_forward_rejects_bad_arguments_on_the_host(L):
     assert call(x=FAKE + 8) == _lib.MOE_ERR_INVALID_ARG           # not 16-byte aligned
     assert call(ws=FAKE + 16) == _lib.MOE_ERR_INVALID_ARG         # workspace not 256-aligned
     assert call(ws_bytes=n - 1) == _lib.MOE_ERR_WORKSPACE
-    assert call(impl=7) == _lib.MOE_ERR_INVALID_ARG
+    assert call(impl=8) == _lib.MOE_ERR_INVALID_ARG
     s0 = _shape(shared_id=-1)
     assert f(C.byref(s0), FAKE, FAKE, None, FAKE, None, FAKE, None, 0, FAKE, FAKE, 1 << 30, 0,
              None) == _lib.MOE_ERR_INVALID_ARG                   # unfused needs a shared expert

@@ -13,11 +13,12 @@ from tests.parity_util import rel_err, to_f64, tol_of
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("impl", [_lib.MOE_FFN_AUTO, _lib.MOE_FFN_TCGEN05_PAIR, _lib.MOE_FFN_TCGEN05_WIDE],
-                         ids=["auto", "cta_pair", "cta_pair_wide"])
-def test_wait_timeout_is_reported_and_the_context_survives(impl):
+@pytest.mark.parametrize("impl,I", [(_lib.MOE_FFN_AUTO, 128), (_lib.MOE_FFN_TCGEN05_PAIR, 128),
+                                    (_lib.MOE_FFN_TCGEN05_WIDE, 128), (_lib.MOE_FFN_TCGEN05_SWAP, 256)],
+                         ids=["auto", "cta_pair", "cta_pair_wide", "cta_pair_swap"])
+def test_wait_timeout_is_reported_and_the_context_survives(impl, I):
     build.build()
-    cfg = synth.variant(synth.CONFIGS["prefill_bf16"], T=64, H=512, I=128, n_routed=8, top_k=2)
+    cfg = synth.variant(synth.CONFIGS["prefill_bf16"], T=64, H=512, I=I, n_routed=8, top_k=2)
     inp = synth.make_inputs(cfg)
     d = synth.to_device(inp, "cuda")
     layer = MoELayer(cfg, d, impl=impl)

@@ -11,7 +11,7 @@ import oracle
 from shared_routed_expert_b200 import _lib, build, synth
 from shared_routed_expert_b200._lib import (MOE_FFN_SIMT, MOE_FFN_TCGEN05, MOE_FFN_TCGEN05_M128,
                                             MOE_FFN_TCGEN05_M256, MOE_FFN_TCGEN05_PAIR,
-                                            MOE_FFN_TCGEN05_WIDE)
+                                            MOE_FFN_TCGEN05_SWAP, MOE_FFN_TCGEN05_WIDE)
 from tests.parity_util import oracle_logits, rel_err, to_f64, tol_of
 
 pytestmark = pytest.mark.gpu
@@ -169,8 +169,41 @@ FFN_CASES = {
 }
 
 
-IMPLS = [MOE_FFN_SIMT, MOE_FFN_TCGEN05_M128, MOE_FFN_TCGEN05_M256, MOE_FFN_TCGEN05_PAIR, MOE_FFN_TCGEN05_WIDE]
-IMPL_IDS = ["simt", "tcgen05_m128", "tcgen05_m256", "tcgen05_pair", "tcgen05_wide"]
+IMPLS = [MOE_FFN_SIMT, MOE_FFN_TCGEN05_M128, MOE_FFN_TCGEN05_M256, MOE_FFN_TCGEN05_PAIR, MOE_FFN_TCGEN05_WIDE,
+         MOE_FFN_TCGEN05_SWAP]
+IMPL_IDS = ["simt", "tcgen05_m128", "tcgen05_m256", "tcgen05_pair", "tcgen05_wide", "tcgen05_swap"]
+
+
+@pytest.mark.parametrize("w", ["bf16", "e4m3"])
+@pytest.mark.parametrize("impl", [MOE_FFN_TCGEN05_SWAP, MOE_FFN_TCGEN05_WIDE], ids=["swap", "wide"])
+def test_grouped_ffn_group_sizes_at_the_unit_limits(w, impl):
+    """Groups of 1, 15, 16, 17, 255, 256, 257, 300 and 513 rows (top-1 routing
+    plus the shared expert, whose group holds all 1630 tokens): with tokens as
+    the MMA's N dimension a group of c rows is cut into ceil(c / 256) units of
+    equal size rounded up to 16 rows; every row against the oracle."""
+    sizes = [1, 15, 16, 17, 255, 256, 257, 300, 513]
+    base = synth.CONFIGS["prefill_bf16" if w == "bf16" else "prefill_fp8"]
+    T = sum(sizes)
+    cfg = synth.variant(base, T=T, H=512, I=256, n_routed=len(sizes), top_k=1)
+    inp = synth.make_inputs(cfg)
+    d = synth.to_device(inp, DEV)
+    rng = np.random.default_rng(11)
+    routed = rng.permutation(np.repeat(np.arange(len(sizes)), sizes))
+    ids = np.stack([routed, np.full(T, cfg.shared_id)], 1).astype(np.int32)
+    counts, offsets, perm, inv = oracle.permute(ids, cfg.n_experts)
+    assert list(counts[:len(sizes)]) == sizes
+    s = _lib.make_shape(cfg)
+    ws = _lib.alloc_workspace(s, True)
+    S = cfg.slots
+    y = torch.empty(T * S, cfg.H, dtype=d["x"].dtype, device=DEV)
+    _lib.moe_grouped_ffn(s, d["x"], torch.from_numpy(perm).to(DEV), torch.from_numpy(offsets).to(DEV),
+                         d["w13"], d["s13"], d["w2"], d["s2"], y, ws, impl=impl)
+    torch.cuda.synchronize()
+    yg = to_f64(y)
+    Ly = oracle.Layer(cfg, inp)
+    xs = inp["x"].float().numpy()
+    ref = np.stack([Ly.expert_ffn(int(ids.ravel()[perm[r]]), xs[perm[r] // S]) for r in range(T * S)])
+    assert rel_err(yg, ref) <= tol_of(cfg)
 
 
 @pytest.mark.parametrize("name", list(FFN_CASES))

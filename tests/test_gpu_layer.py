@@ -67,7 +67,7 @@ def test_forward_simt_and_tensor_core_paths_agree(name):
     d = synth.to_device(synth.make_inputs(cfg), DEV)
     simt = _run(cfg, d, True, MOE_FFN_SIMT)
     for impl in (_lib.MOE_FFN_TCGEN05_M128, _lib.MOE_FFN_TCGEN05_M256, _lib.MOE_FFN_TCGEN05_PAIR,
-                 _lib.MOE_FFN_TCGEN05_WIDE):
+                 _lib.MOE_FFN_TCGEN05_WIDE, _lib.MOE_FFN_TCGEN05_SWAP):
         assert rel_err(simt, _run(cfg, d, True, impl)) <= tol_of(cfg)
 
 

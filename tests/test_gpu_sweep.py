@@ -3,7 +3,8 @@ oracle: token counts with ragged tails, hidden and intermediate sizes the
 tensor-core tiles divide differently, expert counts from 1 to 48, top-k from 1
 to 8, bf16 and E4M3 weights, routed scaling factors and selection-only bias,
 fused and unfused, and every GEMM variant (the CUDA-core one, single-CTA 128-
-and 256-row units, CTA pairs with 256 x 256 and 256 x 512 tiles). Each case
+and 256-row units, CTA pairs with 256 x 256 and 256 x 512 tiles, and CTA pairs
+with the tokens as the MMA's N dimension). Each case
 compares every output and the routing of every token."""
 import numpy as np
 import pytest
@@ -17,7 +18,7 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 IMPLS = [_lib.MOE_FFN_AUTO, _lib.MOE_FFN_SIMT, _lib.MOE_FFN_TCGEN05_M128, _lib.MOE_FFN_TCGEN05_M256,
-         _lib.MOE_FFN_TCGEN05_PAIR, _lib.MOE_FFN_TCGEN05_WIDE]
+         _lib.MOE_FFN_TCGEN05_PAIR, _lib.MOE_FFN_TCGEN05_WIDE, _lib.MOE_FFN_TCGEN05_SWAP]
 
 
 def _case(seed: int):
