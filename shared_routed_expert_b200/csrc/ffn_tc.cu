@@ -830,7 +830,11 @@ __device__ __forceinline__ void stage_store_t(uint8_t* slice, const uint16_t (&v
 }
 
 __device__ __forceinline__ uint16_t bf16_bits(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
-__device__ __forceinline__ uint16_t f16_bits(float x) { return __half_as_ushort(__float2half_rn(x)); }
+
+// 12 epilogue warps (three per TMEM lane group): TMEM holds one unit, so the
+// epilogue is not overlapped with MMAs and its length is paid in full
+constexpr int SW_EPI_WARPS = 12;
+constexpr int SW_THREADS = (2 + SW_EPI_WARPS) * 32;
 
 template <int kRowB>
 struct RingS {
@@ -839,18 +843,23 @@ struct RingS {
     static constexpr int B_TILE = 128 * kRowB;          // this CTA's token rows (N / 2 <= 128)
     static constexpr int STAGE = A_TILE + B_TILE;
     static constexpr int N = (TC_RING_BYTES / STAGE) > 8 ? 8 : (TC_RING_BYTES / STAGE);
-    static constexpr int SMEM = N * STAGE + 8 * 2048 + 1024;
+    static constexpr int SMEM = N * STAGE + SW_EPI_WARPS * 2048 + 1024;
 };
 
+// silu(g) = g / (1 + e^-g) with the hardware's approximate reciprocal (a few
+// ulp; e^-g = inf gives 0) instead of an IEEE division
+__device__ __forceinline__ float silu_fast(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
+
 template <bool kFp8, bool kGemm1, int kRowB>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SW_THREADS, 1)
     grouped_gemm_swap_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                              const __grid_constant__ CUtensorMap tmX2, const TcParams p) {
     using RG = RingS<kRowB>;
     constexpr int NSTAGE = RG::N;
     constexpr int KEL = kFp8 ? kRowB : kRowB / 2;
     constexpr int KSTEPS = kRowB / 32;
-    constexpr int EPI_WARPS = 8;
+    constexpr int EPI_WARPS = SW_EPI_WARPS;
+    constexpr int EG = EPI_WARPS / 4;           // epilogue warps per TMEM lane group
 
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t full_bar[NSTAGE], empty_bar[NSTAGE], tfull_bar, tempty_bar, drain_bar;
@@ -1023,7 +1032,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
     } else {
         // ---------------------------------------------------------------- epilogue (both CTAs)
         const int sub = warp & 3;
-        const int eg = (warp - 2) >> 2;
+        const int eg = (warp - 2) >> 2;          // 0 .. EG-1
         const uint32_t tempty0 = ptx::mapa(&tempty_bar, 0);
         uint8_t* stage_w = sStage + (warp - 2) * 2048;
         uint32_t acc_phase = 0;
@@ -1050,7 +1059,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
                     su = s[p.I];
                 }
 #pragma unroll 1
-                for (int c = eg; c < nch; c += 2) {
+                for (int c = eg; c < nch; c += EG) {
                     uint32_t g[32], v[32];
                     ptx::tmem_ld_32x32b_x32(tmem_base + lanes + c * 32, g);
                     ptx::tmem_ld_32x32b_x32(tmem_base + lanes + 256 + c * 32, v);
@@ -1070,44 +1079,79 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
                             gi = gi * rs * sg;
                             ui = ui * rs * su;
                         }
-                        o[i] = bf16_bits(silu_f32(gi) * ui);
+                        o[i] = bf16_bits(silu_fast(gi) * ui);
                     }
                     stage_store_t(stage_w, o, lane, p.out, p.out_ld, t.row0 + c * 32, row_end, col0);
                 }
             } else {
-                const int col0 = t.n0 + eg * 256 + static_cast<int>(rank) * TC_BM + sub * 32;   // y columns
-                float sc = 1.0f;
-                if constexpr (kFp8) sc = p.col_scale[static_cast<size_t>(t.e) * p.H + col0 + lane];
+                // Each 32-token chunk goes through the warp's slice as fp32 in two
+                // halves of 16 tokens: written one token row (128 bytes) per
+                // instruction, 16-byte chunks XOR-swizzled by row & 7; read back with
+                // two lanes per row, 16 columns each, so that the chunk exponent is a
+                // max over 16 registers and one shuffle.
 #pragma unroll 1
-                for (int c = 0; c < nch; ++c) {
+                for (int q = eg; q < 2 * nch; q += EG) {
+                    const int j = q & 1, c = q >> 1;     // sub-tile, 32-token chunk
+                    const int col0 = t.n0 + j * 256 + static_cast<int>(rank) * TC_BM + sub * 32;   // y columns
+                    float sc = 1.0f;
+                    if constexpr (kFp8) sc = p.col_scale[static_cast<size_t>(t.e) * p.H + col0 + lane];
                     uint32_t v[32];
-                    ptx::tmem_ld_32x32b_x32(tmem_base + lanes + static_cast<uint32_t>(eg * 256) + c * 32, v);
-                    float my_rs = 1.0f;
-                    if constexpr (kFp8) {
-                        const int r = c * 32 + lane;
-                        if (r < t.rows) my_rs = p.row_scale[t.row0 + r];
-                    }
+                    ptx::tmem_ld_32x32b_x32(tmem_base + lanes + static_cast<uint32_t>(j * 256) + c * 32, v);
                     ptx::tmem_ld_wait(v);
-                    uint16_t o[32];
-                    int my_k = 0;
+                    const int r = lane >> 1, hh = lane & 1;      // read side: row, column half
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        float a = __uint_as_float(v[i]);
-                        if constexpr (kFp8) a = a * __shfl_sync(0xFFFFFFFFu, my_rs, i) * sc;
+                    for (int h2 = 0; h2 < 2; ++h2) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            float a = __uint_as_float(v[h2 * 16 + i]);
+                            if constexpr (kFp8) a *= sc;
+                            *reinterpret_cast<float*>(stage_w + i * 128 + (((lane >> 2) ^ (i & 7)) << 4) +
+                                                      (lane & 3) * 4) = a;
+                        }
+                        __syncwarp();
+                        float a[16];
+#pragma unroll
+                        for (int k4 = 0; k4 < 4; ++k4) {
+                            const float4 w4 = *reinterpret_cast<const float4*>(
+                                stage_w + r * 128 + (((hh * 4 + k4) ^ (r & 7)) << 4));
+                            a[4 * k4] = w4.x;
+                            a[4 * k4 + 1] = w4.y;
+                            a[4 * k4 + 2] = w4.z;
+                            a[4 * k4 + 3] = w4.w;
+                        }
+                        __syncwarp();
+                        const int rr = c * 32 + h2 * 16 + r;     // row within the unit
+                        const bool valid = rr < t.rows;
+                        if constexpr (kFp8) {
+                            const float rs = valid ? p.row_scale[t.row0 + rr] : 0.0f;
+#pragma unroll
+                            for (int k = 0; k < 16; ++k) a[k] *= rs;
+                        }
+                        uint32_t pk[8];
+                        int kexp = 0;
                         if (p.yexp != nullptr) {
-                            const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(a) & 0x7FFFFFFFu);
-                            const int k = f16_chunk_exp(__uint_as_float(m));
-                            if (lane == i) my_k = k;
-                            o[i] = f16_bits(a * exp2_int(-k));
+                            float amax = 0.0f;
+#pragma unroll
+                            for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(a[k]));
+                            amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+                            kexp = f16_chunk_exp(amax);
+                            const float down = exp2_int(-kexp);
+#pragma unroll
+                            for (int k = 0; k < 16; k += 2) pk[k >> 1] = pack_f16x2(a[k] * down, a[k + 1] * down);
                         } else {
-                            o[i] = bf16_bits(a);
+#pragma unroll
+                            for (int k = 0; k < 16; k += 2) pk[k >> 1] = pack_bf16x2(a[k], a[k + 1]);
+                        }
+                        if (valid) {
+                            uint4* dst = reinterpret_cast<uint4*>(
+                                p.out + static_cast<size_t>(t.row0 + rr) * p.out_ld + col0 + hh * 16);
+                            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                            if (p.yexp != nullptr && hh == 0)
+                                p.yexp[static_cast<size_t>(t.row0 + rr) * (p.H / 32) + col0 / 32] =
+                                    static_cast<int8_t>(kexp);
                         }
                     }
-                    const int r0 = t.row0 + c * 32;
-                    stage_store_t(stage_w, o, lane, p.out, p.out_ld, r0, row_end, col0);
-                    if (p.yexp != nullptr && r0 + lane < row_end)
-                        p.yexp[static_cast<size_t>(r0 + lane) * (p.H / 32) + col0 / 32] =
-                            static_cast<int8_t>(my_k);
                 }
             }
             ptx::tc_fence_before();
@@ -1237,7 +1281,7 @@ cudaError_t launch_swap(const CUtensorMap& w, const CUtensorMap& x, const CUtens
         if (attr_err != cudaSuccess) return;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(static_cast<unsigned>(num_sms() & ~1), 1, 1);
-        cfg.blockDim = dim3(320, 1, 1);
+        cfg.blockDim = dim3(SW_THREADS, 1, 1);
         cfg.dynamicSmemBytes = smem;
         int n = 0;
         attr_err = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
@@ -1246,7 +1290,7 @@ cudaError_t launch_swap(const CUtensorMap& w, const CUtensorMap& x, const CUtens
     });
     if (attr_err != cudaSuccess) return attr_err;
     ProfileScope ps(name, st);
-    kern<<<2 * clusters, 320, smem, st>>>(w, x, x2, p);
+    kern<<<2 * clusters, SW_THREADS, smem, st>>>(w, x, x2, p);
     note_launch();
     return cudaGetLastError();
 }
