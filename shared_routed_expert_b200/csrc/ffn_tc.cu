@@ -765,7 +765,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
 // rows of one expert (N, a multiple of 16, half staged by each CTA). A group
 // of c rows is cut into ceil(c / 256) units of equal size rounded up to 16
 // rows, so a routed group of ~205 rows costs 208 rows of MMA work instead of a
-// 256-row M tile. TMEM lane = output feature, column = token.
+// 256-row M tile. The group scheduled first (the shared expert's, every token)
+// is cut into units of the routed groups' mean size (16-row multiple in
+// [192, 256]) so that all units cost about the same. TMEM lane = output
+// feature, column = token.
 //   GEMM1: sub-tile 0 = gate rows n0 + 128 r .. +127 of W13[e] (CTA rank r),
 //          sub-tile 1 = the up rows of the same h columns; accumulators in
 //          TMEM columns 0 and 256; every epilogue warp reads both and applies
@@ -783,8 +786,8 @@ struct SwapUnit {
     int e, row0, rows, n0;
 };
 
-__device__ __forceinline__ SwapUnit decode_swap(int id, const int* s_unit, const int* s_off, int E, int NT,
-                                                int bn_out) {
+__device__ __forceinline__ SwapUnit decode_swap(int id, const int* s_unit, const int* s_off, const int* s_rpu,
+                                                int E, int NT, int bn_out) {
     int lo = 0, hi = E - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -796,7 +799,7 @@ __device__ __forceinline__ SwapUnit decode_swap(int id, const int* s_unit, const
     const int nt = local / nu;
     const int mu = local - nt * nu;
     const int count = s_off[e + 1] - s_off[e];
-    const int rpu = ((count + nu - 1) / nu + 15) & ~15;      // <= 256 since nu = ceil(count / 256)
+    const int rpu = s_rpu[e];                                 // rows per unit, <= 256
     SwapUnit t;
     t.e = e;
     t.row0 = s_off[e] + mu * rpu;
@@ -865,7 +868,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SW_THREADS, 1)
     __shared__ uint64_t full_bar[NSTAGE], empty_bar[NSTAGE], tfull_bar, tempty_bar, drain_bar;
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
-    __shared__ int s_off[TC_MAXE], s_unit[TC_MAXE];
+    __shared__ int s_off[TC_MAXE], s_unit[TC_MAXE], s_rpu[TC_MAXE];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = ptx::cluster_ctarank();
@@ -880,11 +883,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SW_THREADS, 1)
 
     for (int i = threadIdx.x; i <= p.E; i += blockDim.x) s_off[i] = p.offsets[i];
     if (warp == 0) {
-        // prefix of units per expert: ceil(count / 256) = pairs of 128-row tiles
+        // units per expert and their rows: ceil(count / 256) units of equal size
+        // rounded up to 16 rows; the first-scheduled group in units of the other
+        // groups' mean size
+        int target = 256;
+        if (p.first_e >= 0 && p.E > 1) {
+            const int cf = p.offsets[p.first_e + 1] - p.offsets[p.first_e];
+            const int mean = (p.offsets[p.E] - cf) / (p.E - 1);
+            target = min(256, max(192, (mean + 15) & ~15));
+        }
         int carry = 0;
         for (int e0 = 0; e0 <= p.E; e0 += 32) {
             const int e = e0 + lane;
-            const int units = (e < p.E) ? (p.tile_off[e + 1] - p.tile_off[e] + 1) >> 1 : 0;
+            int units = 0;
+            if (e < p.E) {
+                const int c = p.offsets[e + 1] - p.offsets[e];
+                int rpu;
+                if (e == p.first_e) {
+                    units = (c + target - 1) / target;
+                    rpu = target;
+                } else {
+                    units = (c + 255) >> 8;
+                    rpu = units ? (((c + units - 1) / units + 15) & ~15) : 0;
+                }
+                s_rpu[e] = rpu;
+            }
             int inc = units;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
@@ -923,7 +946,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SW_THREADS, 1)
     const int rot = p.first_e >= 0 ? s_unit[p.first_e] * p.n_tiles_n : 0;
     auto unit = [&](int u) {
         const int v = u + rot;
-        return decode_swap(v < total ? v : v - total, s_unit, s_off, p.E, p.n_tiles_n, p.bn_out);
+        return decode_swap(v < total ? v : v - total, s_unit, s_off, s_rpu, p.E, p.n_tiles_n, p.bn_out);
     };
 
     if (warp == 0) {

@@ -61,6 +61,20 @@ def test_forward_small_matches_oracle(name):
     assert rel_err(fused, unfused) <= tol_of(cfg)
 
 
+@pytest.mark.parametrize("T,K,E_r", [(1000, 1, 8), (1500, 2, 12), (700, 8, 16)])
+def test_shared_group_units_of_the_routed_mean_size(T, K, E_r):
+    """With the tokens as the MMA's N dimension the shared expert's group (all T
+    rows, scheduled first) is cut into units of the routed groups' mean size,
+    a 16-row multiple clamped to [192, 256], the last unit ragged: T = 1000 with
+    mean 125 gives 5 units of 192 and one of 40; the others 256-row units."""
+    cfg = synth.variant(synth.CONFIGS["prefill_bf16"], T=T, H=512, I=256, n_routed=E_r, top_k=K)
+    inp = synth.make_inputs(cfg)
+    d = synth.to_device(inp, DEV)
+    ref = oracle.Layer(cfg, inp).forward()
+    for impl in (_lib.MOE_FFN_TCGEN05_SWAP, MOE_FFN_AUTO):
+        assert rel_err(_run(cfg, d, True, impl), ref["out"]) <= tol_of(cfg)
+
+
 @pytest.mark.parametrize("name", ["bf16_small", "fp8_small"])
 def test_forward_simt_and_tensor_core_paths_agree(name):
     cfg = SMALL[name]
