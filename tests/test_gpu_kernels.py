@@ -34,6 +34,11 @@ ROUTE_CASES = {
     "bias_select_only": synth.variant(synth.CONFIGS["skewed_fp8"], T=257, I=64, bias_select_only=True),
     "bias_select_full_softmax": synth.variant(synth.CONFIGS["skewed_fp8"], T=100, I=64, bias_select_only=True,
                                               renormalize=False, routed_scale=0.5),
+    # batches over 256 tokens take the wide tile (64 tokens x 160 experts per block):
+    # fp32 activations, a second expert block (200 experts), ragged token tiles
+    "fp32_wide_E200": synth.variant(synth.CONFIGS["tiny_fp32"], T=301, H=512, I=64, n_routed=200, top_k=4),
+    "bf16_wide_E200": synth.variant(synth.CONFIGS["prefill_bf16"], T=1000, H=1024, I=64, n_routed=200,
+                                    top_k=8),
 }
 
 
