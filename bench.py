@@ -554,20 +554,30 @@ def main():
         raise SystemExit(f"layer reported {_lib.status_string(st)}")
 
     if args.quick:
-        ms_unf = ms_e2e = float("nan")
+        ms_unf = ms_e2e = ms_fused_il = float("nan")
+        unf_steps = args.steps
         tab_unf = {}
         x_host = out_host = d["x"]
     else:
-        # unfused GPU baseline (shared expert as its own dense pass), same process
+        # unfused GPU baseline (shared expert as its own dense pass), same process,
+        # timed in blocks interleaved with blocks of the fused layer so that both
+        # see the same clocks (the power cap moves them by several percent over
+        # a run); per-kernel events on during the unfused blocks only
         unfused = MoELayer(cfg, d, fuse_shared=False, impl=impl)
         for _ in range(args.warmup):
             unfused.forward(d["x"], out)
         torch.cuda.synchronize()
         _lib.moe_profile_reset()
-        _lib.moe_profile_enable(True)
-        ms_unf = time_steps(lambda: unfused.forward(d["x"], out), args.steps, 0, dist, stream)
-        _lib.moe_profile_enable(False)
-        tab_unf = kernel_table(args.steps)
+        n_blocks = max(1, min(10, args.steps))
+        per = max(1, args.steps // n_blocks)
+        ms_unf = ms_fused_il = 0.0
+        for _ in range(n_blocks):
+            ms_fused_il += time_steps(step, per, 0, dist, stream)
+            _lib.moe_profile_enable(True)
+            ms_unf += time_steps(lambda: unfused.forward(d["x"], out), per, 0, dist, stream)
+            _lib.moe_profile_enable(False)
+        tab_unf = kernel_table(n_blocks * per)
+        unf_steps = n_blocks * per
         del unfused
 
         # end to end through the public API with pinned host buffers: every step
@@ -625,9 +635,11 @@ def main():
         "tensor_frac": flops / (ms_step / 1000.0) / 1e12 / tensor_peak,
         "hbm_gbs": alg_bytes / (ms_step / 1000.0) / 1e9,
         "hbm_frac": alg_bytes / (ms_step / 1000.0) / 1e9 / pk["hbm_gbs"],
-        "unfused": {"value": N * cfg.T * args.steps / (ms_unf / 1000.0), "ms_per_step": ms_unf / args.steps,
-                    "fused_speedup": ms_unf / ms,
-                    "kernels": {k: {"launches": v["launches"], "ms_per_step": v["total_ms"] / args.steps}
+        "unfused": {"value": N * cfg.T * unf_steps / (ms_unf / 1000.0), "ms_per_step": ms_unf / unf_steps,
+                    "fused_ms_per_step_interleaved": ms_fused_il / unf_steps,
+                    "fused_speedup": ms_unf / ms_fused_il,
+                    "timing": f"{n_blocks} blocks of {per} steps, fused and unfused alternating",
+                    "kernels": {k: {"launches": v["launches"], "ms_per_step": v["total_ms"] / unf_steps}
                                 for k, v in tab_unf.items()}},
         "e2e": {"value": N * cfg.T * args.steps / (ms_e2e / 1000.0), "unit": "tokens/s",
                 "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),

@@ -43,3 +43,21 @@ def test_throttle_reasons_are_named():
     import bench
     assert set(bench.Clocks.NAMES) == {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
                                        "sw_power_cap"}
+
+
+def test_work_unit_and_traffic_ratio_of_each_gemm():
+    """The tensor-core work unit bench.py attributes to each GEMM (it keys the
+    ncu traffic ratio): on the bf16 bench workload GEMM1 takes the tokens-as-N
+    kernel and GEMM2 the 256 x 512 pair tiles; E4M3 and small batches take
+    single-CTA 128-row units; a forced kernel choice wins."""
+    import bench
+    from shared_routed_expert_b200 import synth
+    bf16, fp8, dec = (synth.CONFIGS[n] for n in ("prefill_bf16", "prefill_fp8", "decode_bf16"))
+    assert bench.unit_rows(bf16, "auto", "gemm1_tc") == "swap"
+    assert bench.unit_rows(bf16, "auto", "gemm2_tc") == "pair256x512"
+    assert bench.unit_rows(fp8, "auto", "gemm1_tc") == 128
+    assert bench.unit_rows(dec, "auto", "gemm1_tc") == 128
+    assert bench.unit_rows(bf16, "tcgen05_wide", "gemm1_tc") == "pair256x512"
+    assert bench.unit_rows(bf16, "tcgen05_m256", "gemm2_tc") == 256
+    r = bench.PROFILED_TRAFFIC_RATIO
+    assert r[("gemm1_tc", "bf16", "swap")] == 1.013 and r[("gemm2_tc", "bf16", "pair256x512")] == 0.97
