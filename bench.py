@@ -556,6 +556,7 @@ def main():
     if args.quick:
         ms_unf = ms_e2e = ms_fused_il = float("nan")
         unf_steps = args.steps
+        n_blocks, per = 0, 0
         tab_unf = {}
         x_host = out_host = d["x"]
     else:
