@@ -251,7 +251,7 @@ def algorithmic(cfg, kernel: str, counts: np.ndarray | None):
 # Keyed by (kernel, weight dtype, tensor-core work unit).
 PROFILED_TRAFFIC_RATIO = {("gemm1_tc", "bf16", 256): 1.09,
                           ("gemm1_tc", "bf16", "pair256x512"): 1.02, ("gemm2_tc", "bf16", "pair256x512"): 0.97,
-                          ("gemm1_tc", "bf16", "swap"): 1.013}
+                          ("gemm1_tc", "bf16", "swap"): 1.008}
 
 
 def unit_rows(cfg, ffn: str, kernel: str = "gemm1_tc"):
