@@ -16,8 +16,9 @@
 // per-output-channel weight scales applied in the epilogue (they factor out of
 // the K-sum).
 //
-// CTA layout (320 threads): warp 0 = TMA producer, warp 1 = TMEM allocator and
-// single-thread MMA issuer, warps 2-9 = epilogue (warp w reads TMEM lanes
+// CTA layout (320 threads; 448 in grouped_gemm_swap_kernel, whose 12 epilogue
+// warps are described there): warp 0 = TMA producer, warp 1 = TMEM allocator
+// and single-thread MMA issuer, warps 2-9 = epilogue (warp w reads TMEM lanes
 // 32*(w%4)..+31; two warps per lane group split the columns or, for 256-row
 // units, take one accumulator each). Stages hold 128 bytes of K per row (64
 // bf16 or 128 E4M3 values) of the A tile(s) and of an N-row B tile, written by
@@ -772,13 +773,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
 //   GEMM1: sub-tile 0 = gate rows n0 + 128 r .. +127 of W13[e] (CTA rank r),
 //          sub-tile 1 = the up rows of the same h columns; accumulators in
 //          TMEM columns 0 and 256; every epilogue warp reads both and applies
-//          SwiGLU, the two warps of a lane group taking alternate 32-token chunks.
-//   GEMM2: sub-tile j = output columns n0 + 256 j + 128 r .. +127; warps 2-5
-//          drain sub-tile 0 and warps 6-9 sub-tile 1. A scaled-fp16 chunk (32
-//          output columns of one row) is one warp's 32 lanes: its exponent comes
-//          from a warp max-reduction per token.
+//          SwiGLU, the three warps of a lane group taking every third
+//          32-token chunk, written out transposed through the warp's slice.
+//   GEMM2: sub-tile j = output columns n0 + 256 j + 128 r .. +127; the three
+//          warps of a lane group share the chunks of both sub-tiles. A
+//          scaled-fp16 chunk (32 output columns of one row) lies across one
+//          warp's 32 lanes, so each block goes through the slice as fp32 and is
+//          read back two lanes per row before its exponent is taken.
 // Both sub-tiles of a stage share the token tile. TMEM is full, so the next
-// unit's MMAs wait for the epilogue of this one. The pair protocol (rank 0
+// unit's MMAs wait for the epilogue of this one (12 epilogue warps keep it
+// short). The pair protocol (rank 0
 // arms and issues, commits multicast to both CTAs, epilogues arrive on rank
 // 0's barrier, bounded waits and abort) is that of grouped_gemm_pair_kernel.
 
