@@ -147,6 +147,38 @@ def test_quant_rows_e4m3_bit_exact():
     assert np.array_equal(codes.cpu().numpy(), rc)
 
 
+def test_quant_rows_e4m3_midpoints_bit_exact():
+    """Rows whose quotients v / scale fall exactly on E4M3 rounding midpoints (and
+    one bf16 step either side): amax = 448 * m with m = 1.5, 1.25, 1.75 makes the
+    scale m exactly, and every midpoint of E4M3's normal range times m is a bf16
+    value. A reciprocal-multiply lands a rounding ulp off such a tie; the codes
+    must still be those of the IEEE divide (ties to even)."""
+    def bf16(a):
+        return torch.tensor(a, dtype=torch.float32).to(torch.bfloat16)
+    rows = []
+    for m in (1.5, 1.25, 1.75):
+        mids = [(1.0 + (2 * k + 1) / 16.0) * 2.0 ** e for e in range(-6, 9) for k in range(8)]
+        v = bf16([x * m for x in mids])
+        assert torch.equal(v.float(), torch.tensor([x * m for x in mids]))     # exact in bf16
+        up = (v.view(torch.int16) + 1).view(torch.bfloat16)
+        dn = (v.view(torch.int16) - 1).view(torch.bfloat16)
+        vals = torch.cat([v, up, dn, -v, -up, -dn, bf16([448.0 * m])])
+        vals = vals[vals.float().abs() <= 448.0 * m]
+        row = torch.zeros(1536, dtype=torch.bfloat16)
+        row[:vals.numel()] = vals
+        rows.append(row)
+    rows = torch.stack(rows)
+    n = rows.shape[0]
+    codes = torch.empty(n, 1536, dtype=torch.uint8, device=DEV)
+    scales = torch.empty(n, dtype=torch.float32, device=DEV)
+    _lib.moe_quant_rows_e4m3(n, 1536, rows.to(DEV), codes, scales)
+    torch.cuda.synchronize()
+    rc, rs = oracle.quant_rows_e4m3(rows.float().numpy())
+    assert np.array_equal(scales.cpu().numpy(), np.array([1.5, 1.25, 1.75], np.float32))
+    assert np.array_equal(scales.cpu().numpy().view(np.uint32), rs.view(np.uint32))
+    assert np.array_equal(codes.cpu().numpy(), rc)
+
+
 @pytest.mark.parametrize("act", ["bf16", "f32"])
 def test_combine_matches_oracle(act):
     T, S, H = 77, 9, 512
