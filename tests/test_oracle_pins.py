@@ -546,3 +546,69 @@ def test_intermediate_slices_sum_to_the_layer(world):
     parts = [oracle.Layer(tp.local_config(cfg, world), tp.shard_weights(inp, cfg.I, r, world))
              .forward(n_threads=2)["out"] for r in range(world)]
     assert np.allclose(sum(parts), full, rtol=1e-12, atol=1e-14)
+
+
+# ------------------------------------------------------------------ E4M3 exactness case
+
+def _e4m3_codes(values: torch.Tensor) -> torch.Tensor:
+    """Codes of values that lie on the E4M3 grid (checked by the round trip)."""
+    c = values.float().to(torch.float8_e4m3fn)
+    assert torch.equal(c.float(), values.float()), "value off the E4M3 grid"
+    return c.view(torch.uint8)
+
+
+def test_e4m3_layer_equals_bf16_layer_when_every_quantisation_is_lossless():
+    """Weights on the E4M3 grid with power-of-two channel scales, tokens whose
+    amax / 448 is a power of two, and an FFN whose h rows are +-amax * 2^-p: then
+    every quantisation the E4M3 layer performs (x per token, h per row) is exact,
+    and the layer must equal the bf16-weight layer on the dequantised weights bit
+    for bit. Gate rows read x_0 = 56 only (silu(56) = 56 in fp64), up rows read
+    x_1 only, so h_j = 56 * x_1 * d_j."""
+    T, H, I, E_r = 4, 256, 64, 2
+    f8 = synth.variant(synth.CONFIGS["prefill_fp8"], T=T, H=H, I=I, n_routed=E_r, top_k=1)
+    b16 = synth.variant(synth.CONFIGS["prefill_bf16"], T=T, H=H, I=I, n_routed=E_r, top_k=1)
+    E = f8.n_experts
+    g = torch.Generator().manual_seed(11)
+    grid = torch.tensor([0.0, 0.25, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])     # E4M3 values
+    # x: x_0 = 56 = 448 * 2^-3 is each token's amax, so its scale is 2^-3
+    x = grid[torch.randint(0, len(grid), (T, H), generator=g)] * 0.125
+    x = x * torch.where(torch.rand(T, H, generator=g) < 0.5, -1.0, 1.0)
+    x[:, 0] = 56.0
+    x[:, 1] = torch.tensor([0.5, 1.0, 2.0, 0.25])
+    x[:, 2] = torch.tensor([0.125, 0.125, -0.125, -0.125])   # routes tokens 0, 1 -> 0 and 2, 3 -> 1
+    router_w = torch.zeros(E_r, H)
+    router_w[0, 2], router_w[1, 2] = 1.0, -1.0
+    # weights as E4M3 values times power-of-two channel scales
+    w13 = torch.zeros(E, 2 * I, H)
+    s13 = torch.zeros(E, 2 * I)
+    w2 = grid[torch.randint(0, len(grid), (E, H, I), generator=g)] * 0.5
+    w2 = w2 * torch.where(torch.rand(E, H, I, generator=g) < 0.5, -1.0, 1.0)
+    s2 = torch.pow(2.0, torch.randint(-9, -5, (E, H), generator=g).float())
+    for e in range(E):
+        w13[e, :I, 0] = 256.0                          # gate_j = 256 * 2^-8 * x_0 = 56
+        s13[e, :I] = 2.0 ** -8
+        p = torch.randint(0, 6, (I,), generator=g)     # d_j = +-2^-p, max |d| = 1
+        p[0] = 0
+        sign = torch.where(torch.rand(I, generator=g) < 0.5, -1.0, 1.0)
+        w13[e, I:, 1] = sign * torch.pow(2.0, -p.float()) * 64.0
+        s13[e, I:] = 2.0 ** -6
+    inp8 = synth.make_inputs(f8)
+    inp8.update(x=x.to(torch.bfloat16), router_w=router_w, w13=_e4m3_codes(w13), s13=s13,
+                w2=_e4m3_codes(w2), s2=s2)
+    inp16 = synth.make_inputs(b16)
+    deq13 = w13 * s13[:, :, None]
+    deq2 = w2 * s2[:, :, None]
+    assert torch.equal(deq13.to(torch.bfloat16).float(), deq13) and torch.equal(deq2.to(torch.bfloat16).float(), deq2)
+    inp16.update(x=x.to(torch.bfloat16), router_w=inp8["router_w"], router_bias=inp8["router_bias"],
+                 w13=deq13.to(torch.bfloat16), w2=deq2.to(torch.bfloat16))
+    r8 = oracle.Layer(f8, inp8).forward(n_threads=2)
+    r16 = oracle.Layer(b16, inp16).forward(n_threads=2)
+    assert np.array_equal(r8["ids"], r16["ids"])
+    assert np.any(r8["out"] != 0.0)
+    assert np.array_equal(r8["out"], r16["out"])
+    assert r8["ids"][:, 0].tolist() == [0, 0, 1, 1]          # both routed experts in use
+    # one up-row scale of the shared expert (used by every token) off by 2: not equal
+    inp8["s13"] = s13.clone()
+    inp8["s13"][E_r, I + 3] *= 2.0
+    r8b = oracle.Layer(f8, inp8).forward(n_threads=2)
+    assert not np.array_equal(r8b["out"], r16["out"])
