@@ -326,8 +326,17 @@ def cpu_baseline(cfg, host_inputs: dict, seconds: float = 12.0):
         dt += time.perf_counter() - t1
         done += more
         used = max(used, r["threads"])
-    return {"value": done / dt, "unit": "tokens/s", "cores": used, "kind": "oracle",
-            "sample": f"{done} tokens of {cfg.name} (router + all {cfg.slots} slots each, fp64 C oracle), {dt:.1f} s"}
+    out = {"value": done / dt, "unit": "tokens/s", "cores": used, "kind": "oracle",
+           "sample": f"{done} tokens of {cfg.name} (router + all {cfg.slots} slots each, fp64 C oracle), {dt:.1f} s"}
+    if cfg.T <= 64:
+        # small batches are also timed on one core: up to 8 tokens, once
+        tok1 = rng.choice(cfg.T, size=min(8, cfg.T), replace=False).astype(np.int32)
+        t1 = time.perf_counter()
+        Ly.forward(tokens=tok1, n_threads=1)
+        dt1 = time.perf_counter() - t1
+        out["single_thread"] = {"value": len(tok1) / dt1, "unit": "tokens/s", "cores": 1,
+                                "sample": f"{len(tok1)} tokens of {cfg.name}, {dt1:.2f} s"}
+    return out
 
 
 def run_reference(args, dist: Dist):

@@ -61,3 +61,14 @@ def test_work_unit_and_traffic_ratio_of_each_gemm():
     assert bench.unit_rows(bf16, "tcgen05_m256", "gemm2_tc") == 256
     r = bench.PROFILED_TRAFFIC_RATIO
     assert r[("gemm1_tc", "bf16", "swap")] == 1.008 and r[("gemm2_tc", "bf16", "pair256x512")] == 0.97
+
+
+def test_cpu_baseline_times_the_oracle_and_small_batches_on_one_core():
+    """The CPU baseline runs the oracle on a token sample with all host cores;
+    batches of <= 64 tokens are also timed on one core."""
+    import bench
+    from shared_routed_expert_b200 import synth
+    cfg = synth.CONFIGS["tiny_fp32"]
+    r = bench.cpu_baseline(cfg, synth.make_inputs(cfg), seconds=0.2)
+    assert r["kind"] == "oracle" and r["unit"] == "tokens/s" and r["value"] > 0 and r["cores"] >= 1
+    assert r["single_thread"]["cores"] == 1 and r["single_thread"]["value"] > 0
