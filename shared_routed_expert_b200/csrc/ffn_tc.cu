@@ -431,7 +431,7 @@ __global__ void __launch_bounds__(320, 1)
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
             const TileInfo t = decode_unit<kPair>(tile, s_unit, s_off, p.E, p.n_tiles_n, p.bn_out);
-            // one lane waits, the warp follows its verdict: tcgen05.ld below needs the whole warp
+            // one lane waits and the warp takes its result: tcgen05.ld below needs the whole warp
             int ok = 0;
             if (lane == 0) ok = ptx::mbar_wait(&tfull_bar[acc], acc_phase, abort_flag, p.wait_limit, p.status, 4u);
             ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
