@@ -72,3 +72,27 @@ def test_cpu_baseline_times_the_oracle_and_small_batches_on_one_core():
     r = bench.cpu_baseline(cfg, synth.make_inputs(cfg), seconds=0.2)
     assert r["kind"] == "oracle" and r["unit"] == "tokens/s" and r["value"] > 0 and r["cores"] >= 1
     assert r["single_thread"]["cores"] == 1 and r["single_thread"]["value"] > 0
+
+
+def test_roofline_of_gemm1_on_the_bf16_bench_workload():
+    """bench.py's roofline entry for GEMM1 of prefill_bf16 against the closed
+    forms: FLOPs 2 R 2I H, bytes = the touched experts' gate/up weights + the
+    gathered rows in + h out; with the measured peaks the launch sits on the HBM
+    side of the ridge (bytes / 6544 GB/s > FLOPs / sustained bf16 peak)."""
+    import numpy as np
+    import bench
+    from shared_routed_expert_b200 import synth
+    cfg = synth.CONFIGS["prefill_bf16"]
+    R, H, I, E = cfg.rows, cfg.H, cfg.I, cfg.n_experts
+    counts = np.full(E, R // E)
+    fl, nb = bench.algorithmic(cfg, "gemm1_tc", counts)
+    assert fl == 2 * R * 2 * I * H
+    assert nb == E * 2 * I * H * 2 + R * H * 2 + R * I * 2
+    pk = {"hbm_gbs": 6544.0, "bf16_tflops": 1414.4, "source": "measured"}
+    ms = 1.0
+    r = bench.roofline_of(cfg, "gemm1_tc", ms, counts, pk, "auto")
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["peak"] == 6544.0
+    assert abs(r["achieved"] - nb / 1e-3 / 1e9) < 1e-6 * r["achieved"]
+    assert abs(r["frac"] - r["achieved"] / 6544.0) < 1e-12
+    assert r["traffic"] == int(1.008 * nb)                    # the tokens-as-N capture's ratio
+    assert abs(r["tensor_frac"] - fl / 1e-3 / 1e12 / 1414.4) < 1e-9
