@@ -29,18 +29,19 @@
  *      from +0 over ascending h; the segment sums are added in ascending
  *      segment order to a running fp32 total that starts at +0; the bias (if
  *      any) is added last in fp32.
- *   R5 permutation: experts in id order, inside an expert stable by the flat
+ *   R5 slot order in a token: slots 0..K-1 by R3, slot K the shared expert.
+ *   R6 permutation: experts in id order, inside an expert stable by the flat
  *      slot index t*S + k.
- *   R6 expert FFN (SwiGLU): w13[e] rows [0, I) = gate, [I, 2I) = up;
+ *   R7 expert FFN (SwiGLU): w13[e] rows [0, I) = gate, [I, 2I) = up;
  *      h = silu(gate . v) * (up . v), silu(g) = g / (1 + exp(-g));
  *      y = w2[e] . h.
- *   R7 roundings that are part of the layer's storage format: bf16 layers round
- *      h to bf16 and the output to bf16 once; E4M3 layers quantise x per token
- *      and h per (token, expert) row to E4M3 with scale = amax/448 computed in
- *      fp32, codes = E4M3_rn_satfinite(v / scale) with an fp32 divide, after h
- *      has been rounded to bf16. Everything else is fp64.
  *   R8 E4M3 is the OCP "E4M3FN" format: bias 7, no infinities, 0x7F/0xFF NaN,
- *      largest finite 448, smallest subnormal 2^-9.
+ *      largest finite 448, smallest subnormal 2^-9. E4M3 layers quantise x per
+ *      token and h per (token, expert) row with scale = amax/448 computed in
+ *      fp32, codes = E4M3_rn_satfinite(v / scale) with an fp32 divide, after h
+ *      has been rounded to bf16.
+ *   R9 roundings that are part of the layer's storage format: bf16 layers round
+ *      h to bf16 and the output to bf16 once. Everything else is fp64.
  *   R15 routed scaling factor s (the de/en pages, section 1, mention that the
  *      shared expert's weight needs special handling): the routed slots weigh
  *      s * softmax and the shared slot keeps shared_weight, the same sum as an
@@ -124,7 +125,7 @@ uint8_t orc_e4m3_encode(float vf) {
     return sign | code;
 }
 
-/* Per-row E4M3 quantisation (R7): scale = amax/448 in fp32 (amax = 0 -> 1),
+/* Per-row E4M3 quantisation (R8): scale = amax/448 in fp32 (amax = 0 -> 1),
  * codes = E4M3(v / scale) with an fp32 divide. */
 float orc_quant_row_e4m3(int n, const float* v, uint8_t* codes) {
     float amax = 0.0f;
@@ -266,7 +267,7 @@ void orc_qk_norm_rope(int T, int n_q, int n_kv, int d, int rot, float eps, const
 
 /* ---------------------------------------------------------------- permute */
 
-/* Counting sort of the R = T*S slots by expert, stable by flat index (R5).
+/* Counting sort of the R = T*S slots by expert, stable by flat index (R6).
  * perm[row] = flat slot index; inv[flat] = row; offsets has E+1 entries.
  * Returns -1 if an id is out of [0, E). */
 int orc_permute(int R, int E, const int32_t* ids, int32_t* counts, int32_t* offsets,
@@ -321,7 +322,7 @@ static double xval(const orc_layer* Ly, int t, int h) {
     return orc_bf16_to_double(((const uint16_t*)Ly->x)[i]);
 }
 
-/* One expert applied to one token (R6, R7). v: the token's activations as the
+/* One expert applied to one token (R7, R8, R9). v: the token's activations as the
  * layer stores them (fp32 values). Writes y[H] in fp64, unrounded.
  * scratch: at least 2I + H doubles + H floats + H + I bytes. */
 static void expert_ffn(const orc_layer* Ly, int e, const float* v, double* y, void* scratch) {
@@ -478,7 +479,7 @@ int orc_forward(const orc_layer* Ly, int n_tok, const int32_t* tok, int fuse_sha
     return n_threads;
 }
 
-/* Weighted combine given expert rows Y (R7's output rounding applied):
+/* Weighted combine given expert rows Y (R9's output rounding applied):
  * out[t] = sum_{k<S} w[t,k] * Y[inv[t*S+k]], fp64 in slot order. Y is fp32. */
 void orc_combine(int T, int S, int H, const float* Y, const int32_t* inv, const double* w,
                  int act_dtype, double* out) {
