@@ -118,3 +118,14 @@ def test_zero_tokens_is_a_no_op(L):
     assert L.moe_forward(C.byref(s), FAKE, FAKE, None, FAKE, None, FAKE, None, 1, FAKE, FAKE, n,
                          0, None) == _lib.MOE_OK
     assert L.moe_launch_count() == 0
+
+
+def test_a_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """No CPU path: without the built CUDA library every entry point raises
+    instead of computing anything."""
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "libsre_moe.so"))
+    with pytest.raises(ImportError):
+        _lib.lib()
+    with pytest.raises(ImportError):
+        _lib.moe_workspace_size(_shape(), True)
