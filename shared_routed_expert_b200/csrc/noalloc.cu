@@ -17,13 +17,19 @@
 // stand-in symbol, not a device address. The device address is looked up with
 // cudaGetSymbolAddress once per device, with that device current, on the first
 // call made on it (so make the first call outside any stream capture), and
-// cached.
+// cached together with the unique id of the CUDA context it belongs to. A
+// cudaDeviceReset ends that context and the module is loaded again in the next
+// one, where the array may sit at another address: a call that finds another
+// current context looks the address up again (and is then, again, a first
+// call).
 //
 // All calls share the array and it keeps the last call's contents. The status
 // word is cleared at the start of every call (report() needs it at zero); the
 // histograms are fully rewritten by each call. Calls that overlap on the GPU
 // (two streams, or two host threads) race on the array and give wrong results:
 // serialise them.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "kernels.cuh"
@@ -38,6 +44,32 @@ __device__ __align__(256) unsigned char g_permute_scratch[kNoAllocScratchBytes];
 
 std::mutex g_scratch_mu;
 void* g_scratch_addr[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxDevices] = {};  // unique id of the context the address belongs to
+
+// The driver's cuCtxGetCurrent and cuCtxGetId, looked up through the runtime
+// (the library links no driver library).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+template <typename Fn>
+Fn driver_fn(const char* name) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint(name, &ptr, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+        return nullptr;
+    return reinterpret_cast<Fn>(ptr);
+}
+
+// Unique id of the calling thread's current context (ids are never reused, unlike
+// context handles); 0 when no context is current or the driver calls are missing.
+unsigned long long current_context_id() {
+    static const CtxGetCurrentFn get = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+    static const CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (get == nullptr || get_id == nullptr || get(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+    if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
 
 cudaError_t scratch_address(void** out) {
     int dev = 0;
@@ -45,11 +77,15 @@ cudaError_t scratch_address(void** out) {
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lk(g_scratch_mu);
-    if (g_scratch_addr[dev] == nullptr) {
+    unsigned long long ctx = current_context_id();    // 0 before the runtime first used this thread
+    if (g_scratch_addr[dev] == nullptr || ctx == 0 || g_scratch_ctx[dev] != ctx) {
         void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_permute_scratch);
+        e = cudaGetSymbolAddress(&p, g_permute_scratch);    // makes the device's context current
         if (e != cudaSuccess) return e;
+        ctx = current_context_id();
+        if (ctx == 0) return cudaErrorInitializationError;
         g_scratch_addr[dev] = p;
+        g_scratch_ctx[dev] = ctx;
     }
     *out = g_scratch_addr[dev];
     return cudaSuccess;

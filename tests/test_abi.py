@@ -129,3 +129,30 @@ def test_a_missing_library_fails_loudly(monkeypatch, tmp_path):
         _lib.lib()
     with pytest.raises(ImportError):
         _lib.moe_workspace_size(_shape(), True)
+
+
+def _noalloc_bound(E: int) -> int:
+    """Largest ceil(T*S/512) * E the fixed scratch of moe_permute_noalloc holds:
+    1 MiB less the 256-byte status word and the (E+1)-int tile prefix rounded
+    up to 256 bytes, in ints."""
+    return (1048576 - 256 - (4 * (E + 1) + 255) // 256 * 256) // 4
+
+
+@pytest.mark.parametrize("E_r,K", [(40, 6), (160, 8), (191, 4), (256, 8)])
+def test_permute_noalloc_size_limit_is_exact(L, E_r, K):
+    """The host check of moe_permute_noalloc rejects exactly the batches whose
+    histograms do not fit its fixed array: at the bound the call gets past the
+    check (and, with no GPU here, fails in the CUDA runtime); one 512-slot chunk
+    more is MOE_ERR_UNSUPPORTED before any CUDA call."""
+    E, S = E_r + 1, K + 1
+    chunks = _noalloc_bound(E) // E
+    T_ok = chunks * 512 // S                  # ceil(T_ok * S / 512) == chunks
+    T_bad = T_ok + 1
+    assert -(-T_ok * S // 512) == chunks and -(-T_bad * S // 512) == chunks + 1
+    for T, want in ((T_ok, None), (T_bad, _lib.MOE_ERR_UNSUPPORTED)):
+        cfg = synth.variant(synth.CONFIGS["prefill_bf16"], T=T, H=256, I=64, n_routed=E_r, top_k=K)
+        rc = L.moe_permute_noalloc(C.byref(_lib.make_shape(cfg)), FAKE, FAKE, FAKE, FAKE, FAKE, None)
+        if want is None:
+            assert rc != _lib.MOE_ERR_UNSUPPORTED
+        else:
+            assert rc == want
