@@ -202,8 +202,7 @@ def time_steps(fn, steps: int, warmup: int, dist: Dist, stream) -> float:
 
 
 KERNELS = ["route_logits", "route_topk", "permute_small", "permute_hist", "permute_scan", "permute_scatter",
-           "quant_rows", "gather", "gemm1_tc", "gemm2_tc", "gemm1_simt", "gemm2_simt", "combine",
-           "round_out"]
+           "quant_x", "quant_h", "gather", "gemm1_tc", "gemm2_tc", "gemm1_simt", "gemm2_simt", "combine"]
 
 
 def kernel_table(steps: int) -> dict:
@@ -219,15 +218,17 @@ def kernel_table(steps: int) -> dict:
     return tab
 
 
-def algorithmic(cfg, kernel: str, counts: np.ndarray | None):
+def algorithmic(cfg, kernel: str, counts: np.ndarray | None, fused: bool = True):
     """(flops, bytes) one launch of `kernel` must do for this workload: flops of
     the dense contraction it performs (None if it is not one), and the bytes it
     must move at least once (touched experts' weights, its own inputs/outputs)."""
     R, T, H, I, Er = cfg.rows, cfg.T, cfg.H, cfg.I, cfg.n_routed
+    E = cfg.n_experts
     wb = 1 if cfg.w_dtype == "e4m3" else (4 if cfg.w_dtype == "f32" else 2)
     ab = 4 if cfg.act_dtype == "f32" else 2
     xb = 1 if wb == 1 else ab                      # bytes per GEMM input activation
     touched = int((counts > 0).sum()) if counts is not None else cfg.n_experts
+    n_chunks = -(-R // 512)                        # 512-slot chunks of the permutation
     if kernel.startswith("gemm1"):
         return 2.0 * R * 2 * I * H, touched * 2 * I * H * wb + R * H * xb + R * I * ab
     if kernel.startswith("gemm2"):
@@ -235,12 +236,30 @@ def algorithmic(cfg, kernel: str, counts: np.ndarray | None):
         return 2.0 * R * I * H, touched * H * I * wb + R * I * xb + R * H * 2 + R * (H // 32)
     if kernel == "route_logits":
         return None, T * H * ab + Er * H * 4 + (H // 256) * T * Er * 4
+    if kernel == "route_topk":
+        # the segment partials in; ids and weights out
+        return None, (H // 256) * T * Er * 4 + R * 8
     if kernel == "combine":
-        return None, R * H * ab + T * H * ab + R * 4 * 2
+        return None, R * H * 2 + R * (H // 32) + T * H * ab + R * 4 * 2
     if kernel == "gather":
-        return None, 2 * R * H * xb
-    if kernel == "round_out":
-        return None, T * H * (4 + ab)
+        # the fused layer's shared rows are read from x by GEMM1 and not copied:
+        # x read once, the routed rows written (plus per-row scales for E4M3)
+        copied = R - T if (fused and cfg.shared) else R
+        return None, T * H * xb + copied * H * xb + (copied * 4 + T * 4 if wb == 1 else 0)
+    if kernel == "quant_x":
+        # x per token (T rows of H): bf16 in, E4M3 codes and one scale per row out
+        return None, T * H * 3 + T * 4
+    if kernel == "quant_h":
+        # h per permuted row (R rows of I)
+        return None, R * I * 3 + R * 4
+    if kernel == "permute_small":
+        return None, R * 4 + 2 * R * 4 + (2 * E + 1) * 4
+    if kernel == "permute_hist":
+        return None, R * 4 + n_chunks * E * 4
+    if kernel == "permute_scan":
+        return None, 2 * n_chunks * E * 4 + 3 * (E + 1) * 4
+    if kernel == "permute_scatter":
+        return None, R * 4 + n_chunks * E * 4 + (E + 1) * 4 + 2 * R * 4
     return None, None
 
 
@@ -486,6 +505,8 @@ def main():
                     choices=["auto", "simt", "tcgen05", "tcgen05_m128", "tcgen05_m256", "tcgen05_pair",
                              "tcgen05_wide", "tcgen05_swap"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="time only --workload (by default the other workloads follow in a 'workloads' object)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--quick", action="store_true",
                     help="only the fused device-timed region (for ncu launch lists and captures)")
@@ -526,6 +547,68 @@ def main():
             "tcgen05_m128": _lib.MOE_FFN_TCGEN05_M128, "tcgen05_m256": _lib.MOE_FFN_TCGEN05_M256,
             "tcgen05_pair": _lib.MOE_FFN_TCGEN05_PAIR, "tcgen05_wide": _lib.MOE_FFN_TCGEN05_WIDE,
             "tcgen05_swap": _lib.MOE_FFN_TCGEN05_SWAP}[args.ffn]
+    N = dist.world
+    base = dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline
+    m = measure(cfg, args, dist, impl, quick=args.quick, want_host=base and not args.quick)
+    line = {
+        "metric": METRIC, "value": m["value"], "unit": "tokens/s", "n_gpus": N, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": m["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if cfg.w_dtype == "bf16" else cfg.w_dtype,
+        "data": "synthetic",
+        "config": {"workload": describe(cfg), "global_batch_tokens": N * cfg.T,
+                   "parallelism": f"replicas x{N} (tokens sharded, weights replicated)",
+                   "l2": "inputs larger than L2: every step streams the touched experts' weights "
+                         f"({m['alg_bytes'] / 1e9:.2f} GB) through the 126 MB L2",
+                   "ffn_impl": args.ffn},
+        "tflops": m["tflops"], "tensor_frac": m["tensor_frac"], "hbm_gbs": m["hbm_gbs"], "hbm_frac": m["hbm_frac"],
+        "fused_speedup": m["unfused"]["fused_speedup"],
+        "unfused": m["unfused"],
+        "combine_separate": m["combine_separate"],
+        "e2e": m["e2e"],
+        "gpu_launches": m["gpu_launches"],
+        "roofline": m["roofline"],
+        "kernels": m["kernels"],
+        "clocks": m["clocks"],
+        "peaks": m["peaks"],
+    }
+    if base and not args.quick:
+        line["cpu_baseline"] = cpu_baseline(cfg, m["host"], args.cpu_seconds)
+    m.pop("host", None)
+    # the other workloads of the layer, measured the same way in the same run
+    extra = [] if (args.quick or args.no_workloads) else [w for w in WORKLOADS if w != cfg.name]
+    if extra:
+        line["workloads"] = {}
+        for name in extra:
+            wcfg = synth.CONFIGS[name]
+            wm = measure(wcfg, args, dist, impl, quick=False, want_host=base and wcfg.T <= 64)
+            entry = {"workload": describe(wcfg), "value": wm["value"], "unit": "tokens/s",
+                     "ms_per_step": wm["ms_per_step"], "steps": args.steps,
+                     "tflops": wm["tflops"], "tensor_frac": wm["tensor_frac"], "hbm_gbs": wm["hbm_gbs"],
+                     "hbm_frac": wm["hbm_frac"], "roofline": wm["roofline"],
+                     "fused_speedup": wm["unfused"]["fused_speedup"], "unfused": wm["unfused"],
+                     "combine_separate": wm["combine_separate"],
+                     "e2e": wm["e2e"], "gpu_launches": wm["gpu_launches"], "clocks": wm["clocks"],
+                     "kernels": {k: {kk: v[kk] for kk in ("launches", "ms_per_launch", "share", "roofline")}
+                                 for k, v in wm["kernels"].items()}}
+            if base and wcfg.T <= 64:
+                entry["cpu_baseline"] = cpu_baseline(wcfg, wm["host"], args.cpu_seconds / 2)
+            wm.pop("host", None)
+            line["workloads"][name] = entry
+            del wm
+            torch.cuda.empty_cache()
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.close()
+
+
+WORKLOADS = ["prefill_bf16", "decode_bf16", "prefill_fp8", "skewed_fp8"]
+
+
+def measure(cfg, args, dist: Dist, impl: int, quick: bool = False, want_host: bool = False) -> dict:
+    """Everything one workload reports: the fused layer device-timed over
+    args.steps back-to-back steps (inputs resident in HBM, per-kernel events on
+    the launching stream), the unfused layer in interleaved blocks, and the end
+    to end path through host buffers."""
     d = synth.make_inputs(cfg, dist.device)
     stream = torch.cuda.current_stream(dist.device)
     fused = MoELayer(cfg, d, fuse_shared=True, impl=impl)
@@ -545,7 +628,6 @@ def main():
     vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
     clocks = Clocks(vis.split(",")[dist.local] if vis else str(dist.local))
     _lib.moe_profile_reset()
-    n0 = _lib.moe_launch_count()
     _lib.moe_profile_enable(True)
     for _ in range(args.warmup):
         step()
@@ -560,10 +642,10 @@ def main():
     tab = kernel_table(args.steps)
     st = fused.status()
     if st != _lib.MOE_OK:
-        raise SystemExit(f"layer reported {_lib.status_string(st)}")
+        raise SystemExit(f"{cfg.name}: layer reported {_lib.status_string(st)}")
 
-    if args.quick:
-        ms_unf = ms_e2e = ms_fused_il = float("nan")
+    if quick:
+        ms_unf = ms_e2e = ms_fused_il = ms_sep = float("nan")
         unf_steps = args.steps
         n_blocks, per = 0, 0
         tab_unf = {}
@@ -574,21 +656,30 @@ def main():
         # see the same clocks (the power cap moves them by several percent over
         # a run); per-kernel events on during the unfused blocks only
         unfused = MoELayer(cfg, d, fuse_shared=False, impl=impl)
+        # the fused layer with its weighted aggregation as a separate pass (the
+        # layout before the aggregation moved into the down-projection)
+        separate = MoELayer(cfg, d, fuse_shared=True, impl=impl | _lib.MOE_FFN_COMBINE_SEPARATE)
         for _ in range(args.warmup):
             unfused.forward(d["x"], out)
+            separate.forward(d["x"], out)
         torch.cuda.synchronize()
         _lib.moe_profile_reset()
         n_blocks = max(1, min(10, args.steps))
         per = max(1, args.steps // n_blocks)
-        ms_unf = ms_fused_il = 0.0
+        ms_unf = ms_fused_il = ms_sep = 0.0
         for _ in range(n_blocks):
             ms_fused_il += time_steps(step, per, 0, dist, stream)
             _lib.moe_profile_enable(True)
             ms_unf += time_steps(lambda: unfused.forward(d["x"], out), per, 0, dist, stream)
             _lib.moe_profile_enable(False)
+            ms_sep += time_steps(lambda: separate.forward(d["x"], out), per, 0, dist, stream)
         tab_unf = kernel_table(n_blocks * per)
         unf_steps = n_blocks * per
-        del unfused
+        for lay, what in ((unfused, "unfused"), (separate, "separate combine")):
+            st = lay.status()
+            if st != _lib.MOE_OK:
+                raise SystemExit(f"{cfg.name} {what}: layer reported {_lib.status_string(st)}")
+        del unfused, separate
 
         # end to end through the public API with pinned host buffers: every step
         # uploads its x and downloads its out; the pipelined submission overlaps
@@ -612,7 +703,6 @@ def main():
         out_host = out_hosts[0]
     N = dist.world
     ms_step = ms / args.steps
-    value = tokens_per_s(N, cfg.T, args.steps, ms)
     pk = peaks()
     flops = cfg.gemm_flops() + cfg.router_flops()
     wb = 1 if cfg.w_dtype == "e4m3" else 2
@@ -630,17 +720,9 @@ def main():
         roof = roofline_of(cfg, top, tab[top]["ms_per_launch"], counts, pk, args.ffn)
         for k in tab:
             tab[k]["roofline"] = roofline_of(cfg, k, tab[k]["ms_per_launch"], counts, pk, args.ffn)
-
-    line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": N, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16" if cfg.w_dtype == "bf16" else cfg.w_dtype,
-        "data": "synthetic",
-        "config": {"workload": describe(cfg), "global_batch_tokens": N * cfg.T,
-                   "parallelism": f"replicas x{N} (tokens sharded, weights replicated)",
-                   "l2": "inputs larger than L2: every step streams the touched experts' weights "
-                         f"({alg_bytes / 1e9:.2f} GB) through the 126 MB L2",
-                   "ffn_impl": args.ffn},
+    host = synth.to_host(d) if want_host else None
+    res = {
+        "value": tokens_per_s(N, cfg.T, args.steps, ms), "ms_per_step": ms_step, "alg_bytes": alg_bytes,
         "tflops": flops / (ms_step / 1000.0) / 1e12,
         "tensor_frac": flops / (ms_step / 1000.0) / 1e12 / tensor_peak,
         "hbm_gbs": alg_bytes / (ms_step / 1000.0) / 1e9,
@@ -651,20 +733,18 @@ def main():
                     "timing": f"{n_blocks} blocks of {per} steps, fused and unfused alternating",
                     "kernels": {k: {"launches": v["launches"], "ms_per_step": v["total_ms"] / unf_steps}
                                 for k, v in tab_unf.items()}},
+        "combine_separate": {"ms_per_step": ms_sep / unf_steps,
+                             "fold_speedup": ms_sep / ms_fused_il,
+                             "timing": "the fused layer with its aggregation as its own pass, in the same "
+                                       "alternating blocks"},
         "e2e": {"value": N * cfg.T * args.steps / (ms_e2e / 1000.0), "unit": "tokens/s",
                 "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
                 "d2h_bytes_per_step": out_host.numel() * out_host.element_size()},
-        "gpu_launches": int(launches),
-        "roofline": roof,
-        "kernels": tab,
-        "clocks": clk,
-        "peaks": pk,
+        "gpu_launches": int(launches), "roofline": roof, "kernels": tab, "clocks": clk, "peaks": pk,
+        "host": host,
     }
-    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline and not args.quick:
-        line["cpu_baseline"] = cpu_baseline(cfg, synth.to_host(d), args.cpu_seconds)
-    if dist.rank == 0:
-        print(json.dumps(line), flush=True)
-    dist.close()
+    del fused, d
+    return res
 
 
 if __name__ == "__main__":

@@ -96,3 +96,37 @@ def test_roofline_of_gemm1_on_the_bf16_bench_workload():
     assert abs(r["frac"] - r["achieved"] / 6544.0) < 1e-12
     assert r["traffic"] == int(1.008 * nb)                    # the tokens-as-N capture's ratio
     assert abs(r["tensor_frac"] - fl / 1e-3 / 1e12 / 1414.4) < 1e-9
+
+
+def test_every_timed_kernel_has_algorithmic_bytes():
+    """Each kernel the bench times gets the bytes it must move at least once,
+    so that no roofline entry is left without its numerator."""
+    import numpy as np
+    import bench
+    from shared_routed_expert_b200 import synth
+    for name in ("prefill_bf16", "prefill_fp8", "decode_bf16"):
+        cfg = synth.CONFIGS[name]
+        counts = np.full(cfg.n_experts, cfg.rows // cfg.n_experts)
+        for k in bench.KERNELS:
+            if k.endswith("_simt") and cfg.w_dtype != "f32":
+                continue
+            fl, nb = bench.algorithmic(cfg, k, counts)
+            assert nb is not None and nb > 0, (name, k)
+
+
+def test_gather_bytes_leave_out_the_shared_rows():
+    """The fused layer's gather copies only the routed rows (the shared
+    expert's rows are x itself, read by GEMM1): prefill_bf16 reads x once
+    (4096 x 5120 x 2 B) and writes 32768 routed rows of 10240 B = 377.5 MB; the
+    unfused layer has no shared rows in its grouped pass and copies all R."""
+    import bench
+    from shared_routed_expert_b200 import synth
+    cfg = synth.CONFIGS["prefill_bf16"]
+    _, nb = bench.algorithmic(cfg, "gather", None)
+    assert nb == 4096 * 5120 * 2 + 32768 * 5120 * 2 == 377_487_360
+    _, nb_u = bench.algorithmic(cfg, "gather", None, fused=False)
+    assert nb_u == 4096 * 5120 * 2 + cfg.rows * 5120 * 2
+    # E4M3: one byte per element plus the per-row scales
+    c8 = synth.CONFIGS["skewed_fp8"]
+    _, nb8 = bench.algorithmic(c8, "gather", None)
+    assert nb8 == 4096 * 5120 + 32768 * 5120 + 32768 * 4 + 4096 * 4
