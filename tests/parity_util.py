@@ -62,3 +62,33 @@ def sample_tokens(T: int, n: int, seed: int = 123) -> np.ndarray:
     while len(pick) < min(n, T):
         pick.add(int(rng.integers(0, T)))
     return np.array(sorted(pick), dtype=np.int32)
+
+
+def full_size_sample(T: int, ids: np.ndarray, n_routed: int, n: int, unit: int = 208,
+                     seed: int = 321) -> np.ndarray:
+    """Tokens whose outputs a full-size parity test checks, chosen to cover the
+    work units of the grouped GEMMs: every `unit`-token block of the shared
+    expert's group (its rows are the tokens in order) gets at least one token
+    when n allows, and for each of the 10 largest routed groups the token of its
+    first row (first work unit), of its last row (last unit) and of the row
+    `unit` positions before its end; the rest are random tokens. All tokens
+    when n >= T."""
+    if n >= T:
+        return np.arange(T, dtype=np.int32)
+    pick = set()
+    counts = np.bincount(ids[:, :-1].ravel() if ids.shape[1] > 1 else ids.ravel(),
+                         minlength=n_routed)[:n_routed]
+    flat = ids.ravel()
+    S = ids.shape[1]
+    for e in np.argsort(-counts, kind="stable")[:10]:
+        rows = np.nonzero(flat == e)[0]             # the group's rows, in slot order
+        if rows.size:
+            for r in (rows[0], rows[-1], rows[max(0, rows.size - unit)]):
+                pick.add(int(r // S))
+    n_even = max(0, n - len(pick) - 8)
+    if n_even:
+        pick.update(int(t) for t in np.linspace(0, T - 1, n_even).round().astype(np.int64))
+    rng = np.random.default_rng(seed)
+    while len(pick) < min(n, T):
+        pick.add(int(rng.integers(0, T)))
+    return np.array(sorted(pick), dtype=np.int32)

@@ -81,6 +81,53 @@ def test_route_zero_router_ties_to_lowest_ids():
     assert np.allclose(w[:, :8], 0.125) and np.all(w[:, 8] == 1.0)
 
 
+@pytest.mark.parametrize("bias_select_only,n_neg_inf", [(False, 9), (True, 9), (False, 36), (True, 36)])
+def test_route_nonfinite_inputs_follow_the_oracle(bias_select_only, n_neg_inf):
+    """Non-finite router inputs (R3: NaN ranks as -inf, ties toward the lower
+    id): tokens with +inf, -inf, both, and NaN entries in x, and a bias that
+    sets some experts' keys to -inf. Ids must equal the oracle's bit for bit;
+    weights must be equal where the oracle's are finite and NaN where its are
+    NaN (a token whose selected weight logits are all -inf, or include +inf,
+    has no defined softmax); finite logits bit for bit, NaN logits at the same
+    places. With 36 of 40 keys at -inf a finite token selects its 4 finite
+    experts and then the two lowest -inf ids, which weigh 0 (or, with the bias
+    for selection only, the softmax of their unbiased logits)."""
+    cfg = synth.variant(synth.CONFIGS["prefill_bf16"], T=64, H=512, I=64, n_routed=40, top_k=6,
+                        bias_select_only=bias_select_only)
+    inp = synth.make_inputs(cfg)
+    x = inp["x"]
+    x[1, 7] = float("inf")                       # logits +-inf by the sign of w[:, 7]
+    x[2, 300] = float("-inf")
+    x[3, 7] = float("inf")                       # +inf and -inf terms: NaN logits
+    x[3, 300] = float("-inf")
+    x[4, 0] = float("nan")                       # every logit NaN: ranks as -inf, ids 0..5
+    x[5, :] = float("inf")
+    bias = torch.zeros(cfg.n_routed, dtype=torch.float32)
+    neg = [0, 2, 3, 11, 17, 29, 30, 31, 39] if n_neg_inf == 9 else [e for e in range(40) if e not in (5, 8, 20, 33)]
+    bias[neg] = float("-inf")
+    bias[5] = 0.75
+    inp["router_bias"] = bias
+    d = synth.to_device(inp, DEV)
+    ids, w, L = _route(cfg, d)
+    Lr = oracle_logits(d["x"], d["router_w"], d["router_bias"])
+    nan = np.isnan(Lr)
+    assert nan[3].any() and nan[4].all() and nan[5].all() and (np.isinf(Lr[1]) | nan[1]).all()
+    assert np.array_equal(np.isnan(L), nan)
+    assert np.array_equal(L[~nan].view(np.uint32), Lr[~nan].view(np.uint32))
+    Lw = oracle_logits(d["x"], d["router_w"], None) if bias_select_only else None
+    rid, rw = oracle.topk(Lr, cfg.top_k, cfg.renormalize, cfg.shared_id, cfg.shared_weight,
+                          weight_logits=Lw, routed_scale=cfg.routed_scale)
+    assert np.array_equal(ids, rid)
+    assert np.array_equal(ids[4, :6], np.arange(6))        # all keys NaN: the lowest ids
+    assert np.array_equal(np.isnan(w), np.isnan(rw))
+    assert np.isnan(rw[4, :6]).all()
+    if n_neg_inf == 36:                                    # finite tokens: 4 finite keys, then ids 0, 1
+        assert np.array_equal(np.sort(rid[10, :4]), [5, 8, 20, 33]) and np.array_equal(rid[10, 4:6], [0, 1])
+        assert (rw[10, 4:6] > 0).all() if bias_select_only else (rw[10, 4:6] == 0).all()
+    fin = ~np.isnan(rw)
+    assert np.allclose(w[fin], rw[fin], rtol=2e-6, atol=1e-7)
+
+
 def _permute(cfg, ids_np):
     s = _lib.make_shape(cfg)
     ws = _lib.alloc_workspace(s, True)
