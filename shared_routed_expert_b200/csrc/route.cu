@@ -19,26 +19,25 @@ namespace sre {
 
 namespace {
 
-#ifndef SRE_RT_TPT
-#define SRE_RT_TPT 4           // tokens per thread: 4 or 8
-#endif
-#ifndef SRE_RT_MINB
-#define SRE_RT_MINB 2          // resident blocks per SM the register budget aims for
-#endif
-constexpr int RT_TPT = SRE_RT_TPT;
-constexpr int RT_BT = 16 * RT_TPT;     // tokens per block (16 token groups)
 constexpr int RT_EL = 16;      // expert lanes per block; a thread owns kEJ experts strided by RT_EL
 constexpr int RT_KC = 32;      // h per shared-memory chunk
 constexpr int RT_SEG = 256;    // segment length of the fixed order
-constexpr int RT_XP = RT_BT + 4;       // row pitch (floats) of the transposed x tile xs[k][t]
 constexpr int RT_WP = RT_KC + 4;       // row pitch (floats) of the w tile ws[e][k]: 144 B rows
-constexpr int RT_THREADS = 256;
 
-template <int kEJ>
-struct RouterSmem {
-    static constexpr int BE = RT_EL * kEJ;     // experts per block
-    float xs[2][RT_KC][RT_XP];
-    float ws[2][BE][RT_WP];
+// Block shape: kTY token groups x RT_EL expert lanes (kTY * 16 threads); thread
+// (ty, tx) owns kTPT tokens and kEJ experts, so a block covers kTY * kTPT tokens
+// and RT_EL * kEJ experts of one segment.
+template <int kTY, int kTPT, int kEJ>
+struct RouterTile {
+    static constexpr int THREADS = kTY * RT_EL;
+    static constexpr int BT = kTY * kTPT;          // tokens per block
+    static constexpr int BE = RT_EL * kEJ;         // experts per block
+    static constexpr int XP = BT + 4;              // row pitch (floats) of the transposed x tile xs[k][t]
+    static constexpr int XG = BT * RT_KC / 8 / THREADS;   // x pieces of 8 h per thread and chunk
+    struct Smem {
+        float xs[2][RT_KC][XP];
+        float ws[2][BE][RT_WP];
+    };
 };
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
@@ -51,38 +50,35 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 
 // w chunk: rows e0.. (kBE experts) x 32 h, copied as is into ws[e][k]
 // (16-byte pieces; rows past E are left unwritten: their results are never stored)
-template <int kBE>
+template <int kBE, int kThreads>
 __device__ __forceinline__ void issue_w_chunk(const float* wr, int E, int H, int e0, int h0,
                                               float (*ws)[RT_WP]) {
-    static_assert((kBE * RT_KC / 4) % RT_THREADS == 0, "whole pieces per thread");
+    static_assert((kBE * RT_KC / 4) % kThreads == 0, "whole pieces per thread");
 #pragma unroll
-    for (int i = 0; i < (kBE * RT_KC / 4) / RT_THREADS; ++i) {
-        const int piece = threadIdx.x + i * RT_THREADS;
+    for (int i = 0; i < (kBE * RT_KC / 4) / kThreads; ++i) {
+        const int piece = threadIdx.x + i * kThreads;
         const int e = piece >> 3, c = piece & 7;
         if (e0 + e < E) cp_async16(&ws[e][c * 4], wr + static_cast<size_t>(e0 + e) * H + h0 + c * 4);
     }
     cp_async_commit();
 }
 
-// x chunk: RT_BT tokens x 32 h in pieces of 8 h; piece p = thread + 256 g holds
-// token t0 + p % RT_BT, h h0 + 8 (p / RT_BT) .. +7
-constexpr int RT_XG = RT_BT * RT_KC / 8 / RT_THREADS;   // pieces per thread
-
 // The next chunk's x is held raw (bf16 pairs or fp32 bits) in registers while
-// the current chunk is multiplied, and converted when stored.
-template <bool kBf16>
+// the current chunk is multiplied, and converted when stored. Piece p = thread
+// + kThreads g holds token t0 + p % BT, h h0 + 8 (p / BT) .. +7.
+template <bool kBf16, int kXG>
 struct XStage {
-    static constexpr int N = RT_XG * (kBf16 ? 4 : 8);   // 32-bit words per thread
+    static constexpr int N = kXG * (kBf16 ? 4 : 8);   // 32-bit words per thread
     uint32_t w[N];
 };
 
-template <bool kBf16>
-__device__ __forceinline__ void load_x_chunk(const void* x, int T, int H, int t0, int h0, XStage<kBf16>& st) {
+template <bool kBf16, int kXG, int kBT, int kThreads>
+__device__ __forceinline__ void load_x_chunk(const void* x, int T, int H, int t0, int h0, XStage<kBf16, kXG>& st) {
 #pragma unroll
-    for (int g = 0; g < RT_XG; ++g) {
-        const int piece = threadIdx.x + g * RT_THREADS;
-        const int t = t0 + (piece & (RT_BT - 1));
-        const int q = (piece / RT_BT) * 8;
+    for (int g = 0; g < kXG; ++g) {
+        const int piece = threadIdx.x + g * kThreads;
+        const int t = t0 + (piece % kBT);
+        const int q = (piece / kBT) * 8;
         if constexpr (kBf16) {
             uint4 a = make_uint4(0u, 0u, 0u, 0u);
             if (t < T)
@@ -104,13 +100,13 @@ __device__ __forceinline__ void load_x_chunk(const void* x, int T, int H, int t0
 }
 
 // transposed into xs[k][t] as fp32 (bf16 -> fp32 is exact)
-template <bool kBf16>
-__device__ __forceinline__ void store_x_chunk(const XStage<kBf16>& st, float (*xs)[RT_XP]) {
+template <bool kBf16, int kXG, int kBT, int kThreads, int kXP>
+__device__ __forceinline__ void store_x_chunk(const XStage<kBf16, kXG>& st, float (*xs)[kXP]) {
 #pragma unroll
-    for (int g = 0; g < RT_XG; ++g) {
-        const int piece = threadIdx.x + g * RT_THREADS;
-        const int tl = piece & (RT_BT - 1);
-        const int q = (piece / RT_BT) * 8;
+    for (int g = 0; g < kXG; ++g) {
+        const int piece = threadIdx.x + g * kThreads;
+        const int tl = piece % kBT;
+        const int q = (piece / kBT) * 8;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             float v;
@@ -125,33 +121,35 @@ __device__ __forceinline__ void store_x_chunk(const XStage<kBf16>& st, float (*x
     }
 }
 
-// grid (ceil(T/RT_BT), ceil(E/160), H/256); 256 threads: thread (ty, tx) =
-// (threadIdx / 16, threadIdx % 16) owns tokens t0 + RT_TPT ty .. +RT_TPT-1 and
-// experts e0 + tx + 16 j (j < 10). P[s][t][e] = fma chain over the 256 h of segment s
-// (blockIdx.z), from +0, h ascending. The next chunk's copies are in flight
-// while this one is multiplied.
-template <bool kBf16, int kEJ>
-__global__ void __launch_bounds__(RT_THREADS, SRE_RT_MINB) router_segment_kernel(const void* __restrict__ x,
-                                                                       const float* __restrict__ wr,
-                                                                       float* __restrict__ P, int T, int H,
-                                                                       int E) {
+// grid (ceil(T/BT), ceil(E/BE), H/256): thread (ty, tx) = (threadIdx / 16,
+// threadIdx % 16) owns tokens t0 + kTPT ty .. +kTPT-1 and experts e0 + tx + 16 j
+// (j < kEJ). P[s][t][e] = fma chain over the 256 h of segment s (blockIdx.z),
+// from +0, h ascending. The next chunk's copies are in flight while this one is
+// multiplied.
+template <bool kBf16, int kTY, int kTPT, int kEJ, int kMinB>
+__global__ void __launch_bounds__(kTY * RT_EL, kMinB) router_segment_kernel(const void* __restrict__ x,
+                                                                          const float* __restrict__ wr,
+                                                                          float* __restrict__ P, int T, int H,
+                                                                          int E) {
+    using RT = RouterTile<kTY, kTPT, kEJ>;
+    constexpr int NT = RT::THREADS, BT = RT::BT, XP = RT::XP, XG = RT::XG;
     extern __shared__ __align__(16) uint8_t rt_smem[];
-    using Smem = RouterSmem<kEJ>;
+    using Smem = typename RT::Smem;
     Smem& sm = *reinterpret_cast<Smem*>(rt_smem);
-    const int t0 = blockIdx.x * RT_BT, e0 = blockIdx.y * Smem::BE, s = blockIdx.z;
+    const int t0 = blockIdx.x * BT, e0 = blockIdx.y * RT::BE, s = blockIdx.z;
     const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
 
-    float acc[RT_TPT][kEJ];
+    float acc[kTPT][kEJ];
 #pragma unroll
-    for (int a = 0; a < RT_TPT; ++a)
+    for (int a = 0; a < kTPT; ++a)
 #pragma unroll
         for (int j = 0; j < kEJ; ++j) acc[a][j] = 0.0f;
 
     constexpr int NCHUNK = RT_SEG / RT_KC;
-    XStage<kBf16> xnext;
-    issue_w_chunk<Smem::BE>(wr, E, H, e0, s * RT_SEG, sm.ws[0]);
-    load_x_chunk<kBf16>(x, T, H, t0, s * RT_SEG, xnext);
-    store_x_chunk<kBf16>(xnext, sm.xs[0]);
+    XStage<kBf16, XG> xnext;
+    issue_w_chunk<RT::BE, NT>(wr, E, H, e0, s * RT_SEG, sm.ws[0]);
+    load_x_chunk<kBf16, XG, BT, NT>(x, T, H, t0, s * RT_SEG, xnext);
+    store_x_chunk<kBf16, XG, BT, NT, XP>(xnext, sm.xs[0]);
     cp_async_wait_all();
     __syncthreads();
 
@@ -161,19 +159,21 @@ __global__ void __launch_bounds__(RT_THREADS, SRE_RT_MINB) router_segment_kernel
         const bool more = c + 1 < NCHUNK;
         if (more) {
             const int h1 = s * RT_SEG + (c + 1) * RT_KC;
-            issue_w_chunk<Smem::BE>(wr, E, H, e0, h1, sm.ws[buf ^ 1]);
-            load_x_chunk<kBf16>(x, T, H, t0, h1, xnext);
+            issue_w_chunk<RT::BE, NT>(wr, E, H, e0, h1, sm.ws[buf ^ 1]);
+            load_x_chunk<kBf16, XG, BT, NT>(x, T, H, t0, h1, xnext);
         }
-        const float (*xs)[RT_XP] = sm.xs[buf];
+        const float (*xs)[XP] = sm.xs[buf];
         const float (*ws)[RT_WP] = sm.ws[buf];
-#pragma unroll
+        // 8-token tiles: two k steps unrolled keep the operands within the register budget
+        constexpr int kUnroll = kTPT >= 8 ? 2 : RT_KC / 4;
+#pragma unroll kUnroll
         for (int k4 = 0; k4 < RT_KC; k4 += 4) {
-            float xv[RT_TPT][4];   // [token][k]
+            float xv[kTPT][4];   // [token][k]
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
 #pragma unroll
-                for (int a4 = 0; a4 < RT_TPT; a4 += 4) {
-                    const float4 v = *reinterpret_cast<const float4*>(&xs[k4 + kk][ty * RT_TPT + a4]);
+                for (int a4 = 0; a4 < kTPT; a4 += 4) {
+                    const float4 v = *reinterpret_cast<const float4*>(&xs[k4 + kk][ty * kTPT + a4]);
                     xv[a4][kk] = v.x; xv[a4 + 1][kk] = v.y; xv[a4 + 2][kk] = v.z; xv[a4 + 3][kk] = v.w;
                 }
             }
@@ -181,7 +181,7 @@ __global__ void __launch_bounds__(RT_THREADS, SRE_RT_MINB) router_segment_kernel
             for (int j = 0; j < kEJ; ++j) {
                 const float4 w = *reinterpret_cast<const float4*>(&ws[tx + RT_EL * j][k4]);
 #pragma unroll
-                for (int a = 0; a < RT_TPT; ++a) {
+                for (int a = 0; a < kTPT; ++a) {
                     float r = acc[a][j];
                     r = __fmaf_rn(xv[a][0], w.x, r);
                     r = __fmaf_rn(xv[a][1], w.y, r);
@@ -192,15 +192,15 @@ __global__ void __launch_bounds__(RT_THREADS, SRE_RT_MINB) router_segment_kernel
             }
         }
         if (more) {
-            store_x_chunk<kBf16>(xnext, sm.xs[buf ^ 1]);
+            store_x_chunk<kBf16, XG, BT, NT, XP>(xnext, sm.xs[buf ^ 1]);
             cp_async_wait_all();
         }
         __syncthreads();
     }
     float* out = P + static_cast<size_t>(s) * T * E;
 #pragma unroll
-    for (int a = 0; a < RT_TPT; ++a) {
-        const int t = t0 + ty * RT_TPT + a;
+    for (int a = 0; a < kTPT; ++a) {
+        const int t = t0 + ty * kTPT + a;
         if (t >= T) continue;
 #pragma unroll
         for (int j = 0; j < kEJ; ++j) {
@@ -323,26 +323,27 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ P, 
     }
 }
 
-template <int kEJ>
+template <int kTY, int kTPT, int kEJ, int kMinB>
 cudaError_t launch_router_segments(const moe_shape& s, const void* x, const float* wr, float* partials, int T,
                                    int H, int E, int split, cudaStream_t st) {
-    constexpr int smem = static_cast<int>(sizeof(RouterSmem<kEJ>));
+    using RT = RouterTile<kTY, kTPT, kEJ>;
+    constexpr int smem = static_cast<int>(sizeof(typename RT::Smem));
+    auto kb = router_segment_kernel<true, kTY, kTPT, kEJ, kMinB>;
+    auto kf = router_segment_kernel<false, kTY, kTPT, kEJ, kMinB>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(router_segment_kernel<true, kEJ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        smem);
+    std::call_once(once, [kb, kf] {
+        attr_err = cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (attr_err == cudaSuccess)
-            attr_err = cudaFuncSetAttribute(router_segment_kernel<false, kEJ>,
-                                            cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            attr_err = cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     });
     if (attr_err != cudaSuccess) return attr_err;
-    dim3 grid(ceil_div(T, RT_BT), ceil_div(E, RouterSmem<kEJ>::BE), split);
+    dim3 grid(ceil_div(T, RT::BT), ceil_div(E, RT::BE), split);
     ProfileScope ps("route_logits", st);
     if (s.act_dtype == MOE_BF16)
-        router_segment_kernel<true, kEJ><<<grid, RT_THREADS, smem, st>>>(x, wr, partials, T, H, E);
+        kb<<<grid, RT::THREADS, smem, st>>>(x, wr, partials, T, H, E);
     else
-        router_segment_kernel<false, kEJ><<<grid, RT_THREADS, smem, st>>>(x, wr, partials, T, H, E);
+        kf<<<grid, RT::THREADS, smem, st>>>(x, wr, partials, T, H, E);
     note_launch();
     return cudaGetLastError();
 }
@@ -364,9 +365,17 @@ cudaError_t launch_route(const moe_shape& s, const void* x, const float* wr, con
     const int T = s.T, H = s.H, E = s.n_routed;
     const int split = router_split_count(T, H);
     // small batches: 32 experts per block (5x the blocks at 160 routed experts)
-    const bool narrow = T <= 4 * RT_BT;
-    cudaError_t err = narrow ? launch_router_segments<2>(s, x, wr, partials, T, H, E, split, st)
-                             : launch_router_segments<10>(s, x, wr, partials, T, H, E, split, st);
+#ifndef SRE_RT_WIDE
+#define SRE_RT_WIDE 1
+#endif
+    const bool narrow = T <= 256;
+    cudaError_t err;
+    if (narrow)
+        err = launch_router_segments<16, 4, 2, 2>(s, x, wr, partials, T, H, E, split, st);
+    else if (SRE_RT_WIDE == 1)
+        err = launch_router_segments<8, 8, 10, 3>(s, x, wr, partials, T, H, E, split, st);
+    else
+        err = launch_router_segments<16, 4, 10, 2>(s, x, wr, partials, T, H, E, split, st);
     if (err != cudaSuccess) return err;
     {
         ProfileScope ps("route_topk", st);
