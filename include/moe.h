@@ -107,6 +107,15 @@ typedef enum moe_ffn_impl {
     MOE_FFN_TCGEN05_WIDE = 6, MOE_FFN_TCGEN05_SWAP = 7
 } moe_ffn_impl;
 
+/* Flag OR'ed into ffn_impl of moe_forward: run the weighted aggregation of the
+ * fused layer inside the down-projection's units of the shared expert instead
+ * of as its own pass over the stored expert rows (where the tensor-core
+ * down-projection runs, i.e. not with TCGEN05_SWAP or SIMT). The output is the
+ * same bit for bit either way. The separate pass is the default: measured on
+ * B200 it is faster (the in-kernel aggregation is bound by the loads a few
+ * epilogue warps can keep in flight). */
+#define MOE_FFN_COMBINE_FOLD 512
+
 /* Bytes of workspace moe_forward needs for this shape (fused or not). The
  * other entry points need at most this much. Returns 0 for an invalid shape. */
 size_t moe_workspace_size(const moe_shape* shape, int fuse_shared);
@@ -176,6 +185,13 @@ moe_status moe_combine(const moe_shape* shape, const void* y, const int32_t* inv
  * The expert rows are kept as fp16 scaled by a power of two per 32 columns
  * (11 significant bits) and aggregated in fp32 in slot order, rounded once to
  * act_dtype (or left in fp32 when shape->out_f32); the result is deterministic.
+ * With MOE_FFN_COMBINE_FOLD in ffn_impl the fused layer's aggregation runs
+ * inside the down-projection's units of the shared expert, which come last:
+ * each stores its rows, waits (bounded; MOE_ERR_TIMEOUT if it runs out) until
+ * the routed units of its columns have stored theirs, and sums every slot of
+ * its tokens in slot order (one launch less: the write-up's section 1 argument
+ * for the fusion). That kernel is a cooperative launch, all of its CTAs resident
+ * at once; where the launch is refused the aggregation runs as its own pass.
  *   x [T, H], router_w [n_routed, H], router_bias [n_routed] or NULL,
  *   w13 [E, 2I, H], s13, w2 [E, H, I], s2 as in moe_grouped_ffn, out [T, H]
  *   (act_dtype, or fp32 when out_f32).
@@ -233,12 +249,18 @@ moe_status moe_profile_read(const char* name, int64_t* launches, double* total_m
  * offsets [E+1], perm [R], inv [R] out, all caller-owned device buffers); the
  * kernels are the same. Their scratch lives in one 1 MiB array in the library's
  * device globals, which every GPU that loads the library holds until the
- * process exits. Limit: ceil(T*S / 512) * E <= 261888 (for 161 experts and 9
- * slots, T <= 92501); larger calls return MOE_ERR_UNSUPPORTED before enqueuing
- * anything. The library allocates nothing in this call.
+ * process exits. Limit, with E the number of expert groups (n_routed, + 1 with
+ * a shared expert) and S the slots per token:
+ *     ceil(T*S / 512) * E <= (1048576 - 256 - round256(4 * (E + 1))) / 4,
+ * round256 rounding up to a multiple of 256. The right side is 262016 for
+ * E <= 63, 261952 for E in 64..127, 261888 for 128..191 (161 experts and 9
+ * slots: T <= 92501), 261824 for 192..255 and 261760 for 256..257. Larger
+ * calls return MOE_ERR_UNSUPPORTED before enqueuing anything.
+ * The library allocates nothing in this call.
  * The first call on a device looks up the array's device address (once per
- * device, with that device current); make that first call before any stream
- * capture. All calls share the array and it keeps the last call's contents, so
+ * device and CUDA context, with that device current); make that first call
+ * before any stream capture. After cudaDeviceReset the next call is again a
+ * first call. All calls share the array and it keeps the last call's contents, so
  * calls that overlap on the GPU (other streams, other host threads) race and
  * must be serialised by the caller. Out-of-range ids are dropped as in
  * moe_permute, but not reported: this call has no status word the caller can
@@ -252,6 +274,14 @@ moe_status moe_permute_noalloc(const moe_shape* shape, const int32_t* ids, int32
  * kernels then drain, free TMEM, return, and leave MOE_ERR_TIMEOUT in the status
  * word (the outputs of those calls are garbage). No GPU fault is involved. */
 void moe_inject_wait_timeout(int n_calls);
+
+/* Failure-injection hook for the wait of the aggregation inside the fused
+ * layer's down-projection: in the next n_calls moe_forward calls that run it,
+ * the shared expert's units wait for one more routed-unit arrival than there
+ * will be, with a limit of about 10 ms; the waits run out, the kernel drains,
+ * frees TMEM and returns, and MOE_ERR_TIMEOUT is left in the status word (the
+ * outputs of those calls are garbage). No GPU fault is involved. */
+void moe_inject_fold_timeout(int n_calls);
 
 /* Fused QK-norm + partial RoPE on the attention's q and k heads, in place.
  * "GLM4-MoE生产环境优化：SGLang降低65%首Token延迟", section 2.2 QK-Norm-RoPE

@@ -16,13 +16,14 @@ MOE_ERR_CUDA, MOE_ERR_TIMEOUT, MOE_ERR_DEVICE = 4, 5, 6
 MOE_F32, MOE_BF16, MOE_E4M3 = 0, 1, 2
 (MOE_FFN_AUTO, MOE_FFN_SIMT, MOE_FFN_TCGEN05, MOE_FFN_TCGEN05_M128, MOE_FFN_TCGEN05_M256,
  MOE_FFN_TCGEN05_PAIR, MOE_FFN_TCGEN05_WIDE, MOE_FFN_TCGEN05_SWAP) = 0, 1, 2, 3, 4, 5, 6, 7
+MOE_FFN_COMBINE_FOLD = 512         # flag: the fused layer's aggregation inside its down-projection
 DTYPES = {"f32": MOE_F32, "bf16": MOE_BF16, "e4m3": MOE_E4M3}
 
 EXPORTS = ("moe_workspace_size", "moe_route_topk", "moe_permute", "moe_grouped_ffn",
            "moe_combine", "moe_forward", "moe_quant_rows_e4m3", "moe_get_status",
            "moe_clear_status", "moe_status_string", "moe_launch_count", "moe_profile_enable",
            "moe_profile_reset", "moe_profile_read", "moe_inject_wait_timeout",
-           "moe_permute_noalloc", "moe_qk_norm_rope", "moe_cast_f32_bf16")
+           "moe_permute_noalloc", "moe_qk_norm_rope", "moe_cast_f32_bf16", "moe_inject_fold_timeout")
 
 
 class MoeError(RuntimeError):
@@ -81,6 +82,8 @@ def lib() -> C.CDLL:
         L.moe_permute_noalloc.argtypes = [S, p, p, p, p, p, p]
         L.moe_inject_wait_timeout.restype = None
         L.moe_inject_wait_timeout.argtypes = [i]
+        L.moe_inject_fold_timeout.restype = None
+        L.moe_inject_fold_timeout.argtypes = [i]
         L.moe_cast_f32_bf16.restype = i
         L.moe_cast_f32_bf16.argtypes = [sz, p, p, p]
         L.moe_qk_norm_rope.restype = i
@@ -225,6 +228,10 @@ def moe_profile_reset():
 
 def moe_inject_wait_timeout(n_calls: int):
     lib().moe_inject_wait_timeout(int(n_calls))
+
+
+def moe_inject_fold_timeout(n_calls: int):
+    lib().moe_inject_fold_timeout(int(n_calls))
 
 
 def moe_profile_read(name: str):

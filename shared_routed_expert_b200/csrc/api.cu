@@ -61,7 +61,7 @@ size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 int act_bytes(int dt) { return dt == MOE_F32 ? 4 : 2; }
 
 struct Layout {
-    size_t status, partials, ids, wts, counts, offsets, tile_off, perm, inv, chunk;
+    size_t status, partials, ids, wts, counts, offsets, tile_off, perm, inv, chunk, ready;
     size_t xq, xscale, xp, xp_scale, h, hq, h_scale, y, yexp;
     // unfused only: the shared expert's dense pass
     size_t sh_off, sh_tile, sh_h, sh_hq, sh_hscale, sh_y, sh_yexp;
@@ -102,6 +102,7 @@ Layout layout_of(const moe_shape& s, const Dims& d) {
     L.perm = take(static_cast<size_t>(d.R) * 4);
     L.inv = take(static_cast<size_t>(d.R) * 4);
     L.chunk = take(permute_scratch_ints(d.R, d.E) * 4);
+    L.ready = take(static_cast<size_t>(d.H / 256) * 4);
     if (fp8) {
         L.xq = take(static_cast<size_t>(d.T) * d.H);
         L.xscale = take(static_cast<size_t>(d.T) * 4);
@@ -193,6 +194,7 @@ cudaError_t run_ffn(const FfnArgs& in, int impl, cudaStream_t st) {
 }
 
 moe_status check_impl(int impl, const moe_shape& s) {
+    impl &= ~MOE_FFN_COMBINE_FOLD;
     if (impl < MOE_FFN_AUTO || impl > MOE_FFN_TCGEN05_SWAP) return MOE_ERR_INVALID_ARG;
     if (impl >= MOE_FFN_TCGEN05 && s.w_dtype == MOE_F32) return MOE_ERR_UNSUPPORTED;
     return MOE_OK;
@@ -206,7 +208,7 @@ cudaError_t prepare_tokens(const moe_shape& s, const Dims& d, const Layout& L, v
         *xt = at<uint8_t>(ws, L.xq);
         *xt_scale = at<float>(ws, L.xscale);
         return launch_quant_rows(d.T, d.H, static_cast<const uint16_t*>(x), at<uint8_t>(ws, L.xq),
-                                 at<float>(ws, L.xscale), st);
+                                 at<float>(ws, L.xscale), st, "quant_x");
     }
     *xt = x;
     *xt_scale = nullptr;
@@ -238,6 +240,12 @@ FfnArgs ffn_args(const moe_shape& s, const Dims& d, const Layout& L, void* ws, c
     a.cta_pair = 0;
     a.direct_e = -1;
     a.max_mtiles = d.R / kTileM + d.E;
+    a.fold_inv = nullptr;
+    a.fold_w = nullptr;
+    a.fold_out = nullptr;
+    a.fold_out_f32 = 0;
+    a.fold_ready = nullptr;
+    a.folded = nullptr;
     a.status = at<DevStatus>(ws, L.status);
     return a;
 }
@@ -294,6 +302,7 @@ moe_status moe_grouped_ffn(const moe_shape* shape, const void* x, const int32_t*
                            int ffn_impl, void* stream) {
     moe_status rc = check_shape(shape);
     if (rc != MOE_OK) return rc;
+    if (ffn_impl & MOE_FFN_COMBINE_FOLD) return MOE_ERR_INVALID_ARG;   // no aggregation here
     if ((rc = check_impl(ffn_impl, *shape)) != MOE_OK) return rc;
     if (!x || !perm || !offsets || !w13 || !w2 || !y || !ws) return MOE_ERR_INVALID_ARG;
     const bool fp8 = shape->w_dtype == MOE_E4M3;
@@ -355,6 +364,8 @@ moe_status moe_forward(const moe_shape* shape, const void* x, const float* route
         return MOE_ERR_INVALID_ARG;
     const bool fused = fuse_shared != 0;
     if (!fused && shape->shared_id < 0) return MOE_ERR_INVALID_ARG;
+    const bool fold_combine = (ffn_impl & MOE_FFN_COMBINE_FOLD) != 0;
+    ffn_impl &= ~MOE_FFN_COMBINE_FOLD;
     const Dims d = dims_of(*shape, fused);
     const Layout L = layout_of(*shape, d);
     if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
@@ -374,6 +385,7 @@ moe_status moe_forward(const moe_shape* shape, const void* x, const float* route
                              at<DevStatus>(ws, L.status), st);
     const void* xt = nullptr;
     const float* xt_scale = nullptr;
+    bool folded = false;
     if (err == cudaSuccess) err = prepare_tokens(*shape, d, L, ws, x, &xt, &xt_scale, st);
     if (err == cudaSuccess) {
         FfnArgs a = ffn_args(*shape, d, L, ws, xt, xt_scale, at<int32_t>(ws, L.perm), w13, s13, w2, s2,
@@ -382,6 +394,16 @@ moe_status moe_forward(const moe_shape* shape, const void* x, const float* route
         // fused layout: the shared expert's group is every token in order (stable
         // permutation, shared id last), so its rows need no gather
         a.direct_e = (fused && d.shared) ? d.E - 1 : -1;
+        if (a.direct_e >= 0 && !f32_act && fold_combine) {
+            // the weighted combine inside GEMM2's shared-expert units, where the
+            // tensor-core GEMM2 runs it (folded tells whether it did)
+            a.fold_inv = at<int32_t>(ws, L.inv);
+            a.fold_w = wts;
+            a.fold_out = out;
+            a.fold_out_f32 = shape->out_f32 != 0;
+            a.fold_ready = at<unsigned>(ws, L.ready);
+            a.folded = &folded;
+        }
         err = run_ffn(a, ffn_impl, st);
     }
 
@@ -415,13 +437,19 @@ moe_status moe_forward(const moe_shape* shape, const void* x, const float* route
         a.cta_pair = 0;
         a.direct_e = -1;
         a.max_mtiles = ceil_div(d.T, kTileM);
+        a.fold_inv = nullptr;
+        a.fold_w = nullptr;
+        a.fold_out = nullptr;
+        a.fold_out_f32 = 0;
+        a.fold_ready = nullptr;
+        a.folded = nullptr;
         a.status = at<DevStatus>(ws, L.status);
         dense_offsets_kernel<<<1, 1, 0, st>>>(d.T, at<int32_t>(ws, L.sh_off), at<int32_t>(ws, L.sh_tile));
         note_launch();
         err = cudaGetLastError();
         if (err == cudaSuccess) err = run_ffn(a, ffn_impl, st);
     }
-    if (err == cudaSuccess) {
+    if (err == cudaSuccess && !folded) {
         const int32_t* inv = at<int32_t>(ws, L.inv);
         if (f32_act)
             err = launch_combine(d.T, d.S, d.H, MOE_F32, at<void>(ws, L.y), inv, wts,
@@ -490,6 +518,8 @@ const char* moe_status_string(moe_status s) {
 uint64_t moe_launch_count(void) { return g_launches.load(); }
 
 void moe_inject_wait_timeout(int n_calls) { ffn_tc_inject_stall(n_calls > 0 ? n_calls : 0); }
+
+void moe_inject_fold_timeout(int n_calls) { ffn_tc_inject_fold_stall(n_calls > 0 ? n_calls : 0); }
 
 void moe_profile_enable(int on) { g_prof_on.store(on != 0); }
 

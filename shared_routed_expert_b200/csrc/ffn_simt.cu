@@ -264,7 +264,7 @@ cudaError_t launch_ffn_simt(const FfnArgs& in, cudaStream_t stream) {
     }
     if (a.w_dtype == MOE_E4M3) {
         cudaError_t err = launch_quant_rows(a.R, a.I, static_cast<const uint16_t*>(a.h), a.hq,
-                                            a.h_scale, stream);
+                                            a.h_scale, stream, "quant_h");
         if (err != cudaSuccess) return err;
     }
     {

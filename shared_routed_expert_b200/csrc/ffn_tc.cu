@@ -51,6 +51,7 @@ constexpr int TC_RING_BYTES = 192 * 1024;          // shared memory for the stag
 #define SRE_STAGE_ROW_BYTES 128
 #endif
 constexpr int TC_MAXE = 260;
+
 constexpr uint32_t TC_TMEM_COLS = 512;
 
 struct TcParams {
@@ -69,6 +70,18 @@ struct TcParams {
     const float* col_scale; // E4M3: per-output-channel weight scale (s13 [E, 2I] or s2 [E, H])
     // GEMM2 with yexp != null: rows stored as fp16(v * 2^-k), k per 32 columns in yexp
     int8_t* yexp;
+    // GEMM2 with the weighted combine folded in (fold_e >= 0): the fold_e group's
+    // units (the shared expert's; its rows are the tokens in order, its units the
+    // last ones) also write the layer output, summing each token's slots; see
+    // fold_combine
+    int fold_e;
+    int fold_S;                 // slots per token; the fold_e group's slot is the last
+    const int32_t* fold_inv;    // [T * S] flat slot -> row
+    const float* fold_w;        // [T * S] slot weights
+    void* fold_out;             // [T, H] bf16, or fp32 when fold_out_f32
+    int fold_out_f32;
+    unsigned* ready;            // [n_tiles_n] routed-unit epilogue warps done, per n-tile (zero at launch)
+    unsigned fold_extra;        // testing hook: added to the arrivals a fold_e unit waits for (never reached)
     DevStatus* status;
     long long wait_limit;   // SM clock cycles per wait
     int inject_stall;       // testing hook: the producer never issues its loads
@@ -130,6 +143,29 @@ __device__ __forceinline__ void stage_store(uint8_t* slice, const uint32_t (&pac
     __syncwarp();
 }
 
+// E4M3 layers: this warp's per-output-channel weight scales of a unit (GEMM2:
+// columns n0 + 32 c_begin .. n0 + 32 c_end of expert e; GEMM1: the gate columns
+// of those h columns, then the up columns) copied once into its 1 KB shared
+// area, coalesced, so that the epilogue reads them as broadcasts instead of one
+// global load per value and chunk.
+template <bool kGemm1>
+__device__ __forceinline__ void stage_scales(const TcParams& p, const TileInfo& t, int c_begin, int c_end,
+                                             float* dst, int lane) {
+    const int n = (c_end - c_begin) * 32;
+    __syncwarp();                                    // the previous unit's reads are done
+    if constexpr (kGemm1) {
+        const float* g = p.col_scale + static_cast<size_t>(t.e) * 2 * p.I + t.n0 + c_begin * 32;
+        for (int i = lane; i < n; i += 32) {
+            dst[i] = g[i];
+            dst[n + i] = g[p.I + i];
+        }
+    } else {
+        const float* g = p.col_scale + static_cast<size_t>(t.e) * p.H + t.n0 + c_begin * 32;
+        for (int i = lane; i < n; i += 32) dst[i] = g[i];
+    }
+    __syncwarp();
+}
+
 // Epilogue of one unit for one warp: TMEM columns [c_begin, c_end) x 32 of the
 // lane group at `tb` (row = this lane's output row, valid if it is stored)
 // become bf16 h (GEMM1, SwiGLU applied) or bf16 / scaled-fp16 y rows (GEMM2),
@@ -137,7 +173,7 @@ __device__ __forceinline__ void stage_store(uint8_t* slice, const uint32_t (&pac
 template <bool kFp8, bool kGemm1, int kBN>
 __device__ __forceinline__ void epilogue_rows(const TcParams& p, const TileInfo& t, uint32_t tb, int c_begin,
                                               int c_end, uint8_t* stage_w, int lane, int row, bool valid,
-                                              float rs, int wrow0) {
+                                              float rs, int wrow0, const float* scs) {
     constexpr int HALF = kBN / 2;
     if constexpr (kGemm1) {
 #pragma unroll 1
@@ -147,20 +183,20 @@ __device__ __forceinline__ void epilogue_rows(const TcParams& p, const TileInfo&
             ptx::tmem_ld_32x32b_x32(tb + HALF + c * 32, u);
             ptx::tmem_ld_wait(g);
             ptx::tmem_ld_wait(u);
-            const float* sg = (kFp8 && valid) ? p.col_scale + static_cast<size_t>(t.e) * 2 * p.I + t.n0 + c * 32 : nullptr;
-            const float* su = (kFp8 && valid) ? sg + p.I : nullptr;
+            // this warp's staged weight scales: gate columns, then up columns (broadcast reads)
+            const float* sg = scs + (c - c_begin) * 32;
+            const float* su = scs + (c_end - c_begin) * 32 + (c - c_begin) * 32;
             uint32_t packed[16];
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
                 float g0 = __uint_as_float(g[j]), g1 = __uint_as_float(g[j + 1]);
                 float u0 = __uint_as_float(u[j]), u1 = __uint_as_float(u[j + 1]);
                 if constexpr (kFp8) {
-                    if (valid) {
-                        g0 = g0 * rs * sg[j];
-                        g1 = g1 * rs * sg[j + 1];
-                        u0 = u0 * rs * su[j];
-                        u1 = u1 * rs * su[j + 1];
-                    }
+                    // rows past the group end are computed too and not stored
+                    g0 = g0 * rs * sg[j];
+                    g1 = g1 * rs * sg[j + 1];
+                    u0 = u0 * rs * su[j];
+                    u1 = u1 * rs * su[j + 1];
                 }
                 packed[j >> 1] = pack_bf16x2(silu_f32(g0) * u0, silu_f32(g1) * u1);
             }
@@ -170,14 +206,12 @@ __device__ __forceinline__ void epilogue_rows(const TcParams& p, const TileInfo&
         // chunk c's TMEM load is in flight while chunk c-1 is converted and stored
         uint64_t exps = 0;
         auto process = [&](const uint32_t (&v)[32], int c) {
-            const float* sc = (kFp8 && valid) ? p.col_scale + static_cast<size_t>(t.e) * p.H + t.n0 + c * 32 : nullptr;
+            const float* sc = scs + (c - c_begin) * 32;      // this warp's staged weight scales
             float a[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
                 a[j] = __uint_as_float(v[j]);
-                if constexpr (kFp8) {
-                    if (valid) a[j] = a[j] * rs * sc[j];
-                }
+                if constexpr (kFp8) a[j] = a[j] * rs * sc[j];   // rows past the group end are not stored
             }
             uint32_t packed[16];
             if (p.yexp != nullptr) {
@@ -195,28 +229,152 @@ __device__ __forceinline__ void epilogue_rows(const TcParams& p, const TileInfo&
             }
             stage_store(stage_w, packed, lane, p.out, p.out_ld, wrow0, t.row_end, t.n0 + c * 32);
         };
-        uint32_t va[32], vb[32];
-        ptx::tmem_ld_32x32b_x32(tb + c_begin * 32, va);
-        ptx::tmem_ld_wait(va);
+        if constexpr (kFp8) {
+            // E4M3: one chunk at a time (the scale products need the registers)
 #pragma unroll 1
-        for (int c = c_begin; c < c_end; c += 2) {
-            const bool has_b = c + 1 < c_end;
-            if (has_b) ptx::tmem_ld_32x32b_x32(tb + (c + 1) * 32, vb);
-            process(va, c);
-            if (has_b) {
-                ptx::tmem_ld_wait(vb);
-                const bool has_a = c + 2 < c_end;
-                if (has_a) ptx::tmem_ld_32x32b_x32(tb + (c + 2) * 32, va);
-                process(vb, c + 1);
-                if (has_a) ptx::tmem_ld_wait(va);
+            for (int c = c_begin; c < c_end; ++c) {
+                uint32_t v[32];
+                ptx::tmem_ld_32x32b_x32(tb + c * 32, v);
+                ptx::tmem_ld_wait(v);
+                process(v, c);
+            }
+        } else {
+            uint32_t va[32], vb[32];
+            ptx::tmem_ld_32x32b_x32(tb + c_begin * 32, va);
+            ptx::tmem_ld_wait(va);
+#pragma unroll 1
+            for (int c = c_begin; c < c_end; c += 2) {
+                const bool has_b = c + 1 < c_end;
+                if (has_b) ptx::tmem_ld_32x32b_x32(tb + (c + 1) * 32, vb);
+                process(va, c);
+                if (has_b) {
+                    ptx::tmem_ld_wait(vb);
+                    const bool has_a = c + 2 < c_end;
+                    if (has_a) ptx::tmem_ld_32x32b_x32(tb + (c + 2) * 32, va);
+                    process(vb, c + 1);
+                    if (has_a) ptx::tmem_ld_wait(va);
+                }
             }
         }
         if (p.yexp != nullptr && valid) {
             int8_t* e = p.yexp + static_cast<size_t>(row) * (p.H / 32) + t.n0 / 32 + c_begin;
-            if (c_end - c_begin == 8) *reinterpret_cast<uint64_t*>(e) = exps;
-            else *reinterpret_cast<uint32_t*>(e) = static_cast<uint32_t>(exps);
+            const int n = c_end - c_begin;
+            if (n == 8) *reinterpret_cast<uint64_t*>(e) = exps;
+            else if (n == 4) *reinterpret_cast<uint32_t*>(e) = static_cast<uint32_t>(exps);
+            else
+                for (int i = 0; i < n; ++i) e[i] = static_cast<int8_t>((exps >> (8 * i)) & 0xFFu);
         }
     }
+}
+
+// Weighted combine inside the down-projection ("Optimizing GLM4-MoE for
+// production" (Novita AI), section 1: the outputs of a token's experts are
+// aggregated with weights), done by the fold_e group's units (the shared
+// expert's, whose rows are the tokens in order and whose units come last)
+// when moe_forward is asked for it (MOE_FFN_COMBINE_FOLD): one launch less,
+// and the reads overlap the MMAs of the units that follow. A warp first stores
+// its rows of the unit as every unit does (epilogue_rows), frees the
+// accumulator so that the next unit's MMAs start, waits until every routed
+// unit of this n-tile has stored its rows (p.ready), and then, for each of its
+// 32 tokens and its columns [col0, col0 + ncols),
+//     out[tok, cols] = sum_{k < S} w[tok, k] * y[inv[tok * S + k], cols]
+// accumulating in fp32 in slot order (one fma per slot with the slot's weight
+// times its chunk's power of two; the unit's own row is the last slot) and
+// rounding once: the operations of the separate combine kernel in the same
+// order, so the output is the same bit for bit. Sixteen lanes cover 128
+// contiguous columns (8 each) of one token's rows, so every load reads 256
+// contiguous bytes of a row. Measured on B200 this is slower than the separate
+// combine pass (prefill_bf16 GEMM2 0.97 ms against 0.61 + 0.08 ms): the eight
+// epilogue warps keep ~20 KB of loads in flight per SM where the separate pass
+// keeps several times that, so the aggregation is latency-bound here.
+constexpr int FOLD_SLOTS = 5;    // slot rows whose loads are issued together
+
+__device__ __forceinline__ void fold_store(const TcParams& p, int tok, int col, const float (&acc)[8]) {
+    if (p.fold_out_f32) {
+        float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.fold_out) + static_cast<size_t>(tok) * p.H + col);
+        o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    } else {
+        *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.fold_out) + static_cast<size_t>(tok) * p.H + col) =
+            make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
+                       pack_bf16x2(acc[6], acc[7]));
+    }
+}
+
+__device__ __forceinline__ void fold_fma(const uint4& q, float wgt, float (&acc)[8]) {
+    const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+        const float2 f = unpack_f16x2(u[h]);
+        acc[2 * h] = __fmaf_rn(wgt, f.x, acc[2 * h]);
+        acc[2 * h + 1] = __fmaf_rn(wgt, f.y, acc[2 * h + 1]);
+    }
+}
+
+// The combine of one warp's 32 rows (unit rows wrow0 .. +31, tokens wrow0 -
+// grp0 ..) over columns [col0, col0 + ncols), ncols a multiple of 128; this warp
+// takes work items item0, item0 + istride, ... Work item i = (token pair i % 16,
+// 128-column block i / 16); lanes 0-15 take the pair's first token, 16-31 its
+// second, 8 columns per lane; the loads of FOLD_SLOTS slot rows are in flight
+// together.
+__device__ __forceinline__ void fold_combine(const TcParams& p, int row_end, int lane, int wrow0, int grp0,
+                                             int col0, int ncols, int item0, int istride) {
+    const int S = p.fold_S;
+    const int ne = p.H / 32;
+    const int items = 16 * (ncols >> 7);
+    const int half = lane >> 4;
+    const int cl = (lane & 15) * 8;
+#pragma unroll 1
+    for (int it = item0; it < items; it += istride) {
+        const int row = wrow0 + 2 * (it % 16) + half;
+        const int col = col0 + (it / 16) * 128 + cl;
+        if (row >= row_end) continue;
+        const int tok = row - grp0;
+        float acc[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
+#pragma unroll 1
+        for (int k0 = 0; k0 < S; k0 += FOLD_SLOTS) {
+            uint4 q[FOLD_SLOTS];
+            int ex[FOLD_SLOTS];
+            float wk[FOLD_SLOTS];
+#pragma unroll
+            for (int g = 0; g < FOLD_SLOTS; ++g) {
+                if (k0 + g < S) {
+                    const size_t f = static_cast<size_t>(tok) * S + k0 + g;
+                    const size_t r = static_cast<size_t>(p.fold_inv[f]);
+                    q[g] = *reinterpret_cast<const uint4*>(p.out + r * p.H + col);
+                    ex[g] = p.yexp[r * ne + (col >> 5)];
+                    wk[g] = p.fold_w[f];
+                }
+            }
+#pragma unroll
+            for (int g = 0; g < FOLD_SLOTS; ++g)
+                if (k0 + g < S) fold_fma(q[g], wk[g] * exp2_int(ex[g]), acc);
+        }
+        fold_store(p, tok, col, acc);
+    }
+}
+
+// A routed unit's epilogue warp is done storing: its rows become visible at GPU
+// scope before the n-tile's counter counts it.
+__device__ __forceinline__ void fold_arrive(const TcParams& p, int nt, int lane) {
+    __threadfence();
+    __syncwarp();
+    if (lane == 0) ptx::red_release_gpu_add(p.ready + nt, 1u);
+}
+
+// Before a fold_e unit reads routed rows: wait until every routed unit's
+// epilogue warps have counted themselves on this n-tile (bounded; false on
+// timeout or abort).
+__device__ __forceinline__ bool fold_wait(const TcParams& p, int nt, unsigned target, volatile int* abort,
+                                          int lane) {
+    int ok = 1;
+    if (lane == 0) ok = ptx::counter_wait(p.ready + nt, target, abort, p.wait_limit, p.status, 5u);
+    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+    __syncwarp();          // the warp's own stores of this unit are visible to all its lanes
+    __threadfence();
+    return ok != 0;
 }
 
 // kBN: MMA N (GEMM1: gate half + up half; GEMM2: 256 output columns).
@@ -229,19 +387,35 @@ __device__ __forceinline__ void epilogue_rows(const TcParams& p, const TileInfo&
 // columns in two halves (two warps per TMEM sub-partition).
 // kRowB: bytes of K per row per stage (128: 128-byte swizzle; 64: 64-byte swizzle,
 // twice as many stages of half the size).
-template <int kRowB, int kBN, bool kPair>
+// Epilogue warps of the single-CTA kernel: 12 (three per TMEM lane group) for
+// the E4M3 down-projection on 128-row units, whose epilogue (per-row and
+// per-column scales, scaled-fp16 rows) is the slowest part of its unit; 8 else
+#ifndef SRE_E4M3_EPI12
+#define SRE_E4M3_EPI12 0
+#endif
+template <bool kFp8, bool kGemm1, bool kPair>
+constexpr int gg_epi_warps() {
+    return (SRE_E4M3_EPI12 && kFp8 && !kGemm1 && !kPair) ? 12 : 8;
+}
+
+template <int kRowB, int kBN, bool kPair, int kEpiW>
 struct Ring {
     static constexpr int A_TILE = TC_BM * kRowB;
     static constexpr int STAGE = (kPair ? 2 : 1) * A_TILE + kBN * kRowB;
     static constexpr int N = (TC_RING_BYTES / STAGE) > 8 ? 8 : (TC_RING_BYTES / STAGE);
-    static constexpr int SMEM = N * STAGE + 8 * 2048 + 1024;   // + epilogue staging + alignment
+    // weight-scale area per epilogue warp: 256 floats, or 128 with 12 warps (three
+    // chunks of 32 columns each at most)
+    static constexpr int SCALE_B = kEpiW == 12 ? 512 : 1024;
+    // + epilogue staging (2 KB per warp), weight scales, alignment
+    static constexpr int SMEM = N * STAGE + kEpiW * 2048 + kEpiW * SCALE_B + 1024;
 };
 
 template <bool kFp8, bool kGemm1, int kBN, bool kPair, int kRowB>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__((2 + gg_epi_warps<kFp8, kGemm1, kPair>()) * 32, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmA2, const TcParams p) {
-    using RG = Ring<kRowB, kBN, kPair>;
+    constexpr int EPI_WARPS = gg_epi_warps<kFp8, kGemm1, kPair>();
+    using RG = Ring<kRowB, kBN, kPair, EPI_WARPS>;
     constexpr int NSTAGE = RG::N;
     constexpr int TC_ABYTES = RG::A_TILE;           // one 128-row A tile per stage
     constexpr int ABYTES = (kPair ? 2 : 1) * TC_ABYTES;
@@ -249,11 +423,11 @@ __global__ void __launch_bounds__(320, 1)
     constexpr int HALF = kBN / 2;
     constexpr int KEL = kFp8 ? kRowB : kRowB / 2;   // K elements per stage
     constexpr int KSTEPS = kRowB / 32;              // MMAs (32 bytes of K each) per stage
-    constexpr int EPI_WARPS = 8;
     constexpr uint32_t IDESC = ptx::instr_desc(TC_BM, kBN, kFp8 ? 0u : 1u);
 
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t full_bar[NSTAGE], empty_bar[NSTAGE], tfull_bar[2], tempty_bar[2], drain_bar;
+    __shared__ uint64_t fold_bar[4];   // per TMEM lane group: its epilogue warps' rows of a unit are stored
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
     __shared__ int s_off[TC_MAXE], s_unit[TC_MAXE];
@@ -264,6 +438,7 @@ __global__ void __launch_bounds__(320, 1)
     uint8_t* sA = base;
     uint8_t* sB = base + NSTAGE * ABYTES;
     uint8_t* sStage = sB + NSTAGE * BBYTES;         // EPI_WARPS x 2 KB
+    float* sScale = reinterpret_cast<float*>(sStage + EPI_WARPS * 2048);   // EPI_WARPS x RG::SCALE_B (E4M3 weight scales)
     volatile int* abort_flag = &s_abort;
 
     for (int i = threadIdx.x; i <= p.E; i += blockDim.x) s_off[i] = p.offsets[i];
@@ -296,6 +471,7 @@ __global__ void __launch_bounds__(320, 1)
             ptx::mbar_init(&tfull_bar[b], 1);
             ptx::mbar_init(&tempty_bar[b], EPI_WARPS * 32);
         }
+        for (int g = 0; g < 4; ++g) ptx::mbar_init(&fold_bar[g], EPI_WARPS / 4);
         ptx::mbar_init(&drain_bar, 1);
         s_abort = 0;
         ptx::fence_mbar_init();
@@ -421,14 +597,16 @@ __global__ void __launch_bounds__(320, 1)
     } else {
         // ---------------------------------------------------------------- epilogue
         const int sub = warp & 3;                  // TMEM lanes 32*sub .. +31
-        const int eg = (warp - 2) >> 2;            // pair: accumulator; single: column half
+        constexpr int EG = EPI_WARPS / 4;          // epilogue warps per TMEM lane group
+        const int eg = (warp - 2) >> 2;            // pair: accumulator; single: column share
         const int r_local = (kPair ? eg * TC_BM : 0) + sub * 32 + lane;
         constexpr int NCH = kGemm1 ? HALF / 32 : kBN / 32;   // 32-column chunks per unit
-        constexpr int PER = kPair ? NCH : (NCH + 1) / 2;
+        constexpr int PER = kPair ? NCH : (NCH + EG - 1) / EG;
         const int c_begin = kPair ? 0 : eg * PER;
         const int c_end = kPair ? NCH : min(NCH, c_begin + PER);
         int acc = 0;
         uint32_t acc_phase = 0;
+        uint32_t fold_phase = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
             const TileInfo t = decode_unit<kPair>(tile, s_unit, s_off, p.E, p.n_tiles_n, p.bn_out);
             // one lane waits and the warp takes its result: tcgen05.ld below needs the whole warp
@@ -445,15 +623,45 @@ __global__ void __launch_bounds__(320, 1)
             float rs = 1.0f;
             if (kFp8 && valid)
                 rs = (t.e == p.direct_e) ? p.direct_scale[row - s_off[t.e]] : p.row_scale[row];
+            const bool fold = !kGemm1 && t.e == p.fold_e;
+            const int wrow0 = t.row0 + (kPair ? eg * TC_BM : 0) + sub * 32;   // first unit row of this warp
             if (active) {
                 // 16-bit outputs leave through this warp's 2 KB staging slice so that
                 // global stores cover whole 64-byte row segments (see stage_store)
                 uint8_t* stage_w = sStage + (warp - 2) * 2048;
-                const int wrow0 = t.row0 + (kPair ? eg * TC_BM : 0) + sub * 32;   // first unit row of this warp
-                epilogue_rows<kFp8, kGemm1, kBN>(p, t, tb, c_begin, c_end, stage_w, lane, row, valid, rs, wrow0);
+                float* scs = sScale + (warp - 2) * (RG::SCALE_B / 4);
+                if constexpr (kFp8) stage_scales<kGemm1>(p, t, c_begin, c_end, scs, lane);
+                epilogue_rows<kFp8, kGemm1, kBN>(p, t, tb, c_begin, c_end, stage_w, lane, row, valid, rs, wrow0, scs);
             }
+            if (!kGemm1 && p.fold_e >= 0 && !fold) fold_arrive(p, t.n0 / p.bn_out, lane);
             ptx::tc_fence_before();
             ptx::mbar_arrive(&tempty_bar[acc]);
+            if (fold && active) {
+                // the accumulator is free for the next unit; the combine reads global memory only
+                // arrivals on the n-tile's counter once every routed unit is stored
+                const unsigned target =
+                    static_cast<unsigned>(s_unit[p.E] - (s_unit[p.fold_e + 1] - s_unit[p.fold_e])) * EPI_WARPS +
+                    p.fold_extra;
+                if (!fold_wait(p, t.n0 / p.bn_out, target, abort_flag, lane)) break;
+                if constexpr (EG == 2 || kPair) {
+                    fold_combine(p, t.row_end, lane, wrow0, s_off[t.e], t.n0 + c_begin * 32, (c_end - c_begin) * 32,
+                                 0, 1);
+                } else {
+                    // the lane group's warps share its rows: all of their stores are done
+                    // before any of them sums (a bounded wait on the group's barrier), and
+                    // they take its 128-column blocks in turn
+                    __syncwarp();
+                    int ok2 = 1;
+                    if (lane == 0) {
+                        ptx::mbar_arrive(&fold_bar[sub]);
+                        ok2 = ptx::mbar_wait(&fold_bar[sub], fold_phase, abort_flag, p.wait_limit, p.status, 6u);
+                    }
+                    ok2 = __shfl_sync(0xFFFFFFFFu, ok2, 0);
+                    fold_phase ^= 1u;
+                    if (!ok2) break;
+                    fold_combine(p, t.row_end, lane, wrow0, s_off[t.e], t.n0, kBN, eg, EG);
+                }
+            }
             if constexpr (kPair) {
                 acc_phase ^= 1u;
             } else {
@@ -504,7 +712,7 @@ struct Ring2 {
     static constexpr int B_HALF = kNSUB * B_SUB;
     static constexpr int STAGE = A_TILE + B_HALF;
     static constexpr int N = (TC_RING_BYTES / STAGE) > 8 ? 8 : (TC_RING_BYTES / STAGE);
-    static constexpr int SMEM = N * STAGE + 8 * 2048 + 1024;
+    static constexpr int SMEM = N * STAGE + 8 * 2048 + 8 * 1024 + 1024;
 };
 
 template <bool kFp8, bool kGemm1, int kBN, int kNSUB, int kRowB>
@@ -536,6 +744,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
     uint8_t* sA = base;
     uint8_t* sB = base + NSTAGE * ABYTES;
     uint8_t* sStage = sB + NSTAGE * BBYTES;
+    float* sScale = reinterpret_cast<float*>(sStage + EPI_WARPS * 2048);   // EPI_WARPS x 1 KB (E4M3 weight scales)
     volatile int* abort_flag = &s_abort;
     const uint32_t peer_abort = ptx::mapa(&s_abort, rank ^ 1u);
 
@@ -728,6 +937,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
                 break;
             }
             ptx::tc_fence_after();
+            const int nt = t.n0 / p.bn_out;
             if constexpr (kNSUB == 2) t.n0 += eg * (kGemm1 ? HALF : kBN);   // this sub-tile's output columns
             const bool active = (rank == 0 || t.two) && c_begin < c_end;    // warp-uniform
             const int row = t.row0 + r_local;
@@ -736,12 +946,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
             float rs = 1.0f;
             if (kFp8 && valid)
                 rs = (t.e == p.direct_e) ? p.direct_scale[row - s_off[t.e]] : p.row_scale[row];
+            const bool fold = !kGemm1 && t.e == p.fold_e;
+            const int wrow0 = t.row0 + static_cast<int>(rank) * TC_BM + sub * 32;
             if (active) {
-                const int wrow0 = t.row0 + static_cast<int>(rank) * TC_BM + sub * 32;
-                epilogue_rows<kFp8, kGemm1, kBN>(p, t, tb, c_begin, c_end, stage_w, lane, row, valid, rs, wrow0);
+                float* scs = sScale + (warp - 2) * 256;
+                if constexpr (kFp8) stage_scales<kGemm1>(p, t, c_begin, c_end, scs, lane);
+                epilogue_rows<kFp8, kGemm1, kBN>(p, t, tb, c_begin, c_end, stage_w, lane, row, valid, rs, wrow0, scs);
             }
+            if (!kGemm1 && p.fold_e >= 0 && !fold) fold_arrive(p, nt, lane);
             ptx::tc_fence_before();
             ptx::mbar_arrive_remote(acc == 0 ? tempty0 : tempty1);
+            if (fold && active) {
+                // the accumulator is free for the next unit; the combine reads global memory only
+                // arrivals (both CTAs' epilogue warps) on the n-tile's counter once
+                // every routed unit is stored
+                const unsigned target =
+                    static_cast<unsigned>(s_unit[p.E] - (s_unit[p.fold_e + 1] - s_unit[p.fold_e])) * 2u * EPI_WARPS +
+                    p.fold_extra;
+                if (!fold_wait(p, nt, target, abort_flag, lane)) {
+                    if (lane == 0) ptx::st_remote_u32(peer_abort, 1u);
+                    break;
+                }
+                fold_combine(p, t.row_end, lane, wrow0, s_off[t.e], t.n0 + c_begin * 32, (c_end - c_begin) * 32, 0, 1);
+            }
             if constexpr (kNSUB == 1) {
                 acc ^= 1;
                 if (acc == 0) acc_phase ^= 1u;
@@ -946,7 +1173,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SW_THREADS, 1)
     const uint32_t tmem_base = s_tmem;
     const int total = s_unit[p.E] * p.n_tiles_n;
     // the largest group's units (all 256 rows) go first, so that the last wave
-    // holds the smaller routed units; every role walks the same rotated order
+    // holds the smaller routed units; every role walks the same rotated order.
+    // (Spreading them evenly through the schedule instead, so that tensor-bound
+    // shared units run beside HBM-bound routed ones, measured 1-1.5% slower.)
     const int rot = p.first_e >= 0 ? s_unit[p.first_e] * p.n_tiles_n : 0;
     auto unit = [&](int u) {
         const int v = u + rot;
@@ -1244,12 +1473,32 @@ int gemm1_half(int I) {
 }
 
 std::atomic<int> g_inject{0};
+std::atomic<int> g_inject_fold{0};
+
+// Launch of a persistent grid; cooperative (every CTA resident at once, or the
+// launch fails) when the kernel's CTAs wait on one another (the folded combine)
+template <typename Kern>
+cudaError_t launch_grid(Kern kern, int grid, int threads, int smem, bool coop, cudaStream_t st,
+                        const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2, const TcParams& p) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    cfg.blockDim = dim3(static_cast<unsigned>(threads), 1, 1);
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = coop ? attr : nullptr;
+    cfg.numAttrs = coop ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, a, b, a2, p);
+}
 
 template <bool kFp8, bool kGemm1, int kBN, bool kPair>
 cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2, const TcParams& p,
                        cudaStream_t st, const char* name) {
     constexpr int kRowB = SRE_STAGE_ROW_BYTES;
-    constexpr int smem = Ring<kRowB, kBN, kPair>::SMEM;
+    constexpr int kEpiW = gg_epi_warps<kFp8, kGemm1, kPair>();
+    constexpr int smem = Ring<kRowB, kBN, kPair, kEpiW>::SMEM;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
@@ -1258,9 +1507,10 @@ cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const CUtenso
     });
     if (attr_err != cudaSuccess) return attr_err;
     ProfileScope ps(name, st);
-    grouped_gemm_kernel<kFp8, kGemm1, kBN, kPair, kRowB><<<num_sms(), 320, smem, st>>>(a, b, a2, p);
+    const cudaError_t err = launch_grid(grouped_gemm_kernel<kFp8, kGemm1, kBN, kPair, kRowB>, num_sms(),
+                                        (2 + kEpiW) * 32, smem, p.fold_e >= 0, st, a, b, a2, p);
     note_launch();
-    return cudaGetLastError();
+    return err;
 }
 
 // CTA pairs: as many clusters of two as can be resident at once (a TPC with
@@ -1288,9 +1538,9 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtens
     });
     if (attr_err != cudaSuccess) return attr_err;
     ProfileScope ps(name, st);
-    kern<<<2 * clusters, 320, smem, st>>>(a, b, a2, p);
+    const cudaError_t err = launch_grid(kern, 2 * clusters, 320, smem, p.fold_e >= 0, st, a, b, a2, p);
     note_launch();
-    return cudaGetLastError();
+    return err;
 }
 
 // tokens as N on CTA pairs: sized like launch_pair
@@ -1342,6 +1592,7 @@ cudaError_t launch_gemm1_pair(const CUtensorMap& a, const CUtensorMap& b, const 
 }  // namespace
 
 void ffn_tc_inject_stall(int n_launches) { g_inject.store(n_launches); }
+void ffn_tc_inject_fold_stall(int n_launches) { g_inject_fold.store(n_launches); }
 
 bool ffn_tc_supported(const FfnArgs& a) {
     if (a.act_dtype != MOE_BF16) return false;
@@ -1435,6 +1686,14 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
     p.direct_scale = fp8 ? a.xt_scale : nullptr;
     p.col_scale = fp8 ? a.s13 : nullptr;
     p.yexp = nullptr;
+    p.fold_e = -1;
+    p.fold_S = 0;
+    p.fold_inv = nullptr;
+    p.fold_w = nullptr;
+    p.fold_out = nullptr;
+    p.fold_out_f32 = 0;
+    p.ready = nullptr;
+    p.fold_extra = 0;
     p.status = a.status;
     p.wait_limit = inject ? (20ll << 20) : (4ll << 30);
     p.inject_stall = inject;
@@ -1458,7 +1717,7 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
 
     const void* hA = a.h;
     if (fp8) {
-        err = launch_quant_rows(a.R, a.I, static_cast<const uint16_t*>(a.h), a.hq, a.h_scale, st);
+        err = launch_quant_rows(a.R, a.I, static_cast<const uint16_t*>(a.h), a.hq, a.h_scale, st, "quant_h");
         if (err != cudaSuccess) return err;
         hA = a.hq;
     }
@@ -1485,17 +1744,54 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
     if (swap2)
         return fp8 ? launch_swap<true, false>(tb, ta, ta, p, st, "gemm2_tc")
                    : launch_swap<false, false>(tb, ta, ta, p, st, "gemm2_tc");
-    if (wide2)
-        return fp8 ? launch_pair<true, false, 256, 2>(ta, tb, ta, p, st, "gemm2_tc")
-                   : launch_pair<false, false, 256, 2>(ta, tb, ta, p, st, "gemm2_tc");
-    if (two_sm)
-        return fp8 ? launch_pair<true, false, 256, 1>(ta, tb, ta, p, st, "gemm2_tc")
-                   : launch_pair<false, false, 256, 1>(ta, tb, ta, p, st, "gemm2_tc");
-    if (fp8)
-        return pair ? launch_one<true, false, 256, true>(ta, tb, ta, p, st, "gemm2_tc")
-                    : launch_one<true, false, 256, false>(ta, tb, ta, p, st, "gemm2_tc");
-    return pair ? launch_one<false, false, 256, true>(ta, tb, ta, p, st, "gemm2_tc")
-                : launch_one<false, false, 256, false>(ta, tb, ta, p, st, "gemm2_tc");
+    // the weighted combine folded into the shared expert's units (its group is
+    // the last one, rows = tokens in order): the kernels below, with scaled-fp16
+    // rows and a layer output to write
+    const bool fold = a.fold_out != nullptr && a.yexp != nullptr && a.fold_ready != nullptr &&
+                      direct_e == a.E - 1;
+    if (fold) {
+        p.fold_e = direct_e;
+        p.fold_S = a.S;
+        p.fold_inv = a.fold_inv;
+        p.fold_w = a.fold_w;
+        p.fold_out = a.fold_out;
+        p.fold_out_f32 = a.fold_out_f32;
+        p.ready = a.fold_ready;
+        int cur = g_inject_fold.load();
+        while (cur > 0 && !g_inject_fold.compare_exchange_weak(cur, cur - 1)) {
+        }
+        if (cur > 0) {
+            p.fold_extra = 1;                 // the fold_e units wait for an arrival that never comes
+            p.wait_limit = 20ll << 20;
+        }
+        err = cudaMemsetAsync(a.fold_ready, 0, static_cast<size_t>(p.n_tiles_n) * sizeof(unsigned), st);
+        if (err != cudaSuccess) return err;
+    }
+    auto gemm2 = [&]() -> cudaError_t {
+        if (wide2)
+            return fp8 ? launch_pair<true, false, 256, 2>(ta, tb, ta, p, st, "gemm2_tc")
+                       : launch_pair<false, false, 256, 2>(ta, tb, ta, p, st, "gemm2_tc");
+        if (two_sm)
+            return fp8 ? launch_pair<true, false, 256, 1>(ta, tb, ta, p, st, "gemm2_tc")
+                       : launch_pair<false, false, 256, 1>(ta, tb, ta, p, st, "gemm2_tc");
+        if (fp8)
+            return pair ? launch_one<true, false, 256, true>(ta, tb, ta, p, st, "gemm2_tc")
+                        : launch_one<true, false, 256, false>(ta, tb, ta, p, st, "gemm2_tc");
+        return pair ? launch_one<false, false, 256, true>(ta, tb, ta, p, st, "gemm2_tc")
+                    : launch_one<false, false, 256, false>(ta, tb, ta, p, st, "gemm2_tc");
+    };
+    err = gemm2();
+    if (fold && err != cudaSuccess) {
+        // the cooperative launch was refused (the grid cannot be made co-resident):
+        // rows of every group, combined separately by the caller
+        cudaGetLastError();
+        p.fold_e = -1;
+        p.ready = nullptr;
+        p.fold_extra = 0;
+        return gemm2();
+    }
+    if (fold && err == cudaSuccess && a.folded != nullptr) *a.folded = true;
+    return err;
 }
 
 }  // namespace sre

@@ -37,7 +37,7 @@ cudaError_t launch_gather_rows(int R, int S, int H, int elem_bytes, const void* 
                                const int32_t* skip, cudaStream_t stream);
 // per-row E4M3 quantisation of bf16 rows
 cudaError_t launch_quant_rows(int rows, int cols, const uint16_t* in, uint8_t* codes,
-                              float* scales, cudaStream_t stream);
+                              float* scales, cudaStream_t stream, const char* name = "quant_rows");
 
 // ---- expert FFN, CUDA-core path (ffn_simt.cu)
 struct FfnArgs {
@@ -68,6 +68,15 @@ struct FfnArgs {
     int direct_e;                 // expert whose rows are tokens 0..T-1 in order (A read from
                                   // xt directly, not gathered), or -1
     int max_mtiles;               // upper bound of sum_e ceil(count_e / kTileM)
+    // moe_forward, fused layer: the weighted combine folded into GEMM2's units of
+    // the direct_e group (the last one) where the tensor-core GEMM2 supports it;
+    // *folded is set when it ran (the caller then skips the combine pass)
+    const int32_t* fold_inv;      // [T*S] flat slot -> row, or null (no fold)
+    const float* fold_w;          // [T*S] slot weights
+    void* fold_out;               // [T, H] layer output (bf16, or fp32 when fold_out_f32)
+    int fold_out_f32;
+    unsigned* fold_ready;         // [H / 256] per n-tile counters (zeroed by the launch)
+    bool* folded;
     DevStatus* status;
 };
 cudaError_t launch_ffn_simt(const FfnArgs& a, cudaStream_t stream);
@@ -84,6 +93,10 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t stream);
 // testing hook: the next n grouped-FFN calls on the tensor-core path run with a
 // producer that never issues its loads and a ~10 ms wait limit
 void ffn_tc_inject_stall(int n_calls);
+// testing hook: in the next n calls that fold the weighted combine into GEMM2,
+// the shared expert's units wait for one routed arrival more than there will
+// be, with a ~10 ms wait limit
+void ffn_tc_inject_fold_stall(int n_calls);
 
 // ---- combine (combine.cu)
 // out[t] = sum_k w[t,k] * y[inv[t*S+k]] (+ add_w * add[t] if add != null)

@@ -347,9 +347,9 @@ cudaError_t launch_gather_rows(int R, int S, int H, int elem_bytes, const void* 
 }
 
 cudaError_t launch_quant_rows(int rows, int cols, const uint16_t* in, uint8_t* codes,
-                              float* scales, cudaStream_t stream) {
+                              float* scales, cudaStream_t stream, const char* name) {
     if (rows == 0) return cudaSuccess;
-    ProfileScope ps("quant_rows", stream);
+    ProfileScope ps(name, stream);
     quant_rows_kernel<<<ceil_div(rows * 32, 256), 256, 0, stream>>>(rows, cols, in, codes, scales);
     note_launch();
     return cudaGetLastError();

@@ -291,11 +291,36 @@ __device__ __forceinline__ void mma_commit_pair(uint64_t* bar, uint16_t cta_mask
         : "memory");
 }
 
-// ------------------------------------------------------------------ global reductions
-// out[0..3] += v (fp32, relaxed, performed at L2); out must be 16-byte aligned
-__device__ __forceinline__ void red_add_v4(float* out, float a, float b, float c, float d) {
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(out), "f"(a), "f"(b), "f"(c), "f"(d)
-                 : "memory");
+// ------------------------------------------------------------------ counters across CTAs
+// 32-bit load with acquire semantics at GPU scope
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// *p += v with release semantics at GPU scope
+__device__ __forceinline__ void red_release_gpu_add(unsigned* p, unsigned v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Waits until *p >= target, bounded like mbar_wait: gives up after
+// `limit_cycles` SM clock cycles or when another role has raised `*abort`, then
+// raises *abort, reports MOE_ERR_TIMEOUT with `site` and returns false.
+__device__ __forceinline__ bool counter_wait(const unsigned* p, unsigned target, volatile int* abort,
+                                             long long limit_cycles, DevStatus* st, unsigned site) {
+    if (ld_acquire_gpu(p) >= target) return true;
+    const long long t0 = clock64();
+    while (true) {
+        __nanosleep(200);
+        if (ld_acquire_gpu(p) >= target) return true;
+        if (*abort) return false;
+        if (clock64() - t0 > limit_cycles) {
+            *abort = 1;
+            report(st, MOE_ERR_TIMEOUT, site);
+            return false;
+        }
+    }
 }
 
 // ------------------------------------------------------------------ descriptors

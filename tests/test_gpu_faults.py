@@ -31,3 +31,26 @@ def test_wait_timeout_is_reported_and_the_context_survives(impl, I):
     ref = oracle.Layer(cfg, inp).forward()["out"]
     assert rel_err(to_f64(out), ref) <= tol_of(cfg)
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("impl,T", [(_lib.MOE_FFN_AUTO, 64), (_lib.MOE_FFN_AUTO, 1100),
+                                    (_lib.MOE_FFN_TCGEN05_PAIR, 64)],
+                         ids=["single_cta", "cta_pair_wide", "cta_pair"])
+def test_folded_combine_wait_timeout_is_reported(impl, T):
+    """The shared expert's down-projection units wait for the routed units of
+    their columns before aggregating; with one arrival too many expected the
+    wait runs out (~10 ms), the kernel drains and returns MOE_ERR_TIMEOUT, and
+    the next pass is clean and right."""
+    build.build()
+    cfg = synth.variant(synth.CONFIGS["prefill_bf16"], T=T, H=1024, I=256, n_routed=8, top_k=4)
+    inp = synth.make_inputs(cfg)
+    d = synth.to_device(inp, "cuda")
+    layer = MoELayer(cfg, d, impl=impl | _lib.MOE_FFN_COMBINE_FOLD)
+    _lib.moe_inject_fold_timeout(1)
+    layer.forward(d["x"])
+    assert layer.status() == _lib.MOE_ERR_TIMEOUT
+    out = layer.forward(d["x"])
+    assert layer.status() == _lib.MOE_OK
+    ref = oracle.Layer(cfg, inp).forward()["out"]
+    assert rel_err(to_f64(out), ref) <= tol_of(cfg)
+    torch.cuda.synchronize()

@@ -9,7 +9,7 @@ import torch
 
 import oracle
 from shared_routed_expert_b200 import MOE_FFN_AUTO, MOE_FFN_SIMT, MoELayer, _lib, build, synth
-from tests.parity_util import oracle_logits, rel_err, sample_tokens, to_f64, tol_of
+from tests.parity_util import full_size_sample, oracle_logits, rel_err, to_f64, tol_of
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -100,10 +100,17 @@ def test_zero_router_routes_everything_to_the_lowest_ids():
 WORKLOADS = ["prefill_bf16", "decode_bf16", "prefill_fp8", "skewed_fp8"]
 
 
+# tokens whose outputs are compared with the oracle at full size (decode: all)
+FULL_SAMPLE = {"prefill_bf16": 256, "decode_bf16": 64, "prefill_fp8": 128, "skewed_fp8": 256}
+
+
 @pytest.mark.parametrize("name", WORKLOADS)
 def test_full_size_workload(name):
     """The benchmark's workloads at full size: routing of every token bit-exact,
-    outputs of sampled tokens within tolerance, properties on all tokens."""
+    outputs of sampled tokens within tolerance, properties on all tokens. The
+    sample covers every 208-token block of the shared expert's group (its
+    GEMM1 work units on the bench workload) and 256-token block (its GEMM2
+    units), and the first and last units of the 10 largest routed groups."""
     cfg = synth.CONFIGS[name]
     d = synth.make_inputs(cfg, DEV)
     s = _lib.make_shape(cfg)
@@ -121,7 +128,9 @@ def test_full_size_workload(name):
     assert np.allclose(w.cpu().numpy(), rw, rtol=2e-6, atol=1e-7)
     # outputs on sampled tokens
     host = synth.to_host(d)
-    tok = sample_tokens(cfg.T, 6 if cfg.T > 1024 else 10)
+    tok = full_size_sample(cfg.T, rid, cfg.n_routed, FULL_SAMPLE[name])
+    if cfg.T <= 4096:
+        assert np.all(np.diff(tok // 208) <= 1) and np.all(np.diff(tok // 256) <= 1)
     ref = oracle.Layer(cfg, host).forward(tokens=tok)
     got = to_f64(out)[tok]
     assert np.all(np.isfinite(to_f64(out)))
@@ -148,9 +157,72 @@ def test_launch_counter_and_profile():
     layer.forward(d["x"])
     _lib.moe_profile_enable(False)
     torch.cuda.synchronize()
-    assert _lib.moe_launch_count() - n0 >= 6
+    assert _lib.moe_launch_count() - n0 >= 5
     n, ms = _lib.moe_profile_read("combine")
     assert n == 1 and ms > 0
+    # with the aggregation folded into the down-projection there is no combine pass
+    _lib.moe_profile_reset()
+    _lib.moe_profile_enable(True)
+    MoELayer(cfg, d, impl=_lib.MOE_FFN_COMBINE_FOLD).forward(d["x"])
+    _lib.moe_profile_enable(False)
+    torch.cuda.synchronize()
+    assert _lib.moe_profile_read("combine")[0] == 0 and _lib.moe_profile_read("gemm2_tc")[0] == 1
+
+
+# Layers whose down-projection runs each tensor-core kernel family with the
+# aggregation folded in: single-CTA 128-row units (bf16, E4M3), single-CTA
+# 256-row units, CTA pairs with 256 x 256 and 256 x 512 tiles.
+FOLD_CASES = {
+    "bf16_small": (SMALL["bf16_small"], MOE_FFN_AUTO),
+    "fp8_small": (SMALL["fp8_small"], MOE_FFN_AUTO),
+    "fp8_i192_zipf": (SMALL["fp8_i192_zipf"], MOE_FFN_AUTO),
+    "routed_scale": (SMALL["routed_scale"], MOE_FFN_AUTO),
+    "shared_w_half": (SMALL["shared_w_half"], MOE_FFN_AUTO),
+    "bf16_m256": (SMALL["bf16_small"], _lib.MOE_FFN_TCGEN05_M256),
+    "fp8_m256": (SMALL["fp8_small"], _lib.MOE_FFN_TCGEN05_M256),
+    "bf16_pair": (SMALL["bf16_small"], _lib.MOE_FFN_TCGEN05_PAIR),
+    "bf16_big_groups": (synth.variant(synth.CONFIGS["prefill_bf16"], T=1100, H=1024, I=256, n_routed=8,
+                                      top_k=4), MOE_FFN_AUTO),
+    "fp8_pair_wide": (synth.variant(synth.CONFIGS["prefill_fp8"], T=700, H=1024, I=256, n_routed=8, top_k=4),
+                      _lib.MOE_FFN_TCGEN05_WIDE),
+}
+
+
+@pytest.mark.parametrize("name", list(FOLD_CASES))
+def test_folded_combine_equals_the_separate_pass(name):
+    """NEXT-4: the weighted aggregation inside the down-projection's shared-expert
+    units gives the output of the separate combine pass bit for bit (same fp32
+    operations in slot order), and the oracle's within tolerance."""
+    cfg, impl = FOLD_CASES[name]
+    inp = synth.make_inputs(cfg)
+    d = synth.to_device(inp, DEV)
+    _lib.moe_profile_reset()
+    _lib.moe_profile_enable(True)
+    folded = _run(cfg, d, True, impl | _lib.MOE_FFN_COMBINE_FOLD)
+    assert _lib.moe_profile_read("combine")[0] == 0        # the fold ran
+    sep = _run(cfg, d, True, impl)
+    assert _lib.moe_profile_read("combine")[0] == 1
+    _lib.moe_profile_enable(False)
+    assert np.array_equal(folded.view(np.uint64), sep.view(np.uint64))
+    ref = oracle.Layer(cfg, inp).forward()
+    assert rel_err(folded, ref["out"]) <= tol_of(cfg)
+
+
+def test_folded_combine_writes_fp32_shares():
+    """With out_f32 (a tensor-parallel rank's unrounded share) the folded
+    aggregation writes the same fp32 bits as the separate pass."""
+    cfg = synth.variant(synth.CONFIGS["prefill_bf16"], T=300, H=512, I=128, n_routed=16, top_k=4, out_f32=True)
+    d = synth.to_device(synth.make_inputs(cfg), DEV)
+    s = _lib.make_shape(cfg)
+    ws = _lib.alloc_workspace(s, True)
+    outs = []
+    for impl in (_lib.MOE_FFN_COMBINE_FOLD, MOE_FFN_AUTO):
+        o = torch.full((cfg.T, cfg.H), float("nan"), dtype=torch.float32, device=DEV)
+        _lib.moe_forward(s, d["x"], d["router_w"], d["router_bias"], d["w13"], d.get("s13"), d["w2"],
+                         d.get("s2"), True, o, ws, impl=impl)
+        assert _lib.moe_get_status(ws) == _lib.MOE_OK
+        outs.append(o)
+    assert torch.equal(outs[0].view(torch.int32), outs[1].view(torch.int32))
 
 
 @pytest.mark.parametrize("name", ["bf16_small", "fp8_i192_zipf"])
