@@ -624,20 +624,27 @@ def measure(cfg, args, dist: Dist, impl: int, quick: bool = False, want_host: bo
     def step():
         fused.forward(d["x"], out)
 
-    # timed region: device-resident inputs, per-kernel events on the launching stream
+    # timed region: device-resident inputs, the layer's kernels back to back with
+    # nothing between them (a kernel may start while its predecessor finishes)
     vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
     clocks = Clocks(vis.split(",")[dist.local] if vis else str(dist.local))
-    _lib.moe_profile_reset()
-    _lib.moe_profile_enable(True)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    _lib.moe_profile_reset()
     n0 = _lib.moe_launch_count()
     clocks.start()
     ms = time_steps(step, args.steps, 0, dist, stream)
     clk = clocks.stop()
     launches = _lib.moe_launch_count() - n0
+    # per-kernel durations: a second pass of as many steps with CUDA events
+    # around every launch on the launching stream (these serialise the kernels)
+    _lib.moe_profile_reset()
+    _lib.moe_profile_enable(True)
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    _lib.moe_profile_reset()
+    time_steps(step, args.steps, 0, dist, stream)
     _lib.moe_profile_enable(False)
     tab = kernel_table(args.steps)
     st = fused.status()
@@ -669,12 +676,15 @@ def measure(cfg, args, dist: Dist, impl: int, quick: bool = False, want_host: bo
         ms_unf = ms_fused_il = ms_sep = 0.0
         for _ in range(n_blocks):
             ms_fused_il += time_steps(step, per, 0, dist, stream)
-            _lib.moe_profile_enable(True)
             ms_unf += time_steps(lambda: unfused.forward(d["x"], out), per, 0, dist, stream)
-            _lib.moe_profile_enable(False)
             ms_sep += time_steps(lambda: separate.forward(d["x"], out), per, 0, dist, stream)
-        tab_unf = kernel_table(n_blocks * per)
         unf_steps = n_blocks * per
+        # the unfused layer's per-kernel durations, in a pass of its own with events
+        _lib.moe_profile_reset()
+        _lib.moe_profile_enable(True)
+        time_steps(lambda: unfused.forward(d["x"], out), unf_steps, 0, dist, stream)
+        _lib.moe_profile_enable(False)
+        tab_unf = kernel_table(unf_steps)
         for lay, what in ((unfused, "unfused"), (separate, "folded combine")):
             st = lay.status()
             if st != _lib.MOE_OK:

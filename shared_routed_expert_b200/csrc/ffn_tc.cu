@@ -258,11 +258,8 @@ __device__ __forceinline__ void epilogue_rows(const TcParams& p, const TileInfo&
         }
         if (p.yexp != nullptr && valid) {
             int8_t* e = p.yexp + static_cast<size_t>(row) * (p.H / 32) + t.n0 / 32 + c_begin;
-            const int n = c_end - c_begin;
-            if (n == 8) *reinterpret_cast<uint64_t*>(e) = exps;
-            else if (n == 4) *reinterpret_cast<uint32_t*>(e) = static_cast<uint32_t>(exps);
-            else
-                for (int i = 0; i < n; ++i) e[i] = static_cast<int8_t>((exps >> (8 * i)) & 0xFFu);
+            if (c_end - c_begin == 8) *reinterpret_cast<uint64_t*>(e) = exps;
+            else *reinterpret_cast<uint32_t*>(e) = static_cast<uint32_t>(exps);
         }
     }
 }
@@ -312,20 +309,19 @@ __device__ __forceinline__ void fold_fma(const uint4& q, float wgt, float (&acc)
 }
 
 // The combine of one warp's 32 rows (unit rows wrow0 .. +31, tokens wrow0 -
-// grp0 ..) over columns [col0, col0 + ncols), ncols a multiple of 128; this warp
-// takes work items item0, item0 + istride, ... Work item i = (token pair i % 16,
-// 128-column block i / 16); lanes 0-15 take the pair's first token, 16-31 its
-// second, 8 columns per lane; the loads of FOLD_SLOTS slot rows are in flight
-// together.
+// grp0 ..) over columns [col0, col0 + ncols), ncols a multiple of 128. Work item
+// i = (token pair i % 16, 128-column block i / 16); lanes 0-15 take the pair's
+// first token, 16-31 its second, 8 columns per lane; the loads of FOLD_SLOTS
+// slot rows are in flight together.
 __device__ __forceinline__ void fold_combine(const TcParams& p, int row_end, int lane, int wrow0, int grp0,
-                                             int col0, int ncols, int item0, int istride) {
+                                             int col0, int ncols) {
     const int S = p.fold_S;
     const int ne = p.H / 32;
     const int items = 16 * (ncols >> 7);
     const int half = lane >> 4;
     const int cl = (lane & 15) * 8;
 #pragma unroll 1
-    for (int it = item0; it < items; it += istride) {
+    for (int it = 0; it < items; ++it) {
         const int row = wrow0 + 2 * (it % 16) + half;
         const int col = col0 + (it / 16) * 128 + cl;
         if (row >= row_end) continue;
@@ -387,35 +383,20 @@ __device__ __forceinline__ bool fold_wait(const TcParams& p, int nt, unsigned ta
 // columns in two halves (two warps per TMEM sub-partition).
 // kRowB: bytes of K per row per stage (128: 128-byte swizzle; 64: 64-byte swizzle,
 // twice as many stages of half the size).
-// Epilogue warps of the single-CTA kernel: 12 (three per TMEM lane group) for
-// the E4M3 down-projection on 128-row units, whose epilogue (per-row and
-// per-column scales, scaled-fp16 rows) is the slowest part of its unit; 8 else
-#ifndef SRE_E4M3_EPI12
-#define SRE_E4M3_EPI12 0
-#endif
-template <bool kFp8, bool kGemm1, bool kPair>
-constexpr int gg_epi_warps() {
-    return (SRE_E4M3_EPI12 && kFp8 && !kGemm1 && !kPair) ? 12 : 8;
-}
-
-template <int kRowB, int kBN, bool kPair, int kEpiW>
+template <int kRowB, int kBN, bool kPair>
 struct Ring {
     static constexpr int A_TILE = TC_BM * kRowB;
     static constexpr int STAGE = (kPair ? 2 : 1) * A_TILE + kBN * kRowB;
     static constexpr int N = (TC_RING_BYTES / STAGE) > 8 ? 8 : (TC_RING_BYTES / STAGE);
-    // weight-scale area per epilogue warp: 256 floats, or 128 with 12 warps (three
-    // chunks of 32 columns each at most)
-    static constexpr int SCALE_B = kEpiW == 12 ? 512 : 1024;
-    // + epilogue staging (2 KB per warp), weight scales, alignment
-    static constexpr int SMEM = N * STAGE + kEpiW * 2048 + kEpiW * SCALE_B + 1024;
+    // + epilogue staging (2 KB per warp), weight scales (1 KB per warp), alignment
+    static constexpr int SMEM = N * STAGE + 8 * 2048 + 8 * 1024 + 1024;
 };
 
 template <bool kFp8, bool kGemm1, int kBN, bool kPair, int kRowB>
-__global__ void __launch_bounds__((2 + gg_epi_warps<kFp8, kGemm1, kPair>()) * 32, 1)
+__global__ void __launch_bounds__(320, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmA2, const TcParams p) {
-    constexpr int EPI_WARPS = gg_epi_warps<kFp8, kGemm1, kPair>();
-    using RG = Ring<kRowB, kBN, kPair, EPI_WARPS>;
+    using RG = Ring<kRowB, kBN, kPair>;
     constexpr int NSTAGE = RG::N;
     constexpr int TC_ABYTES = RG::A_TILE;           // one 128-row A tile per stage
     constexpr int ABYTES = (kPair ? 2 : 1) * TC_ABYTES;
@@ -423,11 +404,11 @@ __global__ void __launch_bounds__((2 + gg_epi_warps<kFp8, kGemm1, kPair>()) * 32
     constexpr int HALF = kBN / 2;
     constexpr int KEL = kFp8 ? kRowB : kRowB / 2;   // K elements per stage
     constexpr int KSTEPS = kRowB / 32;              // MMAs (32 bytes of K each) per stage
+    constexpr int EPI_WARPS = 8;
     constexpr uint32_t IDESC = ptx::instr_desc(TC_BM, kBN, kFp8 ? 0u : 1u);
 
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t full_bar[NSTAGE], empty_bar[NSTAGE], tfull_bar[2], tempty_bar[2], drain_bar;
-    __shared__ uint64_t fold_bar[4];   // per TMEM lane group: its epilogue warps' rows of a unit are stored
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
     __shared__ int s_off[TC_MAXE], s_unit[TC_MAXE];
@@ -438,7 +419,7 @@ __global__ void __launch_bounds__((2 + gg_epi_warps<kFp8, kGemm1, kPair>()) * 32
     uint8_t* sA = base;
     uint8_t* sB = base + NSTAGE * ABYTES;
     uint8_t* sStage = sB + NSTAGE * BBYTES;         // EPI_WARPS x 2 KB
-    float* sScale = reinterpret_cast<float*>(sStage + EPI_WARPS * 2048);   // EPI_WARPS x RG::SCALE_B (E4M3 weight scales)
+    float* sScale = reinterpret_cast<float*>(sStage + EPI_WARPS * 2048);   // EPI_WARPS x 1 KB (E4M3 weight scales)
     volatile int* abort_flag = &s_abort;
 
     for (int i = threadIdx.x; i <= p.E; i += blockDim.x) s_off[i] = p.offsets[i];
@@ -471,7 +452,6 @@ __global__ void __launch_bounds__((2 + gg_epi_warps<kFp8, kGemm1, kPair>()) * 32
             ptx::mbar_init(&tfull_bar[b], 1);
             ptx::mbar_init(&tempty_bar[b], EPI_WARPS * 32);
         }
-        for (int g = 0; g < 4; ++g) ptx::mbar_init(&fold_bar[g], EPI_WARPS / 4);
         ptx::mbar_init(&drain_bar, 1);
         s_abort = 0;
         ptx::fence_mbar_init();
@@ -597,16 +577,14 @@ __global__ void __launch_bounds__((2 + gg_epi_warps<kFp8, kGemm1, kPair>()) * 32
     } else {
         // ---------------------------------------------------------------- epilogue
         const int sub = warp & 3;                  // TMEM lanes 32*sub .. +31
-        constexpr int EG = EPI_WARPS / 4;          // epilogue warps per TMEM lane group
-        const int eg = (warp - 2) >> 2;            // pair: accumulator; single: column share
+        const int eg = (warp - 2) >> 2;            // pair: accumulator; single: column half
         const int r_local = (kPair ? eg * TC_BM : 0) + sub * 32 + lane;
         constexpr int NCH = kGemm1 ? HALF / 32 : kBN / 32;   // 32-column chunks per unit
-        constexpr int PER = kPair ? NCH : (NCH + EG - 1) / EG;
+        constexpr int PER = kPair ? NCH : (NCH + 1) / 2;
         const int c_begin = kPair ? 0 : eg * PER;
         const int c_end = kPair ? NCH : min(NCH, c_begin + PER);
         int acc = 0;
         uint32_t acc_phase = 0;
-        uint32_t fold_phase = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
             const TileInfo t = decode_unit<kPair>(tile, s_unit, s_off, p.E, p.n_tiles_n, p.bn_out);
             // one lane waits and the warp takes its result: tcgen05.ld below needs the whole warp
@@ -629,7 +607,7 @@ __global__ void __launch_bounds__((2 + gg_epi_warps<kFp8, kGemm1, kPair>()) * 32
                 // 16-bit outputs leave through this warp's 2 KB staging slice so that
                 // global stores cover whole 64-byte row segments (see stage_store)
                 uint8_t* stage_w = sStage + (warp - 2) * 2048;
-                float* scs = sScale + (warp - 2) * (RG::SCALE_B / 4);
+                float* scs = sScale + (warp - 2) * 256;
                 if constexpr (kFp8) stage_scales<kGemm1>(p, t, c_begin, c_end, scs, lane);
                 epilogue_rows<kFp8, kGemm1, kBN>(p, t, tb, c_begin, c_end, stage_w, lane, row, valid, rs, wrow0, scs);
             }
@@ -643,24 +621,7 @@ __global__ void __launch_bounds__((2 + gg_epi_warps<kFp8, kGemm1, kPair>()) * 32
                     static_cast<unsigned>(s_unit[p.E] - (s_unit[p.fold_e + 1] - s_unit[p.fold_e])) * EPI_WARPS +
                     p.fold_extra;
                 if (!fold_wait(p, t.n0 / p.bn_out, target, abort_flag, lane)) break;
-                if constexpr (EG == 2 || kPair) {
-                    fold_combine(p, t.row_end, lane, wrow0, s_off[t.e], t.n0 + c_begin * 32, (c_end - c_begin) * 32,
-                                 0, 1);
-                } else {
-                    // the lane group's warps share its rows: all of their stores are done
-                    // before any of them sums (a bounded wait on the group's barrier), and
-                    // they take its 128-column blocks in turn
-                    __syncwarp();
-                    int ok2 = 1;
-                    if (lane == 0) {
-                        ptx::mbar_arrive(&fold_bar[sub]);
-                        ok2 = ptx::mbar_wait(&fold_bar[sub], fold_phase, abort_flag, p.wait_limit, p.status, 6u);
-                    }
-                    ok2 = __shfl_sync(0xFFFFFFFFu, ok2, 0);
-                    fold_phase ^= 1u;
-                    if (!ok2) break;
-                    fold_combine(p, t.row_end, lane, wrow0, s_off[t.e], t.n0, kBN, eg, EG);
-                }
+                fold_combine(p, t.row_end, lane, wrow0, s_off[t.e], t.n0 + c_begin * 32, (c_end - c_begin) * 32);
             }
             if constexpr (kPair) {
                 acc_phase ^= 1u;
@@ -967,7 +928,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
                     if (lane == 0) ptx::st_remote_u32(peer_abort, 1u);
                     break;
                 }
-                fold_combine(p, t.row_end, lane, wrow0, s_off[t.e], t.n0 + c_begin * 32, (c_end - c_begin) * 32, 0, 1);
+                fold_combine(p, t.row_end, lane, wrow0, s_off[t.e], t.n0 + c_begin * 32, (c_end - c_begin) * 32);
             }
             if constexpr (kNSUB == 1) {
                 acc ^= 1;
@@ -1497,8 +1458,7 @@ template <bool kFp8, bool kGemm1, int kBN, bool kPair>
 cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2, const TcParams& p,
                        cudaStream_t st, const char* name) {
     constexpr int kRowB = SRE_STAGE_ROW_BYTES;
-    constexpr int kEpiW = gg_epi_warps<kFp8, kGemm1, kPair>();
-    constexpr int smem = Ring<kRowB, kBN, kPair, kEpiW>::SMEM;
+    constexpr int smem = Ring<kRowB, kBN, kPair>::SMEM;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
@@ -1507,8 +1467,8 @@ cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const CUtenso
     });
     if (attr_err != cudaSuccess) return attr_err;
     ProfileScope ps(name, st);
-    const cudaError_t err = launch_grid(grouped_gemm_kernel<kFp8, kGemm1, kBN, kPair, kRowB>, num_sms(),
-                                        (2 + kEpiW) * 32, smem, p.fold_e >= 0, st, a, b, a2, p);
+    const cudaError_t err = launch_grid(grouped_gemm_kernel<kFp8, kGemm1, kBN, kPair, kRowB>, num_sms(), 320, smem,
+                                        p.fold_e >= 0, st, a, b, a2, p);
     note_launch();
     return err;
 }
