@@ -428,12 +428,17 @@ def bench_tp(args, dist):
 
 
 def bench_qk_norm_rope(args, dist):
+    line = measure_qk_norm_rope(synth.ATTN_CONFIGS[args.attn_workload], args, dist)
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def measure_qk_norm_rope(cfg, args, dist) -> dict:
     """The fused QK-norm + partial RoPE kernel on its own: tokens/s from the
     kernel's CUDA events (L2 flushed between launches by an untimed 256 MB
     read, which leaves no dirty lines to write back during the kernel), rated
     against the measured HBM copy peak; e2e uploads qkv and downloads it every
     step."""
-    cfg = synth.ATTN_CONFIGS[args.attn_workload]
     inp = synth.make_attn_inputs(cfg, dist.device)
     stream = torch.cuda.current_stream()
     flush = torch.ones(64 << 20, dtype=torch.float32, device=dist.device)
@@ -490,8 +495,7 @@ def bench_qk_norm_rope(args, dist):
                      "algorithmic_bytes": nbytes},
         "clocks": clk,
     }
-    if dist.rank == 0:
-        print(json.dumps(line), flush=True)
+    return line
 
 
 def main():
@@ -595,6 +599,12 @@ def main():
             wm.pop("host", None)
             line["workloads"][name] = entry
             del wm
+            torch.cuda.empty_cache()
+        # the attention-side step the pages fuse (QK-norm + partial RoPE), prefill and decode
+        for name in ("qknorm_prefill", "qknorm_decode"):
+            q = measure_qk_norm_rope(synth.ATTN_CONFIGS[name], args, dist)
+            line["workloads"][name] = {k: q[k] for k in ("metric", "value", "unit", "ms_per_step", "steps", "config",
+                                                          "e2e", "gpu_launches", "roofline", "clocks")}
             torch.cuda.empty_cache()
     if dist.rank == 0:
         print(json.dumps(line), flush=True)

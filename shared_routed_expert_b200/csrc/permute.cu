@@ -259,8 +259,23 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(int R, int S, int row_
     if (xscale != nullptr && lane == 0) xpscale[r] = xscale[t];
 }
 
+// v / s correctly rounded, from y = RN(1 / s): Markstein's theorem (P. Markstein,
+// "Computation of elementary functions on the IBM RISC System/6000 processor",
+// IBM J. Res. Dev. 34(1), 1990): q0 = RN(v y) lies within an ulp of v / s, the
+// residual v - s q0 is then exact (one fma), and RN(q0 + r y) = RN(v / s),
+// provided no intermediate underflows or overflows.
+__device__ __forceinline__ float div_by_recip(float v, float s, float y) {
+    const float q0 = __fmul_rn(v, y);
+    const float r = __fmaf_rn(-q0, s, v);
+    return __fmaf_rn(r, y, q0);
+}
+
 // One warp per row: amax (fp32), scale = amax / 448 (IEEE divide, amax = 0 -> 1),
-// codes = E4M3_rn_satfinite(v / scale) (IEEE divide).
+// codes = E4M3_rn_satfinite(v / scale) with the quotient rounded as the IEEE
+// divide rounds it: by div_by_recip when amax >= 2^-60 (then every quotient of
+// 2^-11 or more, the only ones whose code depends on its last bit, has a normal
+// residual; smaller ones are codes of +-0 either way), by the divide otherwise.
+constexpr float kMarksteinMinAmax = 8.6736174e-19f;    // 2^-60
 __global__ void __launch_bounds__(256) quant_rows_kernel(int rows, int cols,
                                                          const uint16_t* __restrict__ in,
                                                          uint8_t* __restrict__ codes,
@@ -283,6 +298,8 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(int rows, int cols,
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
     const float scale = (amax > 0.0f) ? __fdiv_rn(amax, 448.0f) : 1.0f;
+    const bool by_recip = amax >= kMarksteinMinAmax && amax <= 3.4028235e38f;     // warp-uniform
+    const float y = by_recip ? __frcp_rn(scale) : 0.0f;
     uint2* dst = reinterpret_cast<uint2*>(codes + static_cast<size_t>(r) * cols);
     for (int i = lane; i < nv; i += 32) {
         const uint4 q = src[i];
@@ -290,8 +307,9 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(int rows, int cols,
         uint32_t packed[2] = {0u, 0u};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const uint32_t lo = f32_to_e4m3(__fdiv_rn(__uint_as_float(w[j] << 16), scale));
-            const uint32_t hi = f32_to_e4m3(__fdiv_rn(__uint_as_float(w[j] & 0xFFFF0000u), scale));
+            const float a = __uint_as_float(w[j] << 16), b = __uint_as_float(w[j] & 0xFFFF0000u);
+            const uint32_t lo = f32_to_e4m3(by_recip ? div_by_recip(a, scale, y) : __fdiv_rn(a, scale));
+            const uint32_t hi = f32_to_e4m3(by_recip ? div_by_recip(b, scale, y) : __fdiv_rn(b, scale));
             packed[j >> 1] |= (lo | (hi << 8)) << ((j & 1) * 16);
         }
         dst[i] = make_uint2(packed[0], packed[1]);

@@ -194,6 +194,36 @@ def test_quant_rows_e4m3_bit_exact():
     assert np.array_equal(codes.cpu().numpy(), rc)
 
 
+@pytest.mark.parametrize("cols", [1536, 5120])
+def test_quant_rows_e4m3_wide_magnitude_sweep_bit_exact(cols):
+    """The quotient v / scale is formed from a correctly rounded reciprocal of the
+    row's scale (Markstein's refinement) when the row's amax is at least 2^-60,
+    by the IEEE divide below that; either way every code must equal the
+    oracle's (IEEE fp32 divide, then E4M3 round-to-nearest-even with
+    saturation). Rows with amax from 1e-37 to 1e37 (both sides of 2^-60),
+    including bf16 subnormals and signed zeros; rows of 1536 and 5120 columns
+    (the h and x rows of the workloads)."""
+    g = torch.Generator().manual_seed(11)
+    n = 160
+    mags = torch.logspace(-37, 37, n)
+    rows = torch.randn(n, cols, generator=g) * mags.unsqueeze(1)
+    rows[::7, ::3] *= torch.rand(rows[::7, ::3].shape, generator=g) * 1e-6      # tiny values beside large ones
+    rows[3, :] = 0.0
+    rows[4, ::2] = -0.0
+    rows[5, :64] = torch.tensor(2.0 ** -133)                                   # bf16 subnormals
+    t = 2.0 ** -60
+    rows[6] = torch.randn(cols, generator=g) * t * 0.5                          # just under the threshold
+    rows[7] = torch.randn(cols, generator=g) * t * 2.0                          # just over
+    rows = rows.to(torch.bfloat16)
+    codes = torch.empty(n, cols, dtype=torch.uint8, device=DEV)
+    scales = torch.empty(n, dtype=torch.float32, device=DEV)
+    _lib.moe_quant_rows_e4m3(n, cols, rows.to(DEV), codes, scales)
+    torch.cuda.synchronize()
+    rc, rs = oracle.quant_rows_e4m3(rows.float().numpy())
+    assert np.array_equal(scales.cpu().numpy().view(np.uint32), rs.view(np.uint32))
+    assert np.array_equal(codes.cpu().numpy(), rc)
+
+
 def test_quant_rows_e4m3_midpoints_bit_exact():
     """Rows whose quotients v / scale fall exactly on E4M3 rounding midpoints (and
     one bf16 step either side): amax = 448 * m with m = 1.5, 1.25, 1.75 makes the
