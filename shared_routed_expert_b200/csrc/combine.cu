@@ -20,7 +20,7 @@ namespace sre {
 namespace {
 
 constexpr int CB_THREADS = 128;
-constexpr int CB_BATCH = 5;      // slot rows loaded together (S = 9: two groups)
+constexpr int CB_BATCH = 9;      // slot rows loaded together (S = 9: all at once)
 
 // bf16 rows: each thread owns 8-element vectors of the token's row.
 __global__ void __launch_bounds__(CB_THREADS) combine_bf16_kernel(int T, int S, int H,
