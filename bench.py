@@ -177,6 +177,20 @@ class Clocks:
 
 # ------------------------------------------------------------------ timing
 
+def emit(line: dict) -> None:
+    """Print one JSON line; a figure that was not measured (NaN, e.g. the unfused arm
+    under --quick) is written as null so that the line stays strict JSON."""
+    def clean(v):
+        if isinstance(v, float) and not math.isfinite(v):
+            return None
+        if isinstance(v, dict):
+            return {k: clean(x) for k, x in v.items()}
+        if isinstance(v, (list, tuple)):
+            return [clean(x) for x in v]
+        return v
+    print(json.dumps(clean(line), allow_nan=False), flush=True)
+
+
 def tokens_per_s(n_ranks: int, tokens_per_rank: int, steps: int, max_ms: float) -> float:
     """Whole-job throughput: every rank's tokens over the slowest rank's time."""
     return n_ranks * tokens_per_rank * steps / (max_ms / 1000.0)
@@ -390,7 +404,7 @@ def run_reference(args, dist: Dist):
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": used, "kind": "oracle",
                              "sample": f"{per_step} random tokens of {cfg.name} per step"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
-    print(json.dumps(line), flush=True)
+    emit(line)
 
 
 def describe(cfg) -> str:
@@ -424,13 +438,13 @@ def bench_tp(args, dist):
             "config": {"workload": describe(cfg), "parallelism": f"tp{N} (intermediate slices of {cfg.I // N}, "
                                                                "one fp32 all-reduce of [T, H] per layer)"}}
     if dist.rank == 0:
-        print(json.dumps(line), flush=True)
+        emit(line)
 
 
 def bench_qk_norm_rope(args, dist):
     line = measure_qk_norm_rope(synth.ATTN_CONFIGS[args.attn_workload], args, dist)
     if dist.rank == 0:
-        print(json.dumps(line), flush=True)
+        emit(line)
 
 
 def measure_qk_norm_rope(cfg, args, dist) -> dict:
@@ -607,7 +621,7 @@ def main():
                                                           "e2e", "gpu_launches", "roofline", "clocks")}
             torch.cuda.empty_cache()
     if dist.rank == 0:
-        print(json.dumps(line), flush=True)
+        emit(line)
     dist.close()
 
 

@@ -130,3 +130,13 @@ def test_gather_bytes_leave_out_the_shared_rows():
     c8 = synth.CONFIGS["skewed_fp8"]
     _, nb8 = bench.algorithmic(c8, "gather", None)
     assert nb8 == 4096 * 5120 + 32768 * 5120 + 32768 * 4 + 4096 * 4
+
+
+def test_unmeasured_figures_print_as_null(capsys):
+    import json
+
+    import bench
+    bench.emit({"value": 1.5, "unfused": {"ms_per_step": float("nan"), "x": [float("inf"), 2]}})
+    out = capsys.readouterr().out
+    assert json.loads(out) == {"value": 1.5, "unfused": {"ms_per_step": None, "x": [None, 2]}}
+    assert "NaN" not in out and "Infinity" not in out
