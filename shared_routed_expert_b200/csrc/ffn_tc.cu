@@ -55,6 +55,12 @@ constexpr int TC_MAXE = 260;
 constexpr uint32_t TC_TMEM_COLS = 512;
 
 struct TcParams {
+    // output rows leave by TMA stores through this map (16-bit elements, 32 x 32
+    // boxes, 64-byte swizzle: the staging slices' layout) when out_tma is set;
+    // the kernels take TcParams as a __grid_constant__ parameter so that the
+    // map's address is valid for the TMA unit
+    CUtensorMap tm_out;
+    int out_tma;
     int E, H, I;
     int n_tiles_n;          // n-tiles per m-tile
     int bn_out;             // output columns per n-tile (GEMM1: I columns; GEMM2: H columns)
@@ -117,18 +123,47 @@ __device__ __forceinline__ TileInfo decode_unit(int id, const int* s_unit, const
     return t;
 }
 
+// A warp's staging slice is free again: the TMA store that last read it (if
+// any; issued by lane 0, whose bulk groups these are) has read it.
+__device__ __forceinline__ void slice_acquire(const CUtensorMap* tm, int lane) {
+    if (tm != nullptr) {
+        if (lane == 0) ptx::bulk_wait_read_all();
+        __syncwarp();
+    }
+}
+
+// A whole 32 x 32 block staged in the slice (64-byte rows, 16-byte chunks
+// XOR-swizzled by (row >> 1) & 3: the TMA 64-byte swizzle) leaves by one TMA
+// store; the warp goes on while the TMA unit reads the slice.
+__device__ __forceinline__ void slice_tma_store(const CUtensorMap* tm, const uint8_t* slice, int lane, int row0,
+                                                int col0) {
+    ptx::fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        ptx::tma_store_2d(tm, slice, col0, row0);
+        ptx::bulk_commit();
+    }
+}
+
 // One warp's 32 rows x 32 columns of 16-bit results (lane = row, packed[] = its
 // 64 bytes) go to global memory through a 2 KB shared-memory slice: written
 // with the 16-byte chunks of row r XOR-swizzled by (r >> 1) & 3 (conflict-free),
-// read back so that 4 lanes cover one row's 64 contiguous bytes (8 rows per
-// instruction); rows at or past row_end are not stored.
+// then either stored by TMA (tm set and all 32 rows below row_end) or read
+// back so that 4 lanes cover one row's 64 contiguous bytes (8 rows per
+// instruction) and stored without the rows at or past row_end (those belong
+// to the next group).
 __device__ __forceinline__ void stage_store(uint8_t* slice, const uint32_t (&packed)[16], int lane, uint16_t* out,
-                                            int ld, int row0, int row_end, int col0) {
+                                            int ld, int row0, int row_end, int col0, const CUtensorMap* tm) {
+    slice_acquire(tm, lane);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         const int pc = q ^ ((lane >> 1) & 3);
         *reinterpret_cast<uint4*>(slice + lane * 64 + pc * 16) =
             make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+    }
+    if (tm != nullptr && row0 + 32 <= row_end) {
+        slice_tma_store(tm, slice, lane, row0, col0);
+        return;
     }
     __syncwarp();
 #pragma unroll
@@ -166,6 +201,15 @@ __device__ __forceinline__ void stage_scales(const TcParams& p, const TileInfo& 
     __syncwarp();
 }
 
+// max |a[j]| over 32 registers as four independent chains (max is exact, so
+// the order does not change the result; a single chain is 32 dependent steps)
+__device__ __forceinline__ float abs_max32(const float (&a)[32]) {
+    float m[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+    for (int j = 0; j < 32; ++j) m[j & 3] = fmaxf(m[j & 3], fabsf(a[j]));
+    return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+}
+
 // Epilogue of one unit for one warp: TMEM columns [c_begin, c_end) x 32 of the
 // lane group at `tb` (row = this lane's output row, valid if it is stored)
 // become bf16 h (GEMM1, SwiGLU applied) or bf16 / scaled-fp16 y rows (GEMM2),
@@ -175,6 +219,7 @@ __device__ __forceinline__ void epilogue_rows(const TcParams& p, const TileInfo&
                                               int c_end, uint8_t* stage_w, int lane, int row, bool valid,
                                               float rs, int wrow0, const float* scs) {
     constexpr int HALF = kBN / 2;
+    const CUtensorMap* tmo = p.out_tma ? &p.tm_out : nullptr;
     if constexpr (kGemm1) {
 #pragma unroll 1
         for (int c = c_begin; c < c_end; ++c) {
@@ -200,7 +245,7 @@ __device__ __forceinline__ void epilogue_rows(const TcParams& p, const TileInfo&
                 }
                 packed[j >> 1] = pack_bf16x2(silu_f32(g0) * u0, silu_f32(g1) * u1);
             }
-            stage_store(stage_w, packed, lane, p.out, p.out_ld, wrow0, t.row_end, t.n0 + c * 32);
+            stage_store(stage_w, packed, lane, p.out, p.out_ld, wrow0, t.row_end, t.n0 + c * 32, tmo);
         }
     } else {
         // chunk c's TMEM load is in flight while chunk c-1 is converted and stored
@@ -215,9 +260,7 @@ __device__ __forceinline__ void epilogue_rows(const TcParams& p, const TileInfo&
             }
             uint32_t packed[16];
             if (p.yexp != nullptr) {
-                float amax = 0.0f;
-#pragma unroll
-                for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(a[j]));
+                const float amax = abs_max32(a);
                 const int k = f16_chunk_exp(amax);
                 const float down = exp2_int(-k);
 #pragma unroll
@@ -227,7 +270,7 @@ __device__ __forceinline__ void epilogue_rows(const TcParams& p, const TileInfo&
 #pragma unroll
                 for (int j = 0; j < 32; j += 2) packed[j >> 1] = pack_bf16x2(a[j], a[j + 1]);
             }
-            stage_store(stage_w, packed, lane, p.out, p.out_ld, wrow0, t.row_end, t.n0 + c * 32);
+            stage_store(stage_w, packed, lane, p.out, p.out_ld, wrow0, t.row_end, t.n0 + c * 32, tmo);
         };
         if constexpr (kFp8) {
             // E4M3: one chunk at a time (the scale products need the registers)
@@ -257,9 +300,19 @@ __device__ __forceinline__ void epilogue_rows(const TcParams& p, const TileInfo&
             }
         }
         if (p.yexp != nullptr && valid) {
+            // one store of the run's exponent bytes: a run of n = 8, 4 or 2 chunks
+            // starts at a multiple of n (and H / 32, n0 / 32 are multiples of 8)
             int8_t* e = p.yexp + static_cast<size_t>(row) * (p.H / 32) + t.n0 / 32 + c_begin;
-            if (c_end - c_begin == 8) *reinterpret_cast<uint64_t*>(e) = exps;
-            else *reinterpret_cast<uint32_t*>(e) = static_cast<uint32_t>(exps);
+            const int n = c_end - c_begin;
+            if (n == 8) {
+                *reinterpret_cast<uint64_t*>(e) = exps;
+            } else if (n == 4) {
+                *reinterpret_cast<uint32_t*>(e) = static_cast<uint32_t>(exps);
+            } else if (n == 2) {
+                *reinterpret_cast<uint16_t*>(e) = static_cast<uint16_t>(exps);
+            } else {
+                for (int i = 0; i < n; ++i) e[i] = static_cast<int8_t>(exps >> (8 * i));
+            }
         }
     }
 }
@@ -395,7 +448,7 @@ struct Ring {
 template <bool kFp8, bool kGemm1, int kBN, bool kPair, int kRowB>
 __global__ void __launch_bounds__(320, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                        const __grid_constant__ CUtensorMap tmA2, const TcParams p) {
+                        const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ TcParams p) {
     using RG = Ring<kRowB, kBN, kPair>;
     constexpr int NSTAGE = RG::N;
     constexpr int TC_ABYTES = RG::A_TILE;           // one 128-row A tile per stage
@@ -630,6 +683,8 @@ __global__ void __launch_bounds__(320, 1)
                 if (acc == 0) acc_phase ^= 1u;
             }
         }
+        // this warp's TMA stores have left shared memory and reached global memory
+        if (lane == 0) ptx::bulk_wait_all();
     }
 
     ptx::tc_fence_before();
@@ -679,7 +734,7 @@ struct Ring2 {
 template <bool kFp8, bool kGemm1, int kBN, int kNSUB, int kRowB>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                             const __grid_constant__ CUtensorMap tmA2, const TcParams p) {
+                             const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ TcParams p) {
     static_assert(kNSUB == 1 || kBN == 256, "two sub-tiles of N = 256");
     using RG = Ring2<kRowB, kBN, kNSUB>;
     constexpr int NSTAGE = RG::N;
@@ -937,6 +992,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
                 acc_phase ^= 1u;
             }
         }
+        // this warp's TMA stores have left shared memory and reached global memory
+        if (lane == 0) ptx::bulk_wait_all();
     }
 
     __syncwarp();
@@ -1003,14 +1060,19 @@ __device__ __forceinline__ SwapUnit decode_swap(int id, const int* s_unit, const
 // One warp's 32 x 32 block of 16-bit results with lane = output column col0 +
 // lane and v[i] = output row row0 + i: written column-wise into the warp's 2 KB
 // slice (rows of 64 bytes, 16-byte chunks XOR-swizzled by (row >> 1) & 3: each
-// instruction writes one row, conflict-free), then stored row-wise as
-// stage_store does; rows at or past row_end are not stored.
+// instruction writes one row, conflict-free), then stored as stage_store does
+// (one TMA store for a whole block; rows at or past row_end are not stored).
 __device__ __forceinline__ void stage_store_t(uint8_t* slice, const uint16_t (&v)[32], int lane, uint16_t* out,
-                                              int ld, int row0, int row_end, int col0) {
+                                              int ld, int row0, int row_end, int col0, const CUtensorMap* tm) {
     const int chunk = lane >> 3, within = (lane & 7) * 2;
+    slice_acquire(tm, lane);
 #pragma unroll
     for (int i = 0; i < 32; ++i)
         *reinterpret_cast<uint16_t*>(slice + i * 64 + ((chunk ^ ((i >> 1) & 3)) * 16) + within) = v[i];
+    if (tm != nullptr && row0 + 32 <= row_end) {
+        slice_tma_store(tm, slice, lane, row0, col0);
+        return;
+    }
     __syncwarp();
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -1048,7 +1110,7 @@ __device__ __forceinline__ float silu_fast(float g) { return __fdividef(g, 1.0f 
 template <bool kFp8, bool kGemm1, int kRowB>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SW_THREADS, 1)
     grouped_gemm_swap_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
-                             const __grid_constant__ CUtensorMap tmX2, const TcParams p) {
+                             const __grid_constant__ CUtensorMap tmX2, const __grid_constant__ TcParams p) {
     using RG = RingS<kRowB>;
     constexpr int NSTAGE = RG::N;
     constexpr int KEL = kFp8 ? kRowB : kRowB / 2;
@@ -1252,6 +1314,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SW_THREADS, 1)
         const int eg = (warp - 2) >> 2;          // 0 .. EG-1
         const uint32_t tempty0 = ptx::mapa(&tempty_bar, 0);
         uint8_t* stage_w = sStage + (warp - 2) * 2048;
+        const CUtensorMap* tmo = (kGemm1 && p.out_tma) ? &p.tm_out : nullptr;
         uint32_t acc_phase = 0;
         for (int u = cluster; u < total; u += nclusters) {
             const SwapUnit t = unit(u);
@@ -1298,7 +1361,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SW_THREADS, 1)
                         }
                         o[i] = bf16_bits(silu_fast(gi) * ui);
                     }
-                    stage_store_t(stage_w, o, lane, p.out, p.out_ld, t.row0 + c * 32, row_end, col0);
+                    stage_store_t(stage_w, o, lane, p.out, p.out_ld, t.row0 + c * 32, row_end, col0, tmo);
                 }
             } else {
                 // Each 32-token chunk goes through the warp's slice as fp32 in two
@@ -1375,6 +1438,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SW_THREADS, 1)
             ptx::mbar_arrive_remote(tempty0);
             acc_phase ^= 1u;
         }
+        // this warp's TMA stores have left shared memory and reached global memory
+        if (lane == 0) ptx::bulk_wait_all();
     }
 
     __syncwarp();
@@ -1418,6 +1483,16 @@ bool make_map(CUtensorMap* m, const void* ptr, bool fp8, int rank, const cuuint6
                           row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+// Map of a 16-bit [rows, cols] output (row pitch cols) for the epilogues' TMA
+// stores: 32 x 32 boxes, 64-byte swizzle. 0 where TMA cannot address it (the
+// epilogues then store every row themselves).
+int out_map(CUtensorMap* m, const void* out, int cols, int rows) {
+    if (rows <= 0 || (reinterpret_cast<uintptr_t>(out) & 15) != 0 || (cols * 2) % 16 != 0) return 0;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+    return make_map(m, out, false, 2, dims, strides, 32, 64) ? 1 : 0;
 }
 
 int num_sms() {
@@ -1640,6 +1715,7 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
     p.tile_off = a.tile_off;
     p.out = static_cast<uint16_t*>(a.h);
     p.out_ld = a.I;
+    p.out_tma = out_map(&p.tm_out, a.h, a.I, a.R);
     p.row_scale = fp8 ? xp_scale : nullptr;
     p.direct_e = direct_e;
     p.first_e = a.perm != nullptr ? a.direct_e : -1;
@@ -1697,6 +1773,7 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
     p.k_blocks = ceil_div(a.I, kel);
     p.out = static_cast<uint16_t*>(a.y);
     p.out_ld = a.H;
+    p.out_tma = out_map(&p.tm_out, a.y, a.H, a.R);
     p.row_scale = fp8 ? a.h_scale : nullptr;
     p.direct_e = -1;
     p.col_scale = fp8 ? a.s2 : nullptr;
@@ -1711,6 +1788,9 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
                       direct_e == a.E - 1;
     if (fold) {
         p.fold_e = direct_e;
+        // the folded combine reads rows other units stored (release / acquire
+        // on p.ready): those rows are written by plain stores
+        p.out_tma = 0;
         p.fold_S = a.S;
         p.fold_inv = a.fold_inv;
         p.fold_w = a.fold_w;
