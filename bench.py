@@ -278,13 +278,14 @@ def algorithmic(cfg, kernel: str, counts: np.ndarray | None, fused: bool = True)
 
 
 # DRAM bytes (read + write) / algorithmic bytes of one launch, from one ncu
-# capture of the same kernel variant on a 1024-token, 32-routed-expert case of
-# the bf16 workload (its per-expert row counts match the full one). Traffic is
-# dominated by the touched experts' weights, so it scales with the launch.
+# capture of the same kernel variant on a 32-routed-expert case of the workload
+# the variant serves (1024 tokens of prefill_bf16 or prefill_fp8, whose
+# per-expert row counts match the full ones; the 64-token decode batch). Traffic
+# is dominated by the touched experts' weights, so it scales with the launch.
 # Keyed by (kernel, weight dtype, tensor-core work unit).
-PROFILED_TRAFFIC_RATIO = {("gemm1_tc", "bf16", 256): 1.09,
-                          ("gemm1_tc", "bf16", "pair256x512"): 1.02, ("gemm2_tc", "bf16", "pair256x512"): 0.97,
-                          ("gemm1_tc", "bf16", "swap"): 1.008}
+PROFILED_TRAFFIC_RATIO = {("gemm1_tc", "bf16", "swap"): 1.007, ("gemm2_tc", "bf16", "pair256x512"): 0.965,
+                          ("gemm1_tc", "bf16", 128): 1.009, ("gemm2_tc", "bf16", 128): 0.998,
+                          ("gemm1_tc", "e4m3", 128): 1.004, ("gemm2_tc", "e4m3", 128): 0.912}
 
 
 def unit_rows(cfg, ffn: str, kernel: str = "gemm1_tc"):
