@@ -58,8 +58,11 @@ def test_workspace_size_and_invalid_shapes(L):
     assert n_f > 0 and n_u > 0 and n_f % 256 == 0
     for bad in (dict(H=500), dict(I=100), dict(top_k=17), dict(shared_id=3),
                 dict(act_dtype=_lib.MOE_F32), dict(w_dtype=_lib.MOE_F32), dict(T=-1),
-                dict(renormalize=2), dict(n_routed=300, top_k=8, shared_id=300)):
+                dict(renormalize=2), dict(n_routed=300, top_k=8, shared_id=300),
+                dict(n_routed=257, top_k=8, shared_id=257)):
         assert L.moe_workspace_size(C.byref(_shape(**bad)), 1) == 0, bad
+    # 256 routed experts (+ the shared one) is the largest layer accepted
+    assert L.moe_workspace_size(C.byref(_shape(n_routed=256, top_k=8, shared_id=256)), 1) > 0
 
 
 FAKE = 1 << 20        # aligned non-null addresses; the host checks never dereference them

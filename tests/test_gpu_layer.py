@@ -61,6 +61,20 @@ def test_forward_small_matches_oracle(name):
     assert rel_err(fused, unfused) <= tol_of(cfg)
 
 
+@pytest.mark.parametrize("w,impl", [("bf16", MOE_FFN_AUTO), ("bf16", _lib.MOE_FFN_TCGEN05_WIDE),
+                                    ("bf16", _lib.MOE_FFN_TCGEN05_SWAP), ("e4m3", MOE_FFN_AUTO)])
+def test_the_largest_expert_count(w, impl):
+    """256 routed experts + the shared one (257 groups, the most the layer accepts)
+    through the tensor-core kernels: fused and unfused match the oracle."""
+    base = synth.CONFIGS["prefill_bf16" if w == "bf16" else "prefill_fp8"]
+    cfg = synth.variant(base, T=600, H=512, I=256, n_routed=256, top_k=8)
+    inp = synth.make_inputs(cfg)
+    d = synth.to_device(inp, DEV)
+    ref = oracle.Layer(cfg, inp).forward()
+    assert rel_err(_run(cfg, d, True, impl), ref["out"]) <= tol_of(cfg)
+    assert rel_err(_run(cfg, d, False, impl), ref["out"]) <= tol_of(cfg)
+
+
 @pytest.mark.parametrize("T,K,E_r", [(1000, 1, 8), (1500, 2, 12), (700, 8, 16)])
 def test_shared_group_units_of_the_routed_mean_size(T, K, E_r):
     """With the tokens as the MMA's N dimension the shared expert's group (all T
