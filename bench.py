@@ -215,8 +215,27 @@ def time_steps(fn, steps: int, warmup: int, dist: Dist, stream) -> float:
     return dist.max(e0.elapsed_time(e1))
 
 
-KERNELS = ["route_logits", "route_topk", "permute_small", "permute_hist", "permute_scan", "permute_scatter",
+KERNELS = ["route_logits", "route_split", "route_approx", "route_candidates", "route_verify", "route_topk",
+           "permute_small", "permute_hist", "permute_scan", "permute_scatter",
            "quant_x", "quant_h", "gather", "gemm1_tc", "gemm2_tc", "gemm1_simt", "gemm2_simt", "combine"]
+
+RV_MAXC = 32            # candidate slots per token of the verified tensor-core routing
+
+
+def route_tc_path(cfg) -> bool:
+    """Whether moe_forward routes through approximate tensor-core logits verified
+    exactly (renormalised top-K over bf16 activations, batches over 256 tokens,
+    32..256 routed experts, K <= 16, H <= 8192), as the library decides."""
+    return (cfg.act_dtype == "bf16" and cfg.renormalize and cfg.T > 256 and 32 <= cfg.n_routed <= 256
+            and cfg.top_k <= 16 and cfg.H % 256 == 0 and cfg.H <= 8192)
+
+
+def route_tc_dims(cfg):
+    """(NP, KS): expert rows padded to 32 and the number of H slices of the
+    approximate logits."""
+    nkb, nseg = cfg.H // 64, cfg.H // 256
+    ks = 4 if (nseg >= 4 and nkb % 4 == 0) else (2 if (nseg >= 2 and nkb % 2 == 0) else 1)
+    return (cfg.n_routed + 31) // 32 * 32, ks
 
 
 def kernel_table(steps: int) -> dict:
@@ -250,9 +269,25 @@ def algorithmic(cfg, kernel: str, counts: np.ndarray | None, fused: bool = True)
         return 2.0 * R * I * H, touched * H * I * wb + R * I * xb + R * H * 2 + R * (H // 32)
     if kernel == "route_logits":
         return None, T * H * ab + Er * H * 4 + (H // 256) * T * Er * 4
+    NP, KS = route_tc_dims(cfg)
+    if kernel == "route_split":
+        # fp32 router weights in, their bf16 high and low parts out
+        return None, Er * H * 4 + 2 * NP * H * 2
+    if kernel == "route_approx":
+        # two bf16 GEMMs (x times the high and the low parts); x and the split
+        # weights in, KS fp32 slices of the approximate logits out
+        return 2.0 * T * 2 * NP * H, T * H * ab + 2 * NP * H * 2 + KS * T * Er * 4
+    if kernel == "route_candidates":
+        # the slices and x (for its norm) in, the candidate lists out
+        return None, KS * T * Er * 4 + T * H * ab + T * (1 + RV_MAXC) * 4
+    if kernel == "route_verify":
+        # x and the router weights once, the candidate lists in; the candidates'
+        # segment partials out
+        return None, T * H * ab + Er * H * 4 + T * (1 + RV_MAXC) * 4 + (H // 256) * T * RV_MAXC * 4
     if kernel == "route_topk":
-        # the segment partials in; ids and weights out
-        return None, (H // 256) * T * Er * 4 + R * 8
+        # the segment partials (all experts', or the candidates') in; ids and weights out
+        per_token = RV_MAXC if route_tc_path(cfg) else Er
+        return None, (H // 256) * T * per_token * 4 + R * 8
     if kernel == "combine":
         return None, R * H * 2 + R * (H // 32) + T * H * ab + R * 4 * 2
     if kernel == "gather":

@@ -133,6 +133,12 @@ size_t moe_workspace_size(const moe_shape* shape, int fuse_shared);
  *            per 256-wide segment of H an fma chain from +0 over ascending h,
  *            segment sums added in ascending order to a total starting at +0,
  *            then the bias; so they are reproducible bit for bit.
+ * ids and weights are those of these logits either way. Without logits, a
+ * batch of more than 256 tokens (bf16 activations, renormalised top-K, 32 to
+ * 256 routed experts, K <= 16, H <= 8192) ranks approximate logits from the
+ * tensor cores and forms in the fixed order only the logits of the experts
+ * within the approximation's error bound of the K-th key: the same ids and
+ * weights, bit for bit.
  * Needs moe_workspace_size(shape, 1) bytes of ws. */
 moe_status moe_route_topk(const moe_shape* shape, const void* x, const float* router_w,
                           const float* router_bias, int32_t* ids, float* weights,

@@ -61,7 +61,7 @@ size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 int act_bytes(int dt) { return dt == MOE_F32 ? 4 : 2; }
 
 struct Layout {
-    size_t status, partials, ids, wts, counts, offsets, tile_off, perm, inv, chunk, ready;
+    size_t status, partials, route, ids, wts, counts, offsets, tile_off, perm, inv, chunk, ready;
     size_t xq, xscale, xp, xp_scale, h, hq, h_scale, y, yexp;
     // unfused only: the shared expert's dense pass
     size_t sh_off, sh_tile, sh_h, sh_hq, sh_hscale, sh_y, sh_yexp;
@@ -94,6 +94,7 @@ Layout layout_of(const moe_shape& s, const Dims& d) {
     const int ab = act_bytes(s.act_dtype);
     L.status = take(sizeof(DevStatus));
     L.partials = take(router_partial_floats(d.T, d.H, d.Er) * 4);
+    L.route = take(route_tc_scratch_bytes(d.T, d.H, d.Er));
     L.ids = take(static_cast<size_t>(d.T) * d.S * 4);
     L.wts = take(static_cast<size_t>(d.T) * d.S * 4);
     L.counts = take(static_cast<size_t>(d.E) * 4);
@@ -263,6 +264,12 @@ size_t moe_workspace_size(const moe_shape* shape, int fuse_shared) {
     return layout_of(*shape, d).total;
 }
 
+// the routing path's scratch (split router weights, candidate lists), or null
+// where that path does not apply to the shape
+void* route_scratch(const moe_shape& s, void* ws, const Layout& L) {
+    return route_tc_scratch_bytes(s.T, s.H, s.n_routed) ? at<uint8_t>(ws, L.route) : nullptr;
+}
+
 moe_status moe_route_topk(const moe_shape* shape, const void* x, const float* router_w,
                           const float* router_bias, int32_t* ids, float* weights, float* logits,
                           void* ws, size_t ws_bytes, void* stream) {
@@ -277,7 +284,8 @@ moe_status moe_route_topk(const moe_shape* shape, const void* x, const float* ro
     if (shape->T == 0) return MOE_OK;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     return cuda_status(launch_route(*shape, x, router_w, router_bias, ids, weights, logits,
-                                    at<float>(ws, L.partials), shape->shared_id, st));
+                                    at<float>(ws, L.partials), route_scratch(*shape, ws, L), shape->shared_id,
+                                    at<DevStatus>(ws, L.status), st));
 }
 
 moe_status moe_permute(const moe_shape* shape, const int32_t* ids, int32_t* counts,
@@ -377,7 +385,8 @@ moe_status moe_forward(const moe_shape* shape, const void* x, const float* route
     const bool f32_act = shape->act_dtype == MOE_F32;
     const int route_shared = fused ? shape->shared_id : -1;
     cudaError_t err = launch_route(*shape, x, router_w, router_bias, ids, wts, nullptr,
-                                   at<float>(ws, L.partials), route_shared, st);
+                                   at<float>(ws, L.partials), route_scratch(*shape, ws, L), route_shared,
+                                   at<DevStatus>(ws, L.status), st);
     if (err == cudaSuccess)
         err = launch_permute(d.R, d.E, ids, at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets),
                              at<int32_t>(ws, L.perm), at<int32_t>(ws, L.inv),

@@ -1626,6 +1626,12 @@ cudaError_t launch_gemm1_pair(const CUtensorMap& a, const CUtensorMap& b, const 
 
 }  // namespace
 
+bool make_map_bf16_2d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+    return make_map(m, ptr, false, 2, dims, strides, box_rows, 128);
+}
+
 void ffn_tc_inject_stall(int n_launches) { g_inject.store(n_launches); }
 void ffn_tc_inject_fold_stall(int n_launches) { g_inject_fold.store(n_launches); }
 

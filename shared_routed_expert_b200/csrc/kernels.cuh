@@ -1,6 +1,8 @@
 // Internal launch interface between the C ABI (api.cu) and the kernels.
 #pragma once
 
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace sre {
@@ -17,9 +19,20 @@ struct ProfileScope {
 // ---- router (route.cu)
 int router_split_count(int T, int H);
 size_t router_partial_floats(int T, int H, int E);
+// route_scratch: route_tc_scratch_bytes(T, H, n_routed) bytes (may be null when 0)
 cudaError_t launch_route(const moe_shape& s, const void* x, const float* wr, const float* bias,
-                         int32_t* ids, float* wts, float* logits, float* partials, int shared_id,
-                         cudaStream_t st);
+                         int32_t* ids, float* wts, float* logits, float* partials, void* route_scratch,
+                         int shared_id, DevStatus* status, cudaStream_t st);
+
+// ---- routing through approximate tensor-core logits, verified exactly (route_tc.cu)
+bool route_tc_applies(const moe_shape& s, const float* logits_out);
+size_t route_tc_scratch_bytes(int T, int H, int E);
+cudaError_t launch_route_tc(const moe_shape& s, const void* x, const float* wr, const float* bias, int32_t* ids,
+                            float* wts, float* partials, void* scratch, int shared_id, DevStatus* status,
+                            cudaStream_t st);
+// 2-D TMA map of a bf16 row-major [rows, cols] matrix: boxes of 64 columns
+// (128 bytes, 128-byte swizzle) by box_rows rows (ffn_tc.cu)
+bool make_map_bf16_2d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint32_t box_rows);
 
 // ---- permutation (permute.cu)
 constexpr int kPermChunk = 512;      // flat slots per scatter chunk

@@ -360,9 +360,15 @@ size_t router_partial_floats(int T, int H, int E) {
 }
 
 cudaError_t launch_route(const moe_shape& s, const void* x, const float* wr, const float* bias,
-                         int32_t* ids, float* wts, float* logits, float* partials, int shared_id,
-                         cudaStream_t st) {
+                         int32_t* ids, float* wts, float* logits, float* partials, void* route_scratch,
+                         int shared_id, DevStatus* status, cudaStream_t st) {
     const int T = s.T, H = s.H, E = s.n_routed;
+#ifndef SRE_ROUTE_TC
+#define SRE_ROUTE_TC 1
+#endif
+    // the same ids and weights from approximate tensor-core logits, verified exactly
+    if (SRE_ROUTE_TC && route_scratch != nullptr && route_tc_applies(s, logits))
+        return launch_route_tc(s, x, wr, bias, ids, wts, partials, route_scratch, shared_id, status, st);
     const int split = router_split_count(T, H);
     // small batches: 32 experts per block (5x the blocks at 160 routed experts)
 #ifndef SRE_RT_WIDE

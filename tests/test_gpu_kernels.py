@@ -81,6 +81,62 @@ def test_route_zero_router_ties_to_lowest_ids():
     assert np.allclose(w[:, :8], 0.125) and np.all(w[:, 8] == 1.0)
 
 
+# batches over 256 tokens with renormalised top-K over bf16 activations route,
+# when no logits are asked for, through approximate tensor-core logits and the
+# exact recomputation of the candidates
+VERIFIED_ROUTE_CASES = {
+    "prefill": synth.variant(synth.CONFIGS["prefill_bf16"], T=1024, I=64),
+    "zipf_bias": synth.variant(synth.CONFIGS["skewed_fp8"], T=700, I=64),
+    "bias_select_only": synth.variant(synth.CONFIGS["skewed_fp8"], T=700, I=64, bias_select_only=True,
+                                      routed_scale=2.5),
+    "max_experts": synth.variant(synth.CONFIGS["prefill_bf16"], T=600, H=1024, I=64, n_routed=256, top_k=8),
+    "min_experts_k16": synth.variant(synth.CONFIGS["prefill_bf16"], T=300, H=768, I=64, n_routed=32, top_k=16),
+    "t257": synth.variant(synth.CONFIGS["prefill_bf16"], T=257, H=512, I=64, n_routed=64, top_k=4),
+    "ties": synth.variant(synth.CONFIGS["prefill_bf16"], T=400, H=512, I=64, n_routed=48, top_k=6),
+    "nonfinite": synth.variant(synth.CONFIGS["prefill_bf16"], T=300, H=512, I=64, n_routed=40, top_k=6),
+}
+
+
+@pytest.mark.parametrize("name", list(VERIFIED_ROUTE_CASES))
+def test_verified_tensor_core_routing_equals_the_exact_path(name):
+    """Routing without logits (approximate tensor-core logits, candidates within
+    the error bound recomputed in the fixed order) gives the exact path's ids
+    and weights bit for bit, and the oracle's ids. "ties" duplicates router rows
+    (equal logits: the lower id first); "nonfinite" has tokens with +-inf and
+    NaN activations, which form every logit exactly."""
+    cfg = VERIFIED_ROUTE_CASES[name]
+    inp = synth.make_inputs(cfg)
+    if name == "ties":
+        wr = inp["router_w"]
+        wr[17] = wr[5]
+        wr[41] = wr[40]
+        wr[3] = wr[30]
+    if name == "nonfinite":
+        x = inp["x"]
+        x[1, 7] = float("inf")
+        x[2, 300] = float("-inf")
+        x[3, 7] = float("inf")
+        x[3, 300] = float("-inf")
+        x[4, 0] = float("nan")
+        x[5, :] = float("inf")
+    d = synth.to_device(inp, DEV)
+    ids_x, w_x, L = _route(cfg, d)              # logits asked for: the exact path
+    s = _lib.make_shape(cfg)
+    ws = _lib.alloc_workspace(s, True)
+    ids = torch.empty(cfg.T, cfg.slots, dtype=torch.int32, device=DEV)
+    w = torch.empty(cfg.T, cfg.slots, dtype=torch.float32, device=DEV)
+    _lib.moe_route_topk(s, d["x"], d["router_w"], d["router_bias"], ids, w, None, ws)
+    torch.cuda.synchronize()
+    ids, w = ids.cpu().numpy(), w.cpu().numpy()
+    assert np.array_equal(ids, ids_x)
+    assert np.array_equal(w.view(np.uint32), w_x.view(np.uint32))
+    Lr = oracle_logits(d["x"], d["router_w"], d["router_bias"])
+    Lw = oracle_logits(d["x"], d["router_w"], None) if cfg.bias_select_only else None
+    rid, _ = oracle.topk(Lr, cfg.top_k, cfg.renormalize, cfg.shared_id, cfg.shared_weight,
+                         weight_logits=Lw, routed_scale=cfg.routed_scale)
+    assert np.array_equal(ids, rid)
+
+
 @pytest.mark.parametrize("bias_select_only,n_neg_inf", [(False, 9), (True, 9), (False, 36), (True, 36)])
 def test_route_nonfinite_inputs_follow_the_oracle(bias_select_only, n_neg_inf):
     """Non-finite router inputs (R3: NaN ranks as -inf, ties toward the lower
