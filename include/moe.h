@@ -289,6 +289,15 @@ void moe_inject_wait_timeout(int n_calls);
  * outputs of those calls are garbage). No GPU fault is involved. */
 void moe_inject_fold_timeout(int n_calls);
 
+/* Failure-injection hook for the routing through approximate tensor-core
+ * logits (moe_route_topk / moe_forward on batches over 256 tokens): in the
+ * next n_calls calls that take that path, the approximate-logit kernel issues
+ * no loads and waits with a limit of about 10 ms; its waits run out, it drains,
+ * frees TMEM and returns, and MOE_ERR_TIMEOUT is left in the status word (the
+ * routing of those calls is garbage, but every id stays in range). No GPU fault
+ * is involved. */
+void moe_inject_route_timeout(int n_calls);
+
 /* Fused QK-norm + partial RoPE on the attention's q and k heads, in place.
  * "GLM4-MoE生产环境优化：SGLang降低65%首Token延迟", section 2.2 QK-Norm-RoPE
  * fusion, and the de/en pages, section 2 "Qknorm Fusion": both steps are

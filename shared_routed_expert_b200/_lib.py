@@ -23,7 +23,8 @@ EXPORTS = ("moe_workspace_size", "moe_route_topk", "moe_permute", "moe_grouped_f
            "moe_combine", "moe_forward", "moe_quant_rows_e4m3", "moe_get_status",
            "moe_clear_status", "moe_status_string", "moe_launch_count", "moe_profile_enable",
            "moe_profile_reset", "moe_profile_read", "moe_inject_wait_timeout",
-           "moe_permute_noalloc", "moe_qk_norm_rope", "moe_cast_f32_bf16", "moe_inject_fold_timeout")
+           "moe_permute_noalloc", "moe_qk_norm_rope", "moe_cast_f32_bf16", "moe_inject_fold_timeout",
+           "moe_inject_route_timeout")
 
 
 class MoeError(RuntimeError):
@@ -84,6 +85,8 @@ def lib() -> C.CDLL:
         L.moe_inject_wait_timeout.argtypes = [i]
         L.moe_inject_fold_timeout.restype = None
         L.moe_inject_fold_timeout.argtypes = [i]
+        L.moe_inject_route_timeout.restype = None
+        L.moe_inject_route_timeout.argtypes = [i]
         L.moe_cast_f32_bf16.restype = i
         L.moe_cast_f32_bf16.argtypes = [sz, p, p, p]
         L.moe_qk_norm_rope.restype = i
@@ -232,6 +235,10 @@ def moe_inject_wait_timeout(n_calls: int):
 
 def moe_inject_fold_timeout(n_calls: int):
     lib().moe_inject_fold_timeout(int(n_calls))
+
+
+def moe_inject_route_timeout(n_calls: int):
+    lib().moe_inject_route_timeout(int(n_calls))
 
 
 def moe_profile_read(name: str):

@@ -530,6 +530,8 @@ void moe_inject_wait_timeout(int n_calls) { ffn_tc_inject_stall(n_calls > 0 ? n_
 
 void moe_inject_fold_timeout(int n_calls) { ffn_tc_inject_fold_stall(n_calls > 0 ? n_calls : 0); }
 
+void moe_inject_route_timeout(int n_calls) { route_tc_inject_stall(n_calls > 0 ? n_calls : 0); }
+
 void moe_profile_enable(int on) { g_prof_on.store(on != 0); }
 
 void moe_profile_reset(void) {

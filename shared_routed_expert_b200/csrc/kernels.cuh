@@ -27,6 +27,7 @@ cudaError_t launch_route(const moe_shape& s, const void* x, const float* wr, con
 // ---- routing through approximate tensor-core logits, verified exactly (route_tc.cu)
 bool route_tc_applies(const moe_shape& s, const float* logits_out);
 size_t route_tc_scratch_bytes(int T, int H, int E);
+void route_tc_inject_stall(int n_calls);     // testing hook (moe_inject_route_timeout)
 cudaError_t launch_route_tc(const moe_shape& s, const void* x, const float* wr, const float* bias, int32_t* ids,
                             float* wts, float* partials, void* scratch, int shared_id, DevStatus* status,
                             cudaStream_t st);

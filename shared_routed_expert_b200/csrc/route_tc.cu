@@ -35,6 +35,7 @@
 // serves renormalised top-K over bf16 activations when no logits are asked
 // for; route.cu serves the rest.
 #include <algorithm>
+#include <atomic>
 
 #include "kernels.cuh"
 #include "tc_ptx.cuh"
@@ -111,7 +112,7 @@ __global__ void __launch_bounds__(256) route_split_kernel(const float* __restric
 __global__ void __launch_bounds__(RTC_THREADS, 1)
     route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, int T, int E,
                     int NP, int kb_per, int nstage, float* __restrict__ approx, DevStatus* status,
-                    long long wait_limit) {
+                    long long wait_limit, int inject_stall) {
     constexpr int A_BYTES = 128 * 128;
     const int B_BYTES = 2 * NP * 128;
     const int STAGE = A_BYTES + B_BYTES;
@@ -145,7 +146,7 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
     const uint32_t tmem = s_tmem;
 
     if (warp == 0) {
-        if (lane == 0) {
+        if (lane == 0 && !inject_stall) {       // testing hook: no loads, so the waits below run out
             int stage = 0;
             uint32_t phase = 0;
             for (int kb = 0; kb < kb_per; ++kb) {
@@ -188,8 +189,12 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
                 ptx::mma_commit(&empty_bar[stage]);
                 if (++stage == nstage) { stage = 0; phase ^= 1u; }
             }
-            // completes once every MMA issued above has finished
+            // completes once every MMA issued above has finished; waited for here
+            // as well, so that its arrival lands before the CTA may leave
             ptx::mma_commit(&tfull_bar);
+            const long long t0 = clock64();
+            while (!ptx::mbar_try_wait(&tfull_bar, 0u) && clock64() - t0 < wait_limit) {
+            }
         }
     } else {
         const int sub = warp & 3;
@@ -555,6 +560,8 @@ __global__ void __launch_bounds__(256) route_select_kernel(const float* __restri
 
 inline size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
 
+std::atomic<int> g_inject_route{0};
+
 int rv_split(int H) {
     const int nkb = H / 64, nseg = H / RV_SEG;
     if (nseg >= 4 && nkb % 4 == 0) return 4;
@@ -563,6 +570,8 @@ int rv_split(int H) {
 }
 
 }  // namespace
+
+void route_tc_inject_stall(int n_calls) { g_inject_route.store(n_calls); }
 
 bool route_tc_applies(const moe_shape& s, const float* logits_out) {
     return logits_out == nullptr && s.act_dtype == MOE_BF16 && s.renormalize != 0 && s.T > 256 &&
@@ -615,9 +624,16 @@ cudaError_t launch_route_tc(const moe_shape& s, const void* x, const float* wr, 
             if (e != cudaSuccess) return e;
             attr = RTC_RING + 2048;
         }
+        int inject = 0;
+        {
+            int cur = g_inject_route.load();
+            while (cur > 0 && !g_inject_route.compare_exchange_weak(cur, cur - 1)) {
+            }
+            inject = cur > 0 ? 1 : 0;
+        }
         ProfileScope ps("route_approx", st);
-        route_tc_kernel<<<dim3((T + 127) / 128, KS), RTC_THREADS, smem, st>>>(tmX, tmW, T, E, NP, H / 64 / KS, nstage,
-                                                                             approx, status, 4ll << 30);
+        route_tc_kernel<<<dim3((T + 127) / 128, KS), RTC_THREADS, smem, st>>>(
+            tmX, tmW, T, E, NP, H / 64 / KS, nstage, approx, status, inject ? (20ll << 20) : (4ll << 30), inject);
         note_launch();
     }
     {

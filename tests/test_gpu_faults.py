@@ -54,3 +54,23 @@ def test_folded_combine_wait_timeout_is_reported(impl, T):
     ref = oracle.Layer(cfg, inp).forward()["out"]
     assert rel_err(to_f64(out), ref) <= tol_of(cfg)
     torch.cuda.synchronize()
+
+
+def test_routing_wait_timeout_is_reported():
+    """Routing through approximate tensor-core logits (batches over 256 tokens):
+    when its GEMM's producer issues no loads, the waits run out (~10 ms), the
+    kernel drains and returns MOE_ERR_TIMEOUT, every id stays in range (the
+    layer still runs), and the next pass is clean and right."""
+    build.build()
+    cfg = synth.variant(synth.CONFIGS["prefill_bf16"], T=300, H=512, I=128, n_routed=40, top_k=6)
+    inp = synth.make_inputs(cfg)
+    d = synth.to_device(inp, "cuda")
+    layer = MoELayer(cfg, d)
+    _lib.moe_inject_route_timeout(1)
+    layer.forward(d["x"])
+    assert layer.status() == _lib.MOE_ERR_TIMEOUT
+    out = layer.forward(d["x"])
+    assert layer.status() == _lib.MOE_OK
+    ref = oracle.Layer(cfg, inp).forward()["out"]
+    assert rel_err(to_f64(out), ref) <= tol_of(cfg)
+    torch.cuda.synchronize()
