@@ -140,3 +140,22 @@ def test_unmeasured_figures_print_as_null(capsys):
     out = capsys.readouterr().out
     assert json.loads(out) == {"value": 1.5, "unfused": {"ms_per_step": None, "x": [None, 2]}}
     assert "NaN" not in out and "Infinity" not in out
+
+
+def test_route_path_and_its_dims_follow_the_library_rule():
+    """bench.py charges the routing kernels by the same rule the library uses:
+    prefill batches (T > 256, bf16 activations, renormalised, 32..256 routed
+    experts, K <= 16) take the tensor-core routing, decode and fp32 layers the
+    fixed-order router; NP pads the experts to 32, KS slices H (<= H/256)."""
+    import bench
+    from shared_routed_expert_b200 import synth
+    C = synth.CONFIGS
+    assert bench.route_tc_path(C["prefill_bf16"]) and bench.route_tc_path(C["prefill_fp8"])
+    assert bench.route_tc_path(C["skewed_fp8"])
+    assert not bench.route_tc_path(C["decode_bf16"]) and not bench.route_tc_path(C["tiny_fp32"])
+    assert not bench.route_tc_path(synth.variant(C["prefill_bf16"], renormalize=False))
+    assert not bench.route_tc_path(synth.variant(C["prefill_bf16"], n_routed=16, top_k=4))
+    assert bench.route_tc_dims(C["prefill_bf16"]) == (160, 4)
+    assert bench.route_tc_dims(synth.variant(C["prefill_bf16"], H=512, n_routed=40)) == (64, 2)
+    assert bench.route_tc_dims(synth.variant(C["prefill_bf16"], H=768, n_routed=33)) == (64, 2)
+    assert bench.route_tc_dims(synth.variant(C["prefill_bf16"], H=256, n_routed=256)) == (256, 1)
