@@ -94,6 +94,8 @@ VERIFIED_ROUTE_CASES = {
     "t257": synth.variant(synth.CONFIGS["prefill_bf16"], T=257, H=512, I=64, n_routed=64, top_k=4),
     "ties": synth.variant(synth.CONFIGS["prefill_bf16"], T=400, H=512, I=64, n_routed=48, top_k=6),
     "nonfinite": synth.variant(synth.CONFIGS["prefill_bf16"], T=300, H=512, I=64, n_routed=40, top_k=6),
+    # the widest H the path takes, and an expert count that is not a multiple of 4
+    "h8192_e37": synth.variant(synth.CONFIGS["prefill_bf16"], T=300, H=8192, I=64, n_routed=37, top_k=5),
 }
 
 
