@@ -278,11 +278,12 @@ def algorithmic(cfg, kernel: str, counts: np.ndarray | None, fused: bool = True)
         # weights in, KS fp32 slices of the approximate logits out
         return 2.0 * T * 2 * NP * H, T * H * ab + 2 * NP * H * 2 + KS * T * Er * 4
     if kernel == "route_candidates":
-        # the slices and x (for its norm) in, the candidate lists out
+        # the slices and x (for its norm) in, the candidate lists out (and each
+        # pair's entry in its expert's bucket, at most RV_MAXC per token)
         return None, KS * T * Er * 4 + T * H * ab + T * (1 + RV_MAXC) * 4
     if kernel == "route_verify":
-        # x and the router weights once, the candidate lists in; the candidates'
-        # segment partials out
+        # x and the router weights once, the bucketed pairs (at most RV_MAXC per
+        # token) in; the candidates' segment partials out
         return None, T * H * ab + Er * H * 4 + T * (1 + RV_MAXC) * 4 + (H // 256) * T * RV_MAXC * 4
     if kernel == "route_topk":
         # the segment partials (all experts', or the candidates') in; ids and weights out

@@ -25,9 +25,10 @@
 //                  approximate key is below Tk - max eps - eps_e is beaten by K
 //                  experts and is not in the exact top-K: the exact top-K lies in
 //                  S = {e : key_e + eps_e >= Tk - max eps}.
-//   D. verify      the fixed-order segment partials of the candidates only (one
-//                  thread per token, its activations in registers, each chunk of
-//                  every expert's weights staged in shared memory).
+//   D. verify      the fixed-order segment partials of the candidates only: the
+//                  (token, candidate) pairs are bucketed by expert, so a warp
+//                  works on pairs of one expert (its weights read once for all
+//                  lanes) and each lane streams its token's activations.
 //   E. select      ordered segment sums, the bias, the ranking (key descending,
 //                  id ascending) and the softmax over the selected slots, with
 //                  the arithmetic of route.cu's top-K kernel.
@@ -48,8 +49,6 @@ namespace {
 constexpr int RV_MAXC = 32;                 // candidate slots per token
 constexpr float RV_C = 1.0e-4f;             // eps coefficient (see step C)
 constexpr int RV_SEG = 256;                 // the fixed order's segment length
-constexpr int RV_KC = 32;                   // h per verify chunk
-constexpr int RV_WP = RV_KC + 4;            // row pitch (floats) of a staged weight chunk
 constexpr int RTC_THREADS = 192;            // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr int RTC_MAX_STAGES = 6;
 constexpr int RTC_RING = 192 * 1024;
@@ -62,11 +61,14 @@ __device__ __forceinline__ bool better(float v, int e, float bv, int be) {
 __device__ __forceinline__ float rank_key(float v) { return isnan(v) ? -INFINITY : v; }
 
 // ---------------------------------------------------------------- A. split
+// Also zeroes the per-expert pair counters that step C fills.
 __global__ void __launch_bounds__(256) route_split_kernel(const float* __restrict__ wr, int E, int H,
-                                                          __nv_bfloat16* __restrict__ ws, float* __restrict__ nw) {
+                                                          __nv_bfloat16* __restrict__ ws, float* __restrict__ nw,
+                                                          int32_t* __restrict__ bcnt) {
     // H <= 8192: every thread's (up to 8) float4 loads are in flight together
     constexpr int VM = 8;
     const int e = blockIdx.x;
+    if (threadIdx.x == 0) bcnt[e] = 0;
     const int nv = H / 4;
     float4 v[VM];
 #pragma unroll
@@ -244,12 +246,18 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
 // ---------------------------------------------------------------- C. candidates
 // One warp per token. cand_n[t] = |S| (every expert when the token's bound is
 // not usable); cand[t][0 .. min(|S|, RV_MAXC)) the candidate ids, ascending.
+// A token whose |S| <= RV_MAXC also appends each pair (t, slot) to its expert's
+// bucket: bucket[e][bcnt[e]++] = t * RV_MAXC + slot (the order inside a bucket
+// is that of the atomics; every pair's result is formed on its own, so it does
+// not matter).
 __global__ void __launch_bounds__(256) route_candidates_kernel(const float* __restrict__ approx, int KS,
                                                                const float* __restrict__ bias,
                                                                const float* __restrict__ nw,
                                                                const uint16_t* __restrict__ x, int T, int H, int E,
                                                                int K, int32_t* __restrict__ cand_n,
-                                                               int32_t* __restrict__ cand) {
+                                                               int32_t* __restrict__ cand,
+                                                               int32_t* __restrict__ bcnt,
+                                                               int32_t* __restrict__ bucket) {
     const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (t >= T) return;
@@ -328,146 +336,184 @@ __global__ void __launch_bounds__(256) route_candidates_kernel(const float* __re
     const float lim = tk - eps_max;             // -inf when Tk is -inf: every expert
     usable = usable && isfinite(eps_max);
     int n = 0;
+    int slot[J];
 #pragma unroll
     for (int j = 0; j < J; ++j) {
         const int e = lane + 32 * j;
         const bool c = e < E && (!usable || key[j] + eps[j] >= lim);
         const unsigned m = __ballot_sync(0xFFFFFFFFu, c);
-        if (c) {
-            const int slot = n + __popc(m & ((1u << lane) - 1u));
-            if (slot < RV_MAXC) cand[static_cast<size_t>(t) * RV_MAXC + slot] = e;
-        }
+        slot[j] = c ? n + __popc(m & ((1u << lane) - 1u)) : RV_MAXC;
+        if (slot[j] < RV_MAXC) cand[static_cast<size_t>(t) * RV_MAXC + slot[j]] = e;
         n += __popc(m);
     }
     if (lane == 0) cand_n[t] = usable ? n : E + 1;    // E + 1: not usable, every logit in step E
+    if (usable && n <= RV_MAXC) {
+        // every atomic of the lane is issued before the first result is used
+        int pos[J];
+#pragma unroll
+        for (int j = 0; j < J; ++j) pos[j] = slot[j] < RV_MAXC ? atomicAdd(&bcnt[lane + 32 * j], 1) : -1;
+#pragma unroll
+        for (int j = 0; j < J; ++j)
+            if (pos[j] >= 0) bucket[static_cast<size_t>(lane + 32 * j) * T + pos[j]] = t * RV_MAXC + slot[j];
+    }
 }
 
 // ---------------------------------------------------------------- D. verify
-// Block (token tile of 128, segment s): thread = token. Every 32-h chunk of the
-// segment stages all experts' weights (cp.async, double-buffered) and each
-// thread extends its candidates' fma chains from its own activations.
+// A warp item is (segment s, expert e, 32 of e's bucketed pairs); lane = pair
+// (t, c). The segment is taken in chunks of RV_KC h. For each chunk the warp
+// copies its 32 tokens' activations (8 lanes per 128-byte row, coalesced) and
+// the expert's RV_KC weights into one of its two shared-memory buffers with
+// cp.async; while one buffer is multiplied the next chunk (of this item, or
+// the first of the warp's next item) is in flight. Each lane reads its own row
+// back (row pitch 144 bytes: the 8 lanes of a quarter-warp hit distinct bank
+// groups), the weights as broadcasts, and extends its fma chain. Items are
+// numbered segment-major, so the activations in use at a time are one
+// segment's columns of x (T x 512 bytes), which stay in L2.
 // pc[s][t][c] = segment partial of candidate c.
-__device__ __forceinline__ void rv_cp16(void* dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
-                 "l"(src)
-                 : "memory");
+constexpr int RV_KC = 64;                   // h per chunk
+constexpr int RV_PITCH = RV_KC * 2 + 16;    // bytes per staged activation row
+constexpr int RV_WARPS = 4;                 // warps per block
+constexpr int RV_BUF = 32 * RV_PITCH + RV_KC * 4;   // a chunk: 32 rows, then the weights
+
+__device__ __forceinline__ void rv_cp16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
 
-__device__ __forceinline__ void rv_load_x(const uint16_t* __restrict__ x, int t, int T, int H, int h0, uint4 (&q)[4]) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) q[i] = make_uint4(0u, 0u, 0u, 0u);
-    if (t < T) {
-        const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H + h0);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) q[i] = xr[i];
+// the pairs of one item, as this lane sees them
+struct RvItem {
+    int s, e, t, c;
+    bool valid;
+    int rowtok[8];                          // tokens of the rows this lane copies
+};
+
+__device__ __forceinline__ RvItem rv_item(int item, int per_seg, const int* pre, int E, int T,
+                                          const int32_t* __restrict__ bcnt, const int32_t* __restrict__ bucket,
+                                          int lane) {
+    RvItem it;
+    it.s = item / per_seg;
+    const int r = item - it.s * per_seg;
+    int lo = 0, hi = E;                     // pre[lo] <= r < pre[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (pre[mid] <= r) lo = mid;
+        else hi = mid;
     }
+    it.e = lo;
+    const int p = (r - pre[lo]) * 32 + lane;
+    it.valid = p < bcnt[lo];
+    const int code = it.valid ? bucket[static_cast<size_t>(lo) * T + p] : 0;
+    it.t = code / RV_MAXC;
+    it.c = code % RV_MAXC;
+    return it;
 }
 
-__global__ void __launch_bounds__(128) route_verify_kernel(const uint16_t* __restrict__ x,
-                                                           const float* __restrict__ wr, int T, int H, int E, int EP,
-                                                           const int32_t* __restrict__ cand_n,
-                                                           const int32_t* __restrict__ cand, float* __restrict__ pc) {
-    extern __shared__ __align__(16) float rv_w[];        // [2][EP][RV_WP]
-    const int t = blockIdx.x * 128 + threadIdx.x;
-    const int s = blockIdx.y;
-    int n = 0;
-    if (t < T) {
-        n = cand_n[t];
-        if (n > RV_MAXC) n = 0;                 // done in full by the select pass
-    }
-    int nmax = n;
+// the tokens of the rows this lane copies (apart from rv_item so that the
+// bucket load of the next item is waited for only when its first chunk is
+// copied)
+__device__ __forceinline__ void rv_rows(RvItem& it, int lane) {
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) nmax = max(nmax, __shfl_xor_sync(0xFFFFFFFFu, nmax, off));
-    // slots past n compute on expert 0's row and are never stored
-    int ce[RV_MAXC];
+    for (int j = 0; j < 8; ++j) it.rowtok[j] = __shfl_sync(0xFFFFFFFFu, it.t, (lane >> 3) + 4 * j);
+}
+
+// chunk kc of an item into the buffer at `dst` (shared-memory address)
+__device__ __forceinline__ void rv_copy(const RvItem& it, int kc, uint32_t dst, const uint16_t* __restrict__ x,
+                                        const float* __restrict__ wr, int H, int lane) {
+    const int h0 = it.s * RV_SEG + kc * RV_KC;
+    const int piece = lane & 7;
 #pragma unroll
-    for (int c = 0; c < RV_MAXC; ++c) ce[c] = (c < n) ? cand[static_cast<size_t>(t) * RV_MAXC + c] : 0;
-    float acc[RV_MAXC];
+    for (int j = 0; j < 8; ++j)
+        rv_cp16(dst + ((lane >> 3) + 4 * j) * RV_PITCH + piece * 16,
+                x + static_cast<size_t>(it.rowtok[j]) * H + h0 + piece * 8);
+    if (lane < RV_KC / 4) rv_cp16(dst + 32 * RV_PITCH + lane * 16, wr + static_cast<size_t>(it.e) * H + h0 + lane * 4);
+}
+
+__global__ void __launch_bounds__(RV_WARPS * 32) route_verify_kernel(const uint16_t* __restrict__ x,
+                                                                     const float* __restrict__ wr, int T, int H,
+                                                                     int E, const int32_t* __restrict__ bcnt,
+                                                                     const int32_t* __restrict__ bucket,
+                                                                     float* __restrict__ pc) {
+    extern __shared__ __align__(16) uint8_t rv_x[];    // [RV_WARPS][2][RV_BUF]
+    __shared__ int pre[257];                // pre[e]: first item of expert e within a segment
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (warp == 0) {
+        int v[8], sum = 0;
 #pragma unroll
-    for (int c = 0; c < RV_MAXC; ++c) acc[c] = 0.0f;
-    constexpr int NCH = RV_SEG / RV_KC;
-    auto stage_w = [&](int ch, int buf) {
-        float* dst = rv_w + static_cast<size_t>(buf) * EP * RV_WP;
-        const int h0 = s * RV_SEG + ch * RV_KC;
-        for (int i = threadIdx.x; i < EP * (RV_KC / 4); i += 128) {
-            const int e = i / (RV_KC / 4), q = i % (RV_KC / 4);
-            if (e < E) rv_cp16(dst + e * RV_WP + q * 4, wr + static_cast<size_t>(e) * H + h0 + q * 4);
+        for (int j = 0; j < 8; ++j) {
+            const int e = lane * 8 + j;
+            v[j] = e < E ? (bcnt[e] + 31) >> 5 : 0;
+            sum += v[j];
         }
-        asm volatile("cp.async.commit_group;" ::: "memory");
-    };
-    stage_w(0, 0);
-    uint4 xq[4];
-    rv_load_x(x, t, T, H, s * RV_SEG, xq);
-    for (int ch = 0; ch < NCH; ++ch) {
-        const int buf = ch & 1;
-        if (ch + 1 < NCH) stage_w(ch + 1, buf ^ 1);
-        // this thread's 32 activations of the chunk (bf16 -> fp32 is exact); the
-        // next chunk's are loaded while this one is multiplied
-        float xv[RV_KC];
+        int incl = sum;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint32_t w[4] = {xq[i].x, xq[i].y, xq[i].z, xq[i].w};
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+            if (lane >= off) incl += y;
+        }
+        int run = incl - sum;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                xv[i * 8 + 2 * j] = __uint_as_float(w[j] << 16);
-                xv[i * 8 + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+        for (int j = 0; j < 8; ++j) {
+            pre[lane * 8 + j] = run;
+            run += v[j];
+        }
+        if (lane == 31) pre[256] = incl;
+    }
+    __syncthreads();
+    const int per_seg = pre[256];
+    const int total = per_seg * (H / RV_SEG);
+    const int nwarp = gridDim.x * RV_WARPS;
+    const uint32_t sbuf = static_cast<uint32_t>(__cvta_generic_to_shared(rv_x)) + warp * 2 * RV_BUF;
+    const uint8_t* gbuf = rv_x + warp * 2 * RV_BUF;
+    int item = blockIdx.x * RV_WARPS + warp;
+    if (item >= total) return;
+    RvItem cur = rv_item(item, per_seg, pre, E, T, bcnt, bucket, lane);
+    rv_rows(cur, lane);
+    rv_copy(cur, 0, sbuf, x, wr, H, lane);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    int b = 0;
+    constexpr int NKC = RV_SEG / RV_KC;
+    while (true) {
+        const int nitem = item + nwarp;
+        const bool more = nitem < total;
+        RvItem nxt = cur;
+        if (more) nxt = rv_item(nitem, per_seg, pre, E, T, bcnt, bucket, lane);
+        float acc = 0.0f;
+#pragma unroll 1
+        for (int kc = 0; kc < NKC; ++kc) {
+            // the next chunk's copy goes out before this one is multiplied
+            if (kc + 1 < NKC) rv_copy(cur, kc + 1, sbuf + (b ^ 1) * RV_BUF, x, wr, H, lane);
+            else if (more) {
+                rv_rows(nxt, lane);
+                rv_copy(nxt, 0, sbuf + (b ^ 1) * RV_BUF, x, wr, H, lane);
             }
-        }
-        if (ch + 1 < NCH) rv_load_x(x, t, T, H, s * RV_SEG + (ch + 1) * RV_KC, xq);
-        if (ch + 1 < NCH) asm volatile("cp.async.wait_group 1;" ::: "memory");
-        else asm volatile("cp.async.wait_group 0;" ::: "memory");
-        __syncthreads();
-        const float* wb = rv_w + static_cast<size_t>(buf) * EP * RV_WP;
-        // four candidates' chains side by side (independent fma chains); the
-        // warp's last group holds only the candidates some lane still has
+            asm volatile("cp.async.commit_group;" ::: "memory");
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+            __syncwarp();                       // every lane's pieces of this chunk have landed
+            const uint8_t* row = gbuf + b * RV_BUF + lane * RV_PITCH;
+            const float* wc = reinterpret_cast<const float*>(gbuf + b * RV_BUF + 32 * RV_PITCH);
 #pragma unroll
-        for (int c0 = 0; c0 < RV_MAXC; c0 += 4) {
-            if (c0 >= nmax) break;              // warp-uniform
-            const int g = nmax - c0;            // warp-uniform, >= 1
-            const float* w0 = wb + ce[c0] * RV_WP;
-            const float* w1 = wb + ce[c0 + 1] * RV_WP;
-            const float* w2 = wb + ce[c0 + 2] * RV_WP;
-            const float* w3 = wb + ce[c0 + 3] * RV_WP;
-            float r0 = acc[c0], r1 = acc[c0 + 1], r2 = acc[c0 + 2], r3 = acc[c0 + 3];
-#pragma unroll
-            for (int q = 0; q < RV_KC / 4; ++q) {
-                const float x0 = xv[4 * q], x1 = xv[4 * q + 1], x2 = xv[4 * q + 2], x3 = xv[4 * q + 3];
-                const float4 a = *reinterpret_cast<const float4*>(w0 + q * 4);
-                r0 = __fmaf_rn(x0, a.x, r0);
-                r0 = __fmaf_rn(x1, a.y, r0);
-                r0 = __fmaf_rn(x2, a.z, r0);
-                r0 = __fmaf_rn(x3, a.w, r0);
-                if (g > 1) {
-                    const float4 b = *reinterpret_cast<const float4*>(w1 + q * 4);
-                    r1 = __fmaf_rn(x0, b.x, r1);
-                    r1 = __fmaf_rn(x1, b.y, r1);
-                    r1 = __fmaf_rn(x2, b.z, r1);
-                    r1 = __fmaf_rn(x3, b.w, r1);
-                }
-                if (g > 2) {
-                    const float4 c = *reinterpret_cast<const float4*>(w2 + q * 4);
-                    r2 = __fmaf_rn(x0, c.x, r2);
-                    r2 = __fmaf_rn(x1, c.y, r2);
-                    r2 = __fmaf_rn(x2, c.z, r2);
-                    r2 = __fmaf_rn(x3, c.w, r2);
-                }
-                if (g > 3) {
-                    const float4 d = *reinterpret_cast<const float4*>(w3 + q * 4);
-                    r3 = __fmaf_rn(x0, d.x, r3);
-                    r3 = __fmaf_rn(x1, d.y, r3);
-                    r3 = __fmaf_rn(x2, d.z, r3);
-                    r3 = __fmaf_rn(x3, d.w, r3);
-                }
+            for (int q = 0; q < RV_KC / 8; ++q) {
+                const uint4 xv = *reinterpret_cast<const uint4*>(row + q * 16);
+                const float4 wa = *reinterpret_cast<const float4*>(wc + q * 8);
+                const float4 wb = *reinterpret_cast<const float4*>(wc + q * 8 + 4);
+                // bf16 -> fp32 is exact; h ascending within the segment
+                acc = __fmaf_rn(__uint_as_float(xv.x << 16), wa.x, acc);
+                acc = __fmaf_rn(__uint_as_float(xv.x & 0xFFFF0000u), wa.y, acc);
+                acc = __fmaf_rn(__uint_as_float(xv.y << 16), wa.z, acc);
+                acc = __fmaf_rn(__uint_as_float(xv.y & 0xFFFF0000u), wa.w, acc);
+                acc = __fmaf_rn(__uint_as_float(xv.z << 16), wb.x, acc);
+                acc = __fmaf_rn(__uint_as_float(xv.z & 0xFFFF0000u), wb.y, acc);
+                acc = __fmaf_rn(__uint_as_float(xv.w << 16), wb.z, acc);
+                acc = __fmaf_rn(__uint_as_float(xv.w & 0xFFFF0000u), wb.w, acc);
             }
-            acc[c0] = r0; acc[c0 + 1] = r1; acc[c0 + 2] = r2; acc[c0 + 3] = r3;
+            __syncwarp();                       // the buffer is copied into again on the next chunk
+            b ^= 1;
         }
-        __syncthreads();                        // the buffer is restaged two chunks on
+        if (cur.valid) pc[(static_cast<size_t>(cur.s) * T + cur.t) * RV_MAXC + cur.c] = acc;
+        if (!more) break;
+        item = nitem;
+        cur = nxt;
     }
-    if (t < T) {
-#pragma unroll
-        for (int c = 0; c < RV_MAXC; ++c)
-            if (c < n) pc[(static_cast<size_t>(s) * T + t) * RV_MAXC + c] = acc[c];
-    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
 // ---------------------------------------------------------------- E. select
@@ -598,7 +644,8 @@ bool route_tc_applies(const moe_shape& s, const float* logits_out) {
 size_t route_tc_scratch_bytes(int T, int H, int E) {
     if (E < 32 || E > 256 || T <= 256 || H % RV_SEG != 0 || H > 8192) return 0;
     return align256(static_cast<size_t>(2) * WS_ROWS * H * 2) + align256(256 * 4) +
-           align256(static_cast<size_t>(T) * 4) + align256(static_cast<size_t>(T) * RV_MAXC * 4);
+           align256(static_cast<size_t>(T) * 4) + align256(static_cast<size_t>(T) * RV_MAXC * 4) +
+           align256(256 * 4) + align256(static_cast<size_t>(E) * T * 4);
 }
 
 cudaError_t launch_route_tc(const moe_shape& s, const void* x, const float* wr, const float* bias, int32_t* ids,
@@ -616,6 +663,10 @@ cudaError_t launch_route_tc(const moe_shape& s, const void* x, const float* wr, 
     int32_t* cand_n = reinterpret_cast<int32_t*>(p);
     p += align256(static_cast<size_t>(T) * 4);
     int32_t* cand = reinterpret_cast<int32_t*>(p);
+    p += align256(static_cast<size_t>(T) * RV_MAXC * 4);
+    int32_t* bcnt = reinterpret_cast<int32_t*>(p);
+    p += align256(256 * 4);
+    int32_t* bucket = reinterpret_cast<int32_t*>(p);
     // the router partials buffer ([H/256][T][E] floats) holds the approximate
     // slices first ([KS][T][E], KS <= H/256) and the candidates' exact segment
     // partials after them ([H/256][T][RV_MAXC], RV_MAXC <= E)
@@ -627,7 +678,7 @@ cudaError_t launch_route_tc(const moe_shape& s, const void* x, const float* wr, 
         return cudaErrorInvalidValue;
     {
         ProfileScope ps("route_split", st);
-        route_split_kernel<<<NP, 256, 0, st>>>(wr, E, H, wsplit, nw);
+        route_split_kernel<<<NP, 256, 0, st>>>(wr, E, H, wsplit, nw, bcnt);
         note_launch();
     }
     {
@@ -657,21 +708,26 @@ cudaError_t launch_route_tc(const moe_shape& s, const void* x, const float* wr, 
         ProfileScope ps("route_candidates", st);
         route_candidates_kernel<<<(T * 32 + 255) / 256, 256, 0, st>>>(approx, KS, bias, nw,
                                                                      static_cast<const uint16_t*>(x), T, H, E, K,
-                                                                     cand_n, cand);
+                                                                     cand_n, cand, bcnt, bucket);
         note_launch();
     }
     {
-        const int smem = 2 * NP * RV_WP * 4;
-        static int attr = 0;
-        if (smem > attr) {
-            const cudaError_t e = cudaFuncSetAttribute(route_verify_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                       2 * 256 * RV_WP * 4);
+        static int grid = 0;
+        if (grid == 0) {
+            int dev = 0, nsm = 0, per = 0;
+            cudaGetDevice(&dev);
+            cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+            cudaError_t e = cudaFuncSetAttribute(route_verify_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 RV_WARPS * 2 * RV_BUF);
+            if (e == cudaSuccess)
+                e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, route_verify_kernel, RV_WARPS * 32,
+                                                                  RV_WARPS * 2 * RV_BUF);
             if (e != cudaSuccess) return e;
-            attr = 2 * 256 * RV_WP * 4;
+            grid = std::max(1, nsm * per);
         }
         ProfileScope ps("route_verify", st);
-        route_verify_kernel<<<dim3((T + 127) / 128, nseg), 128, smem, st>>>(static_cast<const uint16_t*>(x), wr, T, H,
-                                                                           E, NP, cand_n, cand, pc);
+        route_verify_kernel<<<grid, RV_WARPS * 32, RV_WARPS * 2 * RV_BUF, st>>>(static_cast<const uint16_t*>(x), wr,
+                                                                               T, H, E, bcnt, bucket, pc);
         note_launch();
     }
     {
