@@ -251,6 +251,12 @@ def kernel_table(steps: int) -> dict:
     return tab
 
 
+def token_major_gather(cfg) -> bool:
+    """The layer gathers its rows token by token (bf16 tokens on the tensor-core
+    path, H <= 5120), quantising them there for E4M3 weights."""
+    return cfg.act_dtype == "bf16" and cfg.w_dtype != "f32" and cfg.H % 8 == 0 and cfg.H <= 5120
+
+
 def algorithmic(cfg, kernel: str, counts: np.ndarray | None, fused: bool = True):
     """(flops, bytes) one launch of `kernel` must do for this workload: flops of
     the dense contraction it performs (None if it is not one), and the bytes it
@@ -295,6 +301,9 @@ def algorithmic(cfg, kernel: str, counts: np.ndarray | None, fused: bool = True)
         # the fused layer's shared rows are read from x by GEMM1 and not copied:
         # x read once, the routed rows written (plus per-row scales for E4M3)
         copied = R - T if (fused and cfg.shared) else R
+        if wb == 1 and token_major_gather(cfg):
+            # bf16 x read once, quantised: the token codes and the routed rows' codes written
+            return None, T * H * ab + (T + copied) * (H + 4)
         return None, T * H * xb + copied * H * xb + (copied * 4 + T * 4 if wb == 1 else 0)
     if kernel == "quant_x":
         # x per token (T rows of H): bf16 in, E4M3 codes and one scale per row out

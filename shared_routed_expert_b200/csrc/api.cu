@@ -177,11 +177,19 @@ __global__ void tile_prefix_kernel(int E, const int32_t* __restrict__ off, int32
 
 // Expert FFN over already-gathered rows (xp). Runs quantisation of h in between
 // for E4M3 layers.
+bool tc_forced_impl(int impl) {
+    return impl == MOE_FFN_TCGEN05 || impl == MOE_FFN_TCGEN05_M128 || impl == MOE_FFN_TCGEN05_M256 ||
+           impl == MOE_FFN_TCGEN05_PAIR || impl == MOE_FFN_TCGEN05_WIDE || impl == MOE_FFN_TCGEN05_SWAP;
+}
+
+// run_ffn takes the tensor-core path for these arguments
+bool ffn_takes_tc(const FfnArgs& in, int impl) {
+    return ffn_tc_supported(in) && (tc_forced_impl(impl) || (impl == MOE_FFN_AUTO && in.w_dtype != MOE_F32));
+}
+
 cudaError_t run_ffn(const FfnArgs& in, int impl, cudaStream_t st) {
     const bool tc_ok = ffn_tc_supported(in);
-    const bool tc_forced = impl == MOE_FFN_TCGEN05 || impl == MOE_FFN_TCGEN05_M128 ||
-                           impl == MOE_FFN_TCGEN05_M256 || impl == MOE_FFN_TCGEN05_PAIR ||
-                           impl == MOE_FFN_TCGEN05_WIDE || impl == MOE_FFN_TCGEN05_SWAP;
+    const bool tc_forced = tc_forced_impl(impl);
     if (tc_forced || (impl == MOE_FFN_AUTO && in.w_dtype != MOE_F32 && tc_ok)) {
         if (!tc_ok) return cudaErrorNotSupported;
         FfnArgs a = in;
@@ -392,17 +400,31 @@ moe_status moe_forward(const moe_shape* shape, const void* x, const float* route
                              at<int32_t>(ws, L.perm), at<int32_t>(ws, L.inv),
                              at<int32_t>(ws, L.tile_off), at<int32_t>(ws, L.chunk),
                              at<DevStatus>(ws, L.status), st);
-    const void* xt = nullptr;
-    const float* xt_scale = nullptr;
+    // the token matrix of the grouped pass: x, or its per-token E4M3 codes
+    const void* xt = fp8 ? static_cast<const void*>(at<uint8_t>(ws, L.xq)) : x;
+    const float* xt_scale = fp8 ? at<float>(ws, L.xscale) : nullptr;
     bool folded = false;
-    if (err == cudaSuccess) err = prepare_tokens(*shape, d, L, ws, x, &xt, &xt_scale, st);
+    FfnArgs a = ffn_args(*shape, d, L, ws, xt, xt_scale, at<int32_t>(ws, L.perm), w13, s13, w2, s2,
+                         at<void>(ws, L.y));
+    a.yexp = f32_act ? nullptr : at<int8_t>(ws, L.yexp);
+    // fused layout: the shared expert's group is every token in order (stable
+    // permutation, shared id last), so its rows need no gather
+    a.direct_e = (fused && d.shared) ? d.E - 1 : -1;
     if (err == cudaSuccess) {
-        FfnArgs a = ffn_args(*shape, d, L, ws, xt, xt_scale, at<int32_t>(ws, L.perm), w13, s13, w2, s2,
-                             at<void>(ws, L.y));
-        a.yexp = f32_act ? nullptr : at<int8_t>(ws, L.yexp);
-        // fused layout: the shared expert's group is every token in order (stable
-        // permutation, shared id last), so its rows need no gather
-        a.direct_e = (fused && d.shared) ? d.E - 1 : -1;
+        if (shape->act_dtype == MOE_BF16 && scatter_rows_supported(d.H) && ffn_takes_tc(a, ffn_impl)) {
+            // the grouped rows by token (each token's row read once, quantised
+            // there for E4M3 layers) instead of quantising the tokens and then
+            // gathering row by row inside the tensor-core pass
+            err = launch_scatter_rows(d.T, d.S, d.R, d.H, x, at<int32_t>(ws, L.inv),
+                                      a.direct_e >= 0 ? at<int32_t>(ws, L.offsets) + a.direct_e : nullptr,
+                                      fp8 ? at<uint8_t>(ws, L.xq) : nullptr, fp8 ? at<float>(ws, L.xscale) : nullptr,
+                                      a.xp, a.xp_scale, st);
+            a.xp_ready = 1;
+        } else {
+            err = prepare_tokens(*shape, d, L, ws, x, &xt, &xt_scale, st);
+        }
+    }
+    if (err == cudaSuccess) {
         if (a.direct_e >= 0 && !f32_act && fold_combine) {
             // the weighted combine inside GEMM2's shared-expert units, where the
             // tensor-core GEMM2 runs it (folded tells whether it did)

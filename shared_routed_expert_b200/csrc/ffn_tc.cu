@@ -1655,7 +1655,10 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
     // tokens themselves when perm is null)
     const void* xp = a.xt;
     const float* xp_scale = a.xt_scale;
-    if (a.perm != nullptr) {
+    if (a.perm != nullptr && a.xp_ready) {
+        xp = a.xp;
+        xp_scale = a.xp_scale;
+    } else if (a.perm != nullptr) {
         // the direct group's rows are not copied: GEMM1 reads them from xt
         const int32_t* skip = a.direct_e >= 0 ? a.offsets + a.direct_e : nullptr;
         const cudaError_t e = launch_gather_rows(a.R, a.S, a.H, esz, a.xt, a.xt_scale, a.perm, a.xp, a.xp_scale,

@@ -49,6 +49,15 @@ cudaError_t launch_permute(int R, int E, const int32_t* ids, int32_t* counts, in
 cudaError_t launch_gather_rows(int R, int S, int H, int elem_bytes, const void* x,
                                const float* xscale, const int32_t* perm, void* xp, float* xpscale,
                                const int32_t* skip, cudaStream_t stream);
+// Token-major form of the same rows from bf16 tokens x [T, H]: for each token t
+// and slot k, row inv[t * S + k] of xp (rows in [skip[0], skip[1]) and slots
+// without a row in [0, R) are left out). With xq != null (E4M3 layers) the
+// token's row is quantised per row first (codes and scale to xq[t], xscale[t],
+// the same codes as launch_quant_rows) and xp / xpscale receive the codes.
+bool scatter_rows_supported(int H);
+cudaError_t launch_scatter_rows(int T, int S, int R, int H, const void* x, const int32_t* inv,
+                                const int32_t* skip, uint8_t* xq, float* xscale, void* xp, float* xpscale,
+                                cudaStream_t stream);
 // per-row E4M3 quantisation of bf16 rows
 cudaError_t launch_quant_rows(int rows, int cols, const uint16_t* in, uint8_t* codes,
                               float* scales, cudaStream_t stream, const char* name = "quant_rows");
@@ -63,9 +72,10 @@ struct FfnArgs {
     int T;
     const int32_t* perm;          // [R] row -> flat slot t*S + k; null: row r is token r
     int S;
-    // CUDA-core path only: rows gathered from xt into xp before the GEMMs
+    // rows gathered from xt into xp before the GEMMs
     void* xp;                     // [R, H] (act dtype, or E4M3 codes)
     float* xp_scale;              // [R] (E4M3)
+    int xp_ready = 0;             // tensor-core path: xp already holds the rows (token-major gather)
     const int32_t* offsets;       // [E+1]
     const int32_t* tile_off;      // [E+1] m-tile prefix (kTileM rows)
     const void* w13; const float* s13;

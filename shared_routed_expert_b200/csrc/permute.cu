@@ -276,6 +276,44 @@ __device__ __forceinline__ float div_by_recip(float v, float s, float y) {
 // 2^-11 or more, the only ones whose code depends on its last bit, has a normal
 // residual; smaller ones are codes of +-0 either way), by the divide otherwise.
 constexpr float kMarksteinMinAmax = 8.6736174e-19f;    // 2^-60
+
+// the quantiser of a row whose largest magnitude is amax
+struct RowQuant {
+    float scale, y;
+    bool by_recip;
+};
+__device__ __forceinline__ RowQuant row_quant(float amax) {
+    RowQuant q;
+    q.scale = (amax > 0.0f) ? __fdiv_rn(amax, 448.0f) : 1.0f;
+    q.by_recip = amax >= kMarksteinMinAmax && amax <= 3.4028235e38f;     // warp-uniform
+    q.y = q.by_recip ? __frcp_rn(q.scale) : 0.0f;
+    return q;
+}
+
+__device__ __forceinline__ float amax_bf16x8(float amax, const uint4 q) {
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        amax = fmaxf(amax, fabsf(__uint_as_float(w[j] << 16)));
+        amax = fmaxf(amax, fabsf(__uint_as_float(w[j] & 0xFFFF0000u)));
+    }
+    return amax;
+}
+
+// eight bf16 values -> eight E4M3 codes (in order, little-endian)
+__device__ __forceinline__ uint2 codes_bf16x8(const uint4 q, const RowQuant& rq) {
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float a = __uint_as_float(w[j] << 16), b = __uint_as_float(w[j] & 0xFFFF0000u);
+        const uint32_t lo = f32_to_e4m3(rq.by_recip ? div_by_recip(a, rq.scale, rq.y) : __fdiv_rn(a, rq.scale));
+        const uint32_t hi = f32_to_e4m3(rq.by_recip ? div_by_recip(b, rq.scale, rq.y) : __fdiv_rn(b, rq.scale));
+        packed[j >> 1] |= (lo | (hi << 8)) << ((j & 1) * 16);
+    }
+    return make_uint2(packed[0], packed[1]);
+}
+
 __global__ void __launch_bounds__(256) quant_rows_kernel(int rows, int cols,
                                                          const uint16_t* __restrict__ in,
                                                          uint8_t* __restrict__ codes,
@@ -286,35 +324,78 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(int rows, int cols,
     const uint4* src = reinterpret_cast<const uint4*>(in + static_cast<size_t>(r) * cols);
     const int nv = cols / 8;
     float amax = 0.0f;
-    for (int i = lane; i < nv; i += 32) {
-        const uint4 q = src[i];
-        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            amax = fmaxf(amax, fabsf(__uint_as_float(w[j] << 16)));
-            amax = fmaxf(amax, fabsf(__uint_as_float(w[j] & 0xFFFF0000u)));
-        }
-    }
+    for (int i = lane; i < nv; i += 32) amax = amax_bf16x8(amax, src[i]);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
-    const float scale = (amax > 0.0f) ? __fdiv_rn(amax, 448.0f) : 1.0f;
-    const bool by_recip = amax >= kMarksteinMinAmax && amax <= 3.4028235e38f;     // warp-uniform
-    const float y = by_recip ? __frcp_rn(scale) : 0.0f;
+    const RowQuant rq = row_quant(amax);
     uint2* dst = reinterpret_cast<uint2*>(codes + static_cast<size_t>(r) * cols);
-    for (int i = lane; i < nv; i += 32) {
-        const uint4 q = src[i];
-        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-        uint32_t packed[2] = {0u, 0u};
+    for (int i = lane; i < nv; i += 32) dst[i] = codes_bf16x8(src[i], rq);
+    if (lane == 0) scales[r] = rq.scale;
+}
+
+// Token-major gather of the grouped pass's rows: one warp per token t reads its
+// row once into registers (H <= kScatterMaxH bf16 values) and writes it to the
+// rows inv[t * S + k] of its slots, leaving out rows in [skip[0], skip[1]) (a
+// group the GEMM reads from the token matrix directly) and slots without a row.
+// kQuant (E4M3 layers): the row is quantised as quant_rows_kernel does it and
+// its codes and scale go to the token matrix (xq, xscale) as well as to the
+// slots' rows (xp, xpscale); otherwise the bf16 row itself is copied.
+constexpr int kScatterVec = 20;                 // 16-byte vectors per lane
+constexpr int kScatterMaxH = kScatterVec * 32 * 8;
+
+template <bool kQuant>
+__global__ void __launch_bounds__(256) scatter_rows_kernel(int T, int S, int R, int H,
+                                                           const uint4* __restrict__ x,
+                                                           const int32_t* __restrict__ inv,
+                                                           const int32_t* __restrict__ skip,
+                                                           uint8_t* __restrict__ xq, float* __restrict__ xscale,
+                                                           void* __restrict__ xp, float* __restrict__ xpscale) {
+    const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (t >= T) return;
+    const int nv = H / 8;
+    uint4 v[kScatterVec];
+    const uint4* src = x + static_cast<size_t>(t) * nv;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float a = __uint_as_float(w[j] << 16), b = __uint_as_float(w[j] & 0xFFFF0000u);
-            const uint32_t lo = f32_to_e4m3(by_recip ? div_by_recip(a, scale, y) : __fdiv_rn(a, scale));
-            const uint32_t hi = f32_to_e4m3(by_recip ? div_by_recip(b, scale, y) : __fdiv_rn(b, scale));
-            packed[j >> 1] |= (lo | (hi << 8)) << ((j & 1) * 16);
+    for (int j = 0; j < kScatterVec; ++j)
+        if (j * 32 + lane < nv) v[j] = src[j * 32 + lane];
+    const int s0 = skip != nullptr ? skip[0] : 0, s1 = skip != nullptr ? skip[1] : 0;
+    if constexpr (kQuant) {
+        float amax = 0.0f;
+#pragma unroll
+        for (int j = 0; j < kScatterVec; ++j)
+            if (j * 32 + lane < nv) amax = amax_bf16x8(amax, v[j]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+        const RowQuant rq = row_quant(amax);
+        uint2 c[kScatterVec];
+#pragma unroll
+        for (int j = 0; j < kScatterVec; ++j)
+            if (j * 32 + lane < nv) c[j] = codes_bf16x8(v[j], rq);
+        uint2* dq = reinterpret_cast<uint2*>(xq + static_cast<size_t>(t) * H);
+#pragma unroll
+        for (int j = 0; j < kScatterVec; ++j)
+            if (j * 32 + lane < nv) dq[j * 32 + lane] = c[j];
+        if (lane == 0) xscale[t] = rq.scale;
+        for (int k = 0; k < S; ++k) {
+            const int r = inv[static_cast<size_t>(t) * S + k];
+            if (r < 0 || r >= R || (r >= s0 && r < s1)) continue;       // warp-uniform
+            uint2* d = reinterpret_cast<uint2*>(static_cast<uint8_t*>(xp) + static_cast<size_t>(r) * H);
+#pragma unroll
+            for (int j = 0; j < kScatterVec; ++j)
+                if (j * 32 + lane < nv) d[j * 32 + lane] = c[j];
+            if (lane == 0) xpscale[r] = rq.scale;
         }
-        dst[i] = make_uint2(packed[0], packed[1]);
+    } else {
+        for (int k = 0; k < S; ++k) {
+            const int r = inv[static_cast<size_t>(t) * S + k];
+            if (r < 0 || r >= R || (r >= s0 && r < s1)) continue;       // warp-uniform
+            uint4* d = static_cast<uint4*>(xp) + static_cast<size_t>(r) * nv;
+#pragma unroll
+            for (int j = 0; j < kScatterVec; ++j)
+                if (j * 32 + lane < nv) d[j * 32 + lane] = v[j];
+        }
     }
-    if (lane == 0) scales[r] = scale;
 }
 
 }  // namespace
@@ -360,6 +441,24 @@ cudaError_t launch_gather_rows(int R, int S, int H, int elem_bytes, const void* 
     ProfileScope ps("gather", stream);
     gather_rows_kernel<<<ceil_div(R * 32, 256), 256, 0, stream>>>(
         R, S, row_vecs, static_cast<const uint4*>(x), xscale, perm, static_cast<uint4*>(xp), xpscale, skip);
+    note_launch();
+    return cudaGetLastError();
+}
+
+bool scatter_rows_supported(int H) { return H > 0 && H % 8 == 0 && H <= kScatterMaxH; }
+
+cudaError_t launch_scatter_rows(int T, int S, int R, int H, const void* x, const int32_t* inv,
+                                const int32_t* skip, uint8_t* xq, float* xscale, void* xp, float* xpscale,
+                                cudaStream_t stream) {
+    if (!scatter_rows_supported(H)) return cudaErrorNotSupported;
+    if (T == 0) return cudaSuccess;
+    ProfileScope ps("gather", stream);
+    if (xq != nullptr)
+        scatter_rows_kernel<true><<<ceil_div(T * 32, 256), 256, 0, stream>>>(
+            T, S, R, H, static_cast<const uint4*>(x), inv, skip, xq, xscale, xp, xpscale);
+    else
+        scatter_rows_kernel<false><<<ceil_div(T * 32, 256), 256, 0, stream>>>(
+            T, S, R, H, static_cast<const uint4*>(x), inv, skip, nullptr, nullptr, xp, nullptr);
     note_launch();
     return cudaGetLastError();
 }
