@@ -126,10 +126,12 @@ def test_gather_bytes_leave_out_the_shared_rows():
     assert nb == 4096 * 5120 * 2 + 32768 * 5120 * 2 == 377_487_360
     _, nb_u = bench.algorithmic(cfg, "gather", None, fused=False)
     assert nb_u == 4096 * 5120 * 2 + cfg.rows * 5120 * 2
-    # E4M3: one byte per element plus the per-row scales
+    # E4M3 layers gather token by token from bf16 x: x read once (2 B per
+    # element), the codes of every token and of the 32768 routed rows written
+    # (1 B per element) with one fp32 scale per row
     c8 = synth.CONFIGS["skewed_fp8"]
     _, nb8 = bench.algorithmic(c8, "gather", None)
-    assert nb8 == 4096 * 5120 + 32768 * 5120 + 32768 * 4 + 4096 * 4
+    assert nb8 == 4096 * 5120 * 2 + (4096 + 32768) * (5120 + 4)
 
 
 def test_unmeasured_figures_print_as_null(capsys):
