@@ -216,7 +216,7 @@ def time_steps(fn, steps: int, warmup: int, dist: Dist, stream) -> float:
 
 
 KERNELS = ["route_logits", "route_split", "route_approx", "route_candidates", "route_verify", "route_topk",
-           "permute_small", "permute_hist", "permute_scan", "permute_scatter",
+           "permute_small", "permute_hist", "permute_scan", "permute_scatter", "permute_fused",
            "quant_x", "quant_h", "gather", "gemm1_tc", "gemm2_tc", "gemm1_simt", "gemm2_simt", "combine"]
 
 RV_MAXC = 32            # candidate slots per token of the verified tensor-core routing
@@ -319,6 +319,9 @@ def algorithmic(cfg, kernel: str, counts: np.ndarray | None, fused: bool = True)
         return None, 2 * n_chunks * E * 4 + 3 * (E + 1) * 4
     if kernel == "permute_scatter":
         return None, R * 4 + n_chunks * E * 4 + (E + 1) * 4 + 2 * R * 4
+    if kernel == "permute_fused":
+        # ids in, perm and inv out, the chunk counts written once and read back once
+        return None, R * 4 + 2 * R * 4 + 2 * n_chunks * E * 4 + 3 * (E + 1) * 4
     return None, None
 
 

@@ -61,7 +61,7 @@ size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 int act_bytes(int dt) { return dt == MOE_F32 ? 4 : 2; }
 
 struct Layout {
-    size_t status, partials, route, ids, wts, counts, offsets, tile_off, perm, inv, chunk, ready;
+    size_t status, partials, route, ids, wts, counts, offsets, tile_off, perm, inv, chunk, pbar, ready;
     size_t xq, xscale, xp, xp_scale, h, hq, h_scale, y, yexp;
     // unfused only: the shared expert's dense pass
     size_t sh_off, sh_tile, sh_h, sh_hq, sh_hscale, sh_y, sh_yexp;
@@ -103,6 +103,7 @@ Layout layout_of(const moe_shape& s, const Dims& d) {
     L.perm = take(static_cast<size_t>(d.R) * 4);
     L.inv = take(static_cast<size_t>(d.R) * 4);
     L.chunk = take(permute_scratch_ints(d.R, d.E) * 4);
+    L.pbar = take(4);
     L.ready = take(static_cast<size_t>(d.H / 256) * 4);
     if (fp8) {
         L.xq = take(static_cast<size_t>(d.T) * d.H);
@@ -309,7 +310,7 @@ moe_status moe_permute(const moe_shape* shape, const int32_t* ids, int32_t* coun
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     return cuda_status(launch_permute(d.R, d.E, ids, counts, offsets, perm, inv,
                                       at<int32_t>(ws, L.tile_off), at<int32_t>(ws, L.chunk),
-                                      at<DevStatus>(ws, L.status), st));
+                                      at<DevStatus>(ws, L.status), st, at<unsigned>(ws, L.pbar)));
 }
 
 moe_status moe_grouped_ffn(const moe_shape* shape, const void* x, const int32_t* perm,
@@ -399,7 +400,7 @@ moe_status moe_forward(const moe_shape* shape, const void* x, const float* route
         err = launch_permute(d.R, d.E, ids, at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets),
                              at<int32_t>(ws, L.perm), at<int32_t>(ws, L.inv),
                              at<int32_t>(ws, L.tile_off), at<int32_t>(ws, L.chunk),
-                             at<DevStatus>(ws, L.status), st);
+                             at<DevStatus>(ws, L.status), st, at<unsigned>(ws, L.pbar));
     // the token matrix of the grouped pass: x, or its per-token E4M3 codes
     const void* xt = fp8 ? static_cast<const void*>(at<uint8_t>(ws, L.xq)) : x;
     const float* xt_scale = fp8 ? at<float>(ws, L.xscale) : nullptr;

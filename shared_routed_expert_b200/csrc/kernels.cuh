@@ -39,10 +39,12 @@ bool make_map_bf16_2d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t r
 constexpr int kPermChunk = 512;      // flat slots per scatter chunk
 constexpr int kTileM = 128;          // rows per expert GEMM tile (tile schedule granularity)
 size_t permute_scratch_ints(int R, int E);
-// Also fills tile_off[E+1] (exclusive scan of ceil(count/kTileM)).
+// Also fills tile_off[E+1] (exclusive scan of ceil(count/kTileM)). With
+// fused_bar (one unsigned of device memory) the batches the three-kernel path
+// would take run as one cooperative kernel where its grid fits on the device.
 cudaError_t launch_permute(int R, int E, const int32_t* ids, int32_t* counts, int32_t* offsets,
                            int32_t* perm, int32_t* inv, int32_t* tile_off, int32_t* scratch,
-                           DevStatus* st, cudaStream_t stream);
+                           DevStatus* st, cudaStream_t stream, unsigned* fused_bar = nullptr);
 // Xp[r] = x[perm[r] / S] (bf16 or fp32 rows, or E4M3 codes + per-row scale);
 // rows in [skip[0], skip[1]) are left out when skip != null (a group whose rows
 // the GEMM reads from x directly)

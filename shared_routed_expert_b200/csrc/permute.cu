@@ -15,6 +15,7 @@
 //   scatter: one warp per chunk walks its slots in order, 32 at a time;
 //            __match_any_sync ranks equal experts inside a group.
 #include "kernels.cuh"
+#include "tc_ptx.cuh"
 
 namespace sre {
 
@@ -157,6 +158,152 @@ __global__ void __launch_bounds__(32) perm_scatter_kernel(const int32_t* __restr
         }
         __syncwarp();
         if (e >= 0 && (peers & lt) == 0) next[e] += __popc(peers);   // lowest lane of the group
+        __syncwarp();
+    }
+}
+
+// The three kernels above as one cooperative launch (every block resident at
+// once), one block of kFusedWarps warps per 512-slot chunk, E <= 256:
+//   1. warp w counts the experts of its 64 slots (chunk slots 64 w .. 64 w + 63)
+//      and the block writes the chunk's column chunk_hist[.][c];
+//   2. grid barrier: each block adds 1 to *bar (zeroed before the launch) and
+//      waits, bounded, until it reads n_chunks (on expiry MOE_ERR_TIMEOUT and
+//      the block returns);
+//   3. warp w sums rows e = w, w + 8, ... of chunk_hist: the expert's rows in
+//      chunks before c and in all chunks; a scan over experts turns the totals
+//      into offsets (block 0 also writes counts, offsets and tile_off), and a
+//      scan over the block's warps gives each warp its first row per expert;
+//   4. each warp ranks its slots in slot order with __match_any_sync.
+// Rows follow slot order inside each expert (chunk, then warp, then lane), as
+// in the three kernels.
+constexpr int kFusedWarps = kPermChunk / 64;
+__global__ void __launch_bounds__(kFusedWarps * 32) perm_fused_kernel(
+    const int32_t* __restrict__ ids, int R, int E, int n_chunks, int32_t* __restrict__ chunk_hist,
+    int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ tile_off,
+    int32_t* __restrict__ perm, int32_t* __restrict__ inv, unsigned* bar, long long wait_limit,
+    DevStatus* status) {
+    __shared__ int32_t s_w[kFusedWarps][256];   // per warp: slots of expert e, then its first row
+    __shared__ int32_t s_pre[256], s_tot[256];
+    __shared__ int s_ok;
+    const int c = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int i = tid; i < kFusedWarps * 256; i += kFusedWarps * 32) s_w[i / 256][i % 256] = 0;
+    __syncthreads();
+    const unsigned lt = (1u << lane) - 1u;
+    int my[2];
+    unsigned peers[2];
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+        const int f = c * kPermChunk + warp * 64 + g * 32 + lane;
+        int e = (f < R) ? ids[f] : -1;
+        if (f < R && (e < 0 || e >= E)) report(status, MOE_ERR_DEVICE, static_cast<unsigned>(f));
+        if (e >= E) e = -1;
+        my[g] = e < 0 ? -1 : e;
+        peers[g] = __match_any_sync(0xFFFFFFFFu, my[g]);
+    }
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+        if (my[g] >= 0 && (peers[g] & lt) == 0) s_w[warp][my[g]] += __popc(peers[g]);   // one leader per expert
+        __syncwarp();
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += kFusedWarps * 32) {
+        int h = 0;
+#pragma unroll
+        for (int w = 0; w < kFusedWarps; ++w) h += s_w[w][e];
+        chunk_hist[static_cast<size_t>(e) * n_chunks + c] = h;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        atomicAdd(bar, 1u);
+        volatile int never = 0;
+        s_ok = ptx::counter_wait(bar, static_cast<unsigned>(n_chunks), &never, wait_limit, status, 30u);
+    }
+    __syncthreads();
+    if (!s_ok) return;
+    __threadfence();
+    {
+        // warp w: experts w + kFusedWarps i; every expert's loads of a 32-chunk
+        // round are in flight together
+        constexpr int IPW = 256 / kFusedWarps;
+        int pre[IPW], tot[IPW];
+#pragma unroll
+        for (int i = 0; i < IPW; ++i) pre[i] = tot[i] = 0;
+        for (int c0 = 0; c0 < n_chunks; c0 += 32) {
+            const int cc = c0 + lane;
+#pragma unroll
+            for (int i = 0; i < IPW; ++i) {
+                const int e = warp + kFusedWarps * i;
+                if (e < E && cc < n_chunks) {
+                    const int v = __ldcg(chunk_hist + static_cast<size_t>(e) * n_chunks + cc);
+                    tot[i] += v;
+                    pre[i] += cc < c ? v : 0;
+                }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < IPW; ++i) {
+            const int e = warp + kFusedWarps * i;
+            if (e >= E) break;                  // warp-uniform
+            int t = tot[i], p = pre[i];
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                t += __shfl_xor_sync(0xFFFFFFFFu, t, off);
+                p += __shfl_xor_sync(0xFFFFFFFFu, p, off);
+            }
+            if (lane == 0) {
+                s_pre[e] = p;
+                s_tot[e] = t;
+            }
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {
+        int carry = 0, tcarry = 0;
+        for (int e0 = 0; e0 < E; e0 += 32) {
+            const int e = e0 + lane;
+            const int n = (e < E) ? s_tot[e] : 0;
+            const int tc = ceil_div(n, kTileM);
+            const int inc = warp_inclusive_scan(n, lane);
+            const int tinc = warp_inclusive_scan(tc, lane);
+            if (e < E) {
+                if (c == 0) {
+                    counts[e] = n;
+                    offsets[e] = carry + inc - n;
+                    tile_off[e] = tcarry + tinc - tc;
+                }
+                s_pre[e] += carry + inc - n;        // the chunk's first row of expert e
+            }
+            carry += __shfl_sync(0xFFFFFFFFu, inc, 31);
+            tcarry += __shfl_sync(0xFFFFFFFFu, tinc, 31);
+        }
+        if (lane == 0 && c == 0) {
+            offsets[E] = carry;
+            tile_off[E] = tcarry;
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += kFusedWarps * 32) {   // exclusive scan over the block's warps
+        int run = s_pre[e];
+#pragma unroll
+        for (int w = 0; w < kFusedWarps; ++w) {
+            const int n = s_w[w][e];
+            s_w[w][e] = run;
+            run += n;
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+        const int f = c * kPermChunk + warp * 64 + g * 32 + lane;
+        const int e = my[g];
+        if (e >= 0) {
+            const int row = s_w[warp][e] + __popc(peers[g] & lt);
+            perm[row] = f;
+            inv[f] = row;
+        }
+        __syncwarp();
+        if (e >= 0 && (peers[g] & lt) == 0) s_w[warp][e] += __popc(peers[g]);
         __syncwarp();
     }
 }
@@ -404,9 +551,24 @@ size_t permute_scratch_ints(int R, int E) {
     return static_cast<size_t>(ceil_div(R, kPermChunk)) * E;
 }
 
+// blocks of perm_fused_kernel that can be resident at once
+int fused_capacity() {
+    static int cap = -1;
+    if (cap < 0) {
+        int dev = 0, nsm = 0, per = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, perm_fused_kernel, kFusedWarps * 32, 0) !=
+            cudaSuccess)
+            per = 0;
+        cap = nsm * per;
+    }
+    return cap;
+}
+
 cudaError_t launch_permute(int R, int E, const int32_t* ids, int32_t* counts, int32_t* offsets,
                            int32_t* perm, int32_t* inv, int32_t* tile_off, int32_t* scratch,
-                           DevStatus* st, cudaStream_t stream) {
+                           DevStatus* st, cudaStream_t stream, unsigned* fused_bar) {
     if (R <= kSmallR && E <= kSmallE) {
         ProfileScope ps("permute_small", stream);
         perm_small_kernel<<<1, 1024, 0, stream>>>(ids, R, E, counts, offsets, tile_off, perm, inv, st);
@@ -414,6 +576,24 @@ cudaError_t launch_permute(int R, int E, const int32_t* ids, int32_t* counts, in
         return cudaGetLastError();
     }
     const int n_chunks = ceil_div(R, kPermChunk);
+    if (fused_bar != nullptr && E <= 256 && n_chunks <= fused_capacity()) {
+        cudaError_t err = cudaMemsetAsync(fused_bar, 0, sizeof(unsigned), stream);
+        if (err != cudaSuccess) return err;
+        ProfileScope ps("permute_fused", stream);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(n_chunks), 1, 1);
+        cfg.blockDim = dim3(kFusedWarps * 32, 1, 1);
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        err = cudaLaunchKernelEx(&cfg, perm_fused_kernel, ids, R, E, n_chunks, scratch, counts, offsets, tile_off,
+                                 perm, inv, fused_bar, 4ll << 30, st);
+        note_launch();
+        return err;
+    }
     const size_t hsm = static_cast<size_t>(E) * sizeof(int32_t);
     if (n_chunks > 0) {
         ProfileScope ps("permute_hist", stream);

@@ -49,6 +49,7 @@ namespace {
 constexpr int RV_MAXC = 32;                 // candidate slots per token
 constexpr float RV_C = 1.0e-4f;             // eps coefficient (see step C)
 constexpr int RV_SEG = 256;                 // the fixed order's segment length
+constexpr int RV_CPAD = 32;                 // ints between two experts' pair counters (one 128-byte line each)
 constexpr int RTC_THREADS = 192;            // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr int RTC_MAX_STAGES = 6;
 constexpr int RTC_RING = 192 * 1024;
@@ -68,7 +69,7 @@ __global__ void __launch_bounds__(256) route_split_kernel(const float* __restric
     // H <= 8192: every thread's (up to 8) float4 loads are in flight together
     constexpr int VM = 8;
     const int e = blockIdx.x;
-    if (threadIdx.x == 0) bcnt[e] = 0;
+    if (threadIdx.x == 0) bcnt[e * RV_CPAD] = 0;
     const int nv = H / 4;
     float4 v[VM];
 #pragma unroll
@@ -247,9 +248,10 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
 // One warp per token. cand_n[t] = |S| (every expert when the token's bound is
 // not usable); cand[t][0 .. min(|S|, RV_MAXC)) the candidate ids, ascending.
 // A token whose |S| <= RV_MAXC also appends each pair (t, slot) to its expert's
-// bucket: bucket[e][bcnt[e]++] = t * RV_MAXC + slot (the order inside a bucket
-// is that of the atomics; every pair's result is formed on its own, so it does
-// not matter).
+// bucket: bucket[e][bcnt[e * RV_CPAD]++] = t * RV_MAXC + slot. Each counter sits
+// on a cache line of its own, so that the atomics spread over the L2 slices.
+// The order inside a bucket is that of the atomics; every pair's result is
+// formed on its own, so it does not matter.
 __global__ void __launch_bounds__(256) route_candidates_kernel(const float* __restrict__ approx, int KS,
                                                                const float* __restrict__ bias,
                                                                const float* __restrict__ nw,
@@ -351,7 +353,8 @@ __global__ void __launch_bounds__(256) route_candidates_kernel(const float* __re
         // every atomic of the lane is issued before the first result is used
         int pos[J];
 #pragma unroll
-        for (int j = 0; j < J; ++j) pos[j] = slot[j] < RV_MAXC ? atomicAdd(&bcnt[lane + 32 * j], 1) : -1;
+        for (int j = 0; j < J; ++j)
+            pos[j] = slot[j] < RV_MAXC ? atomicAdd(&bcnt[(lane + 32 * j) * RV_CPAD], 1) : -1;
 #pragma unroll
         for (int j = 0; j < J; ++j)
             if (pos[j] >= 0) bucket[static_cast<size_t>(lane + 32 * j) * T + pos[j]] = t * RV_MAXC + slot[j];
@@ -400,7 +403,7 @@ __device__ __forceinline__ RvItem rv_item(int item, int per_seg, const int* pre,
     }
     it.e = lo;
     const int p = (r - pre[lo]) * 32 + lane;
-    it.valid = p < bcnt[lo];
+    it.valid = p < bcnt[lo * RV_CPAD];
     const int code = it.valid ? bucket[static_cast<size_t>(lo) * T + p] : 0;
     it.t = code / RV_MAXC;
     it.c = code % RV_MAXC;
@@ -440,7 +443,7 @@ __global__ void __launch_bounds__(RV_WARPS * 32) route_verify_kernel(const uint1
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int e = lane * 8 + j;
-            v[j] = e < E ? (bcnt[e] + 31) >> 5 : 0;
+            v[j] = e < E ? (bcnt[e * RV_CPAD] + 31) >> 5 : 0;
             sum += v[j];
         }
         int incl = sum;
@@ -645,7 +648,7 @@ size_t route_tc_scratch_bytes(int T, int H, int E) {
     if (E < 32 || E > 256 || T <= 256 || H % RV_SEG != 0 || H > 8192) return 0;
     return align256(static_cast<size_t>(2) * WS_ROWS * H * 2) + align256(256 * 4) +
            align256(static_cast<size_t>(T) * 4) + align256(static_cast<size_t>(T) * RV_MAXC * 4) +
-           align256(256 * 4) + align256(static_cast<size_t>(E) * T * 4);
+           align256(256 * RV_CPAD * 4) + align256(static_cast<size_t>(E) * T * 4);
 }
 
 cudaError_t launch_route_tc(const moe_shape& s, const void* x, const float* wr, const float* bias, int32_t* ids,
@@ -665,7 +668,7 @@ cudaError_t launch_route_tc(const moe_shape& s, const void* x, const float* wr, 
     int32_t* cand = reinterpret_cast<int32_t*>(p);
     p += align256(static_cast<size_t>(T) * RV_MAXC * 4);
     int32_t* bcnt = reinterpret_cast<int32_t*>(p);
-    p += align256(256 * 4);
+    p += align256(256 * RV_CPAD * 4);
     int32_t* bucket = reinterpret_cast<int32_t*>(p);
     // the router partials buffer ([H/256][T][E] floats) holds the approximate
     // slices first ([KS][T][E], KS <= H/256) and the candidates' exact segment
