@@ -253,8 +253,9 @@ def kernel_table(steps: int) -> dict:
 
 def token_major_gather(cfg) -> bool:
     """The layer gathers its rows token by token (bf16 tokens on the tensor-core
-    path, H <= 5120), quantising them there for E4M3 weights."""
-    return cfg.act_dtype == "bf16" and cfg.w_dtype != "f32" and cfg.H % 8 == 0 and cfg.H <= 5120
+    path, at least 1024 of them, H <= 5120), quantising them there for E4M3 weights."""
+    return (cfg.act_dtype == "bf16" and cfg.w_dtype != "f32" and cfg.T >= 1024 and cfg.H % 8 == 0
+            and cfg.H <= 5120)
 
 
 def algorithmic(cfg, kernel: str, counts: np.ndarray | None, fused: bool = True):

@@ -412,10 +412,13 @@ moe_status moe_forward(const moe_shape* shape, const void* x, const float* route
     // permutation, shared id last), so its rows need no gather
     a.direct_e = (fused && d.shared) ? d.E - 1 : -1;
     if (err == cudaSuccess) {
-        if (shape->act_dtype == MOE_BF16 && scatter_rows_supported(d.H) && ffn_takes_tc(a, ffn_impl)) {
+        if (shape->act_dtype == MOE_BF16 && d.T >= 1024 && scatter_rows_supported(d.H) &&
+            ffn_takes_tc(a, ffn_impl)) {
             // the grouped rows by token (each token's row read once, quantised
             // there for E4M3 layers) instead of quantising the tokens and then
-            // gathering row by row inside the tensor-core pass
+            // gathering row by row inside the tensor-core pass; small batches
+            // keep the row gather (a warp per token leaves too few warps:
+            // decode_bf16, 64 tokens, 25 against 11 us)
             err = launch_scatter_rows(d.T, d.S, d.R, d.H, x, at<int32_t>(ws, L.inv),
                                       a.direct_e >= 0 ? at<int32_t>(ws, L.offsets) + a.direct_e : nullptr,
                                       fp8 ? at<uint8_t>(ws, L.xq) : nullptr, fp8 ? at<float>(ws, L.xscale) : nullptr,

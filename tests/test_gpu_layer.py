@@ -29,6 +29,10 @@ SMALL = {
                                top_k=2, renormalize=False),
     "routed_scale": synth.variant(synth.CONFIGS["prefill_bf16"], T=150, H=512, I=128, n_routed=16,
                                   top_k=4, routed_scale=2.5),
+    # 1024 tokens or more: the rows are gathered token by token (and quantised
+    # there for E4M3 weights); odd token counts leave ragged groups
+    "token_gather_bf16": synth.variant(synth.CONFIGS["prefill_bf16"], T=1100, H=512, I=128, n_routed=16, top_k=4),
+    "token_gather_fp8": synth.variant(synth.CONFIGS["prefill_fp8"], T=1031, H=768, I=128, n_routed=12, top_k=3),
     "bias_select_only_fp8": synth.variant(synth.CONFIGS["skewed_fp8"], T=200, H=512, I=192, n_routed=24,
                                           top_k=4, bias_select_only=True, routed_scale=1.5),
 }
