@@ -417,8 +417,8 @@ moe_status moe_forward(const moe_shape* shape, const void* x, const float* route
             // the grouped rows by token (each token's row read once, quantised
             // there for E4M3 layers) instead of quantising the tokens and then
             // gathering row by row inside the tensor-core pass; small batches
-            // keep the row gather (a warp per token leaves too few warps:
-            // decode_bf16, 64 tokens, 25 against 11 us)
+            // keep the row gather (a few tokens leave most SMs idle:
+            // decode_bf16, 64 tokens, 25 against 11 us with a warp per token)
             err = launch_scatter_rows(d.T, d.S, d.R, d.H, x, at<int32_t>(ws, L.inv),
                                       a.direct_e >= 0 ? at<int32_t>(ws, L.offsets) + a.direct_e : nullptr,
                                       fp8 ? at<uint8_t>(ws, L.xq) : nullptr, fp8 ? at<float>(ws, L.xscale) : nullptr,

@@ -480,67 +480,78 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(int rows, int cols,
     if (lane == 0) scales[r] = rq.scale;
 }
 
-// Token-major gather of the grouped pass's rows: one warp per token t reads its
-// row once into registers (H <= kScatterMaxH bf16 values) and writes it to the
-// rows inv[t * S + k] of its slots, leaving out rows in [skip[0], skip[1]) (a
-// group the GEMM reads from the token matrix directly) and slots without a row.
-// kQuant (E4M3 layers): the row is quantised as quant_rows_kernel does it and
-// its codes and scale go to the token matrix (xq, xscale) as well as to the
-// slots' rows (xp, xpscale); otherwise the bf16 row itself is copied.
-constexpr int kScatterVec = 20;                 // 16-byte vectors per lane
-constexpr int kScatterMaxH = kScatterVec * 32 * 8;
+// Token-major gather of the grouped pass's rows: one 128-thread block per token
+// t reads its row once into registers (H <= kScatterMaxH bf16 values, a
+// quarter of the row per warp) and writes it to the rows inv[t * S + k] of its
+// slots, leaving out rows in [skip[0], skip[1]) (a group the GEMM reads from
+// the token matrix directly) and slots without a row. Four warps per token
+// keep the items small, so the grid has no tail of whole-row warps.
+// kQuant (E4M3 layers): the row is quantised as quant_rows_kernel does it (the
+// row's amax is a max, so its order does not matter) and its codes and scale go
+// to the token matrix (xq, xscale) as well as to the slots' rows (xp,
+// xpscale); otherwise the bf16 row itself is copied.
+constexpr int kScatterThreads = 128;
+constexpr int kScatterVec = 8;                  // 16-byte vectors per thread
+constexpr int kScatterMaxH = kScatterVec * kScatterThreads * 8;
 
 template <bool kQuant>
-__global__ void __launch_bounds__(256) scatter_rows_kernel(int T, int S, int R, int H,
-                                                           const uint4* __restrict__ x,
-                                                           const int32_t* __restrict__ inv,
-                                                           const int32_t* __restrict__ skip,
-                                                           uint8_t* __restrict__ xq, float* __restrict__ xscale,
-                                                           void* __restrict__ xp, float* __restrict__ xpscale) {
-    const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    if (t >= T) return;
+__global__ void __launch_bounds__(kScatterThreads) scatter_rows_kernel(int T, int S, int R, int H,
+                                                                       const uint4* __restrict__ x,
+                                                                       const int32_t* __restrict__ inv,
+                                                                       const int32_t* __restrict__ skip,
+                                                                       uint8_t* __restrict__ xq,
+                                                                       float* __restrict__ xscale,
+                                                                       void* __restrict__ xp,
+                                                                       float* __restrict__ xpscale) {
+    const int t = blockIdx.x;
+    const int i = threadIdx.x;
     const int nv = H / 8;
     uint4 v[kScatterVec];
     const uint4* src = x + static_cast<size_t>(t) * nv;
 #pragma unroll
     for (int j = 0; j < kScatterVec; ++j)
-        if (j * 32 + lane < nv) v[j] = src[j * 32 + lane];
+        if (j * kScatterThreads + i < nv) v[j] = src[j * kScatterThreads + i];
     const int s0 = skip != nullptr ? skip[0] : 0, s1 = skip != nullptr ? skip[1] : 0;
+    const int32_t* tinv = inv + static_cast<size_t>(t) * S;
     if constexpr (kQuant) {
+        __shared__ float s_amax[kScatterThreads / 32];
         float amax = 0.0f;
 #pragma unroll
         for (int j = 0; j < kScatterVec; ++j)
-            if (j * 32 + lane < nv) amax = amax_bf16x8(amax, v[j]);
+            if (j * kScatterThreads + i < nv) amax = amax_bf16x8(amax, v[j]);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+        if ((i & 31) == 0) s_amax[i >> 5] = amax;
+        __syncthreads();
+#pragma unroll
+        for (int w = 0; w < kScatterThreads / 32; ++w) amax = fmaxf(amax, s_amax[w]);
         const RowQuant rq = row_quant(amax);
         uint2 c[kScatterVec];
 #pragma unroll
         for (int j = 0; j < kScatterVec; ++j)
-            if (j * 32 + lane < nv) c[j] = codes_bf16x8(v[j], rq);
+            if (j * kScatterThreads + i < nv) c[j] = codes_bf16x8(v[j], rq);
         uint2* dq = reinterpret_cast<uint2*>(xq + static_cast<size_t>(t) * H);
 #pragma unroll
         for (int j = 0; j < kScatterVec; ++j)
-            if (j * 32 + lane < nv) dq[j * 32 + lane] = c[j];
-        if (lane == 0) xscale[t] = rq.scale;
+            if (j * kScatterThreads + i < nv) dq[j * kScatterThreads + i] = c[j];
+        if (i == 0) xscale[t] = rq.scale;
         for (int k = 0; k < S; ++k) {
-            const int r = inv[static_cast<size_t>(t) * S + k];
-            if (r < 0 || r >= R || (r >= s0 && r < s1)) continue;       // warp-uniform
+            const int r = tinv[k];
+            if (r < 0 || r >= R || (r >= s0 && r < s1)) continue;       // block-uniform
             uint2* d = reinterpret_cast<uint2*>(static_cast<uint8_t*>(xp) + static_cast<size_t>(r) * H);
 #pragma unroll
             for (int j = 0; j < kScatterVec; ++j)
-                if (j * 32 + lane < nv) d[j * 32 + lane] = c[j];
-            if (lane == 0) xpscale[r] = rq.scale;
+                if (j * kScatterThreads + i < nv) d[j * kScatterThreads + i] = c[j];
+            if (i == 0) xpscale[r] = rq.scale;
         }
     } else {
         for (int k = 0; k < S; ++k) {
-            const int r = inv[static_cast<size_t>(t) * S + k];
-            if (r < 0 || r >= R || (r >= s0 && r < s1)) continue;       // warp-uniform
+            const int r = tinv[k];
+            if (r < 0 || r >= R || (r >= s0 && r < s1)) continue;       // block-uniform
             uint4* d = static_cast<uint4*>(xp) + static_cast<size_t>(r) * nv;
 #pragma unroll
             for (int j = 0; j < kScatterVec; ++j)
-                if (j * 32 + lane < nv) d[j * 32 + lane] = v[j];
+                if (j * kScatterThreads + i < nv) d[j * kScatterThreads + i] = v[j];
         }
     }
 }
@@ -634,10 +645,10 @@ cudaError_t launch_scatter_rows(int T, int S, int R, int H, const void* x, const
     if (T == 0) return cudaSuccess;
     ProfileScope ps("gather", stream);
     if (xq != nullptr)
-        scatter_rows_kernel<true><<<ceil_div(T * 32, 256), 256, 0, stream>>>(
+        scatter_rows_kernel<true><<<T, kScatterThreads, 0, stream>>>(
             T, S, R, H, static_cast<const uint4*>(x), inv, skip, xq, xscale, xp, xpscale);
     else
-        scatter_rows_kernel<false><<<ceil_div(T * 32, 256), 256, 0, stream>>>(
+        scatter_rows_kernel<false><<<T, kScatterThreads, 0, stream>>>(
             T, S, R, H, static_cast<const uint4*>(x), inv, skip, nullptr, nullptr, xp, nullptr);
     note_launch();
     return cudaGetLastError();
