@@ -47,10 +47,6 @@ __device__ __forceinline__ float e4m3_to_f32(uint8_t c) {
     return static_cast<float>(v);
 }
 
-// round to nearest even, saturate to +-448 (cvt.rn.satfinite)
-__device__ __forceinline__ uint8_t f32_to_e4m3(float f) {
-    return static_cast<uint8_t>(__nv_cvt_float_to_fp8(f, __NV_SATFINITE, __NV_E4M3));
-}
 
 // Power-of-two exponent k for a chunk whose largest magnitude is amax, so that
 // amax * 2^-k lies in [2^14, 2^15) (fp16 keeps 11 significant bits there and

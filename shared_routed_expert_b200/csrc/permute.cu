@@ -447,16 +447,26 @@ __device__ __forceinline__ float amax_bf16x8(float amax, const uint4 q) {
     return amax;
 }
 
-// eight bf16 values -> eight E4M3 codes (in order, little-endian)
+// eight bf16 values -> eight E4M3 codes (round to nearest even, saturated to
+// +-448; in order, little-endian); kRecip:
+// the quotients by div_by_recip (rq.by_recip, decided once per row), else by
+// the IEEE divide. Two quotients go through one paired conversion (the first
+// in the low byte), the same rounding as one at a time.
+template <bool kRecip>
 __device__ __forceinline__ uint2 codes_bf16x8(const uint4 q, const RowQuant& rq) {
     const uint32_t w[4] = {q.x, q.y, q.z, q.w};
     uint32_t packed[2] = {0u, 0u};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const float a = __uint_as_float(w[j] << 16), b = __uint_as_float(w[j] & 0xFFFF0000u);
-        const uint32_t lo = f32_to_e4m3(rq.by_recip ? div_by_recip(a, rq.scale, rq.y) : __fdiv_rn(a, rq.scale));
-        const uint32_t hi = f32_to_e4m3(rq.by_recip ? div_by_recip(b, rq.scale, rq.y) : __fdiv_rn(b, rq.scale));
-        packed[j >> 1] |= (lo | (hi << 8)) << ((j & 1) * 16);
+        float2 qv;
+        if constexpr (kRecip) {
+            qv = make_float2(div_by_recip(a, rq.scale, rq.y), div_by_recip(b, rq.scale, rq.y));
+        } else {
+            qv = make_float2(__fdiv_rn(a, rq.scale), __fdiv_rn(b, rq.scale));
+        }
+        const uint32_t two = static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(qv, __NV_SATFINITE, __NV_E4M3));
+        packed[j >> 1] |= two << ((j & 1) * 16);
     }
     return make_uint2(packed[0], packed[1]);
 }
@@ -476,7 +486,11 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(int rows, int cols,
     for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
     const RowQuant rq = row_quant(amax);
     uint2* dst = reinterpret_cast<uint2*>(codes + static_cast<size_t>(r) * cols);
-    for (int i = lane; i < nv; i += 32) dst[i] = codes_bf16x8(src[i], rq);
+    if (rq.by_recip) {
+        for (int i = lane; i < nv; i += 32) dst[i] = codes_bf16x8<true>(src[i], rq);
+    } else {
+        for (int i = lane; i < nv; i += 32) dst[i] = codes_bf16x8<false>(src[i], rq);
+    }
     if (lane == 0) scales[r] = rq.scale;
 }
 
@@ -527,9 +541,15 @@ __global__ void __launch_bounds__(kScatterThreads) scatter_rows_kernel(int T, in
         for (int w = 0; w < kScatterThreads / 32; ++w) amax = fmaxf(amax, s_amax[w]);
         const RowQuant rq = row_quant(amax);
         uint2 c[kScatterVec];
+        if (rq.by_recip) {
 #pragma unroll
-        for (int j = 0; j < kScatterVec; ++j)
-            if (j * kScatterThreads + i < nv) c[j] = codes_bf16x8(v[j], rq);
+            for (int j = 0; j < kScatterVec; ++j)
+                if (j * kScatterThreads + i < nv) c[j] = codes_bf16x8<true>(v[j], rq);
+        } else {
+#pragma unroll
+            for (int j = 0; j < kScatterVec; ++j)
+                if (j * kScatterThreads + i < nv) c[j] = codes_bf16x8<false>(v[j], rq);
+        }
         uint2* dq = reinterpret_cast<uint2*>(xq + static_cast<size_t>(t) * H);
 #pragma unroll
         for (int j = 0; j < kScatterVec; ++j)
