@@ -237,11 +237,15 @@ __device__ __forceinline__ void epilogue_rows(const TcParams& p, const TileInfo&
                 float g0 = __uint_as_float(g[j]), g1 = __uint_as_float(g[j + 1]);
                 float u0 = __uint_as_float(u[j]), u1 = __uint_as_float(u[j + 1]);
                 if constexpr (kFp8) {
-                    // rows past the group end are computed too and not stored
-                    g0 = g0 * rs * sg[j];
-                    g1 = g1 * rs * sg[j + 1];
-                    u0 = u0 * rs * su[j];
-                    u1 = u1 * rs * su[j + 1];
+                    // (v * rs) * scale, two at a time; rows past the group end are
+                    // computed too and not stored
+                    const float2 rs2 = make_float2(rs, rs);
+                    const float2 gg = __fmul2_rn(__fmul2_rn(make_float2(g0, g1), rs2), make_float2(sg[j], sg[j + 1]));
+                    const float2 uu = __fmul2_rn(__fmul2_rn(make_float2(u0, u1), rs2), make_float2(su[j], su[j + 1]));
+                    g0 = gg.x;
+                    g1 = gg.y;
+                    u0 = uu.x;
+                    u1 = uu.y;
                 }
                 packed[j >> 1] = pack_bf16x2(silu_f32(g0) * u0, silu_f32(g1) * u1);
             }
@@ -254,17 +258,26 @@ __device__ __forceinline__ void epilogue_rows(const TcParams& p, const TileInfo&
             const float* sc = scs + (c - c_begin) * 32;      // this warp's staged weight scales
             float a[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                a[j] = __uint_as_float(v[j]);
-                if constexpr (kFp8) a[j] = a[j] * rs * sc[j];   // rows past the group end are not stored
+            for (int j = 0; j < 32; j += 2) {
+                float2 q = make_float2(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
+                if constexpr (kFp8) {
+                    // (a * rs) * sc per element, two at a time; rows past the group end are not stored
+                    q = __fmul2_rn(__fmul2_rn(q, make_float2(rs, rs)), make_float2(sc[j], sc[j + 1]));
+                }
+                a[j] = q.x;
+                a[j + 1] = q.y;
             }
             uint32_t packed[16];
             if (p.yexp != nullptr) {
                 const float amax = abs_max32(a);
                 const int k = f16_chunk_exp(amax);
                 const float down = exp2_int(-k);
+                const float2 down2 = make_float2(down, down);
 #pragma unroll
-                for (int j = 0; j < 32; j += 2) packed[j >> 1] = pack_f16x2(a[j] * down, a[j + 1] * down);
+                for (int j = 0; j < 32; j += 2) {
+                    const float2 q = __fmul2_rn(make_float2(a[j], a[j + 1]), down2);
+                    packed[j >> 1] = pack_f16x2(q.x, q.y);
+                }
                 exps |= static_cast<uint64_t>(static_cast<uint8_t>(static_cast<int8_t>(k))) << (8 * (c - c_begin));
             } else {
 #pragma unroll
