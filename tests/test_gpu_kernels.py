@@ -432,3 +432,50 @@ def test_grouped_ffn_ragged_group_sizes(w_dtype, impl):
     rows = [0, 1, 127, 128, 129, 255, 256, 257, 384, 385, 600, 684]
     ref = np.stack([Ly.expert_ffn(int(expert_of[r]), xs[perm[r] // cfg.slots]) for r in rows])
     assert rel_err(yg[rows], ref) <= tol_of(cfg)
+
+
+@pytest.mark.parametrize("w_dtype,inter", [("bf16", 128), ("e4m3", 128), ("e4m3", 192)],
+                         ids=["bf16", "e4m3", "e4m3_i192"])
+def test_grouped_ffn_small_groups_match_the_256_row_units(w_dtype, inter):
+    """Single-CTA 128-row units of small groups: groups of 1, 31, 32, 33, 63,
+    64 and 65 rows, and groups whose last unit holds 1, 32 or 62 rows (129,
+    160, 190), where a unit's rows fill one or two of the four TMEM lane
+    quarters. Every row is written, and is bit-identical to the 256-row units'
+    (the same M = 128 MMAs and epilogue arithmetic per 128-row tile, with two
+    tiles sharing each weight stage). Against the oracle: every row on the E4M3
+    layers; on the bf16 layer the rows the other grouped-FFN tests sample
+    (every 7th, and each group's first and last), because one row of this case
+    (row 31 of expert 8) has its largest h element within 2e-4 ulp of a bf16
+    rounding midpoint, which the kernel's fp32 SiLU and the oracle's fp64 one
+    round to different neighbours; that moves the row by 1.1e-2 of the RMS,
+    although the layer output, where a routed row carries about 1/8 of the
+    weight, stays inside its 1e-2."""
+    base = synth.CONFIGS["prefill_bf16" if w_dtype == "bf16" else "skewed_fp8"]
+    cfg = synth.variant(base, T=192, H=512, I=inter, n_routed=9, top_k=3)   # S = 4, R = 768
+    counts = np.array([1, 31, 32, 33, 63, 64, 65, 129, 160, 190], np.int32)
+    assert counts.sum() == cfg.rows and counts.size == cfg.n_experts
+    offsets = np.r_[0, np.cumsum(counts)].astype(np.int32)
+    perm = np.random.default_rng(17).permutation(cfg.rows).astype(np.int32)
+    inp = synth.make_inputs(cfg)
+    d = synth.to_device(inp, DEV)
+    s = _lib.make_shape(cfg)
+    ws = _lib.alloc_workspace(s, True)
+    ys = []
+    for impl in (MOE_FFN_TCGEN05_M128, MOE_FFN_TCGEN05_M256):
+        y = torch.full((cfg.rows, cfg.H), float("nan"), dtype=torch.bfloat16, device=DEV)
+        _lib.moe_grouped_ffn(s, d["x"], torch.from_numpy(perm).to(DEV), torch.from_numpy(offsets).to(DEV),
+                             d["w13"], d["s13"], d["w2"], d["s2"], y, ws, impl=impl)
+        assert _lib.moe_get_status(ws) == _lib.MOE_OK
+        ys.append(y)
+    assert torch.equal(ys[0], ys[1])
+    yg = to_f64(ys[0])
+    assert np.all(np.isfinite(yg))
+    Ly = oracle.Layer(cfg, inp)
+    xs = inp["x"].float().numpy()
+    expert_of = np.repeat(np.arange(cfg.n_experts), counts)
+    if w_dtype == "bf16":
+        rows = sorted(set(range(0, cfg.rows, 7)) | set(offsets[:-1].tolist()) | set((offsets[1:] - 1).tolist()))
+    else:
+        rows = list(range(cfg.rows))
+    ref = np.stack([Ly.expert_ffn(int(expert_of[r]), xs[perm[r] // cfg.slots]) for r in rows])
+    assert rel_err(yg[rows], ref) <= tol_of(cfg)
