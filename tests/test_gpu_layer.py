@@ -33,6 +33,12 @@ SMALL = {
     # there for E4M3 weights); odd token counts leave ragged groups
     "token_gather_bf16": synth.variant(synth.CONFIGS["prefill_bf16"], T=1100, H=512, I=128, n_routed=16, top_k=4),
     "token_gather_fp8": synth.variant(synth.CONFIGS["prefill_fp8"], T=1031, H=768, I=128, n_routed=12, top_k=3),
+    # the token-major gather holds rows of up to 8192 values (a quarter per warp).
+    # E4M3 weights here: with bf16 h and I this small, one h element that the
+    # kernel's fp32 SiLU and the oracle's fp64 one round to different bf16
+    # neighbours can move the output by ~1e-2 by itself (at I = 1536 it is ~3e-3)
+    "token_gather_h8192_fp8": synth.variant(synth.CONFIGS["prefill_fp8"], T=1030, H=8192, I=64, n_routed=10,
+                                            top_k=3),
     "bias_select_only_fp8": synth.variant(synth.CONFIGS["skewed_fp8"], T=200, H=512, I=192, n_routed=24,
                                           top_k=4, bias_select_only=True, routed_scale=1.5),
 }
